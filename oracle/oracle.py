@@ -1,0 +1,133 @@
+"""Python face of the CPU oracle (smc_oracle.cpp).
+
+TEST INFRASTRUCTURE ONLY: imported by the tests, the smoke check and the
+benchmark's CPU-baseline leg, never by the product path.  It shares nothing
+with the CUDA library: it compiles and loads its own C++ file with g++, takes
+numpy arrays, and computes in fp64.
+
+Functions
+---------
+neighbour_map(coords, grid, k=3)          -> int32 [N, k^3]
+pair_lists(nbr)                           -> (counts int64[T], offsets int64[T+1], in_idx, out_idx)
+conv(coords, grid, feats, weight, bias, k=3, orientation=+1, rows=None, threads=1) -> fp64 [rows, Cout]
+
+The definition each follows is cited in smc_oracle.cpp.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "smc_oracle.cpp")
+_LIB = os.path.join(_HERE, "libsmc_oracle.so")
+
+ERRORS = {-1: "bad argument", -2: "coordinate out of range", -3: "duplicate coordinate"}
+
+
+class OracleError(RuntimeError):
+    def __init__(self, code: int):
+        super().__init__(f"oracle error {code}: {ERRORS.get(code, 'unknown')}")
+        self.code = code
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into oracle/libsmc_oracle.so (g++, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["g++", "-O2", "-std=c++17", "-fopenmp", "-shared", "-fPIC",
+                               _SRC, "-o", tmp])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i64, i32 = ctypes.c_int64, ctypes.c_int32
+        lib.oracle_neighbour_map.argtypes = [P, i64, P, i32, P]
+        lib.oracle_pair_lists.argtypes = [P, i64, i32, P, P, P]
+        lib.oracle_conv.argtypes = [P, i64, P, P, i64, P, P, i64, i32, i32, P, i64, P, i32]
+        for f in (lib.oracle_neighbour_map, lib.oracle_pair_lists, lib.oracle_conv):
+            f.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _coords(coords) -> np.ndarray:
+    c = np.ascontiguousarray(coords, dtype=np.int32)
+    if c.ndim != 2 or c.shape[1] != 4:
+        raise ValueError("coords must be int32 [N, 4] (b, z, y, x)")
+    return c
+
+
+def _grid(grid: Sequence[int]) -> np.ndarray:
+    g = np.ascontiguousarray(grid, dtype=np.int32)
+    if g.shape != (3,):
+        raise ValueError("grid must be (Z, Y, X)")
+    return g
+
+
+def neighbour_map(coords, grid, k: int = 3) -> np.ndarray:
+    c, g = _coords(coords), _grid(grid)
+    n = c.shape[0]
+    nbr = np.empty((n, k ** 3), dtype=np.int32)
+    rc = _load().oracle_neighbour_map(_ptr(c), n, _ptr(g), k, _ptr(nbr))
+    if rc:
+        raise OracleError(rc)
+    return nbr
+
+
+def pair_lists(nbr: np.ndarray):
+    nbr = np.ascontiguousarray(nbr, dtype=np.int32)
+    n, taps = nbr.shape
+    counts = np.zeros(taps, dtype=np.int64)
+    lib = _load()
+    rc = lib.oracle_pair_lists(_ptr(nbr), n, taps, _ptr(counts), None, None)
+    if rc:
+        raise OracleError(rc)
+    total = int(counts.sum())
+    in_idx = np.empty(total, dtype=np.int32)
+    out_idx = np.empty(total, dtype=np.int32)
+    rc = lib.oracle_pair_lists(_ptr(nbr), n, taps, _ptr(counts), _ptr(in_idx), _ptr(out_idx))
+    if rc:
+        raise OracleError(rc)
+    offsets = np.zeros(taps + 1, dtype=np.int64)
+    np.cumsum(counts, out=offsets[1:])
+    return counts, offsets, in_idx, out_idx
+
+
+def conv(coords, grid, feats, weight, bias=None, k: int = 3, orientation: int = 1,
+         rows=None, threads: int = 1) -> np.ndarray:
+    c, g = _coords(coords), _grid(grid)
+    n = c.shape[0]
+    f = np.ascontiguousarray(feats, dtype=np.float64)
+    w = np.ascontiguousarray(weight, dtype=np.float64)
+    if f.shape[0] != n:
+        raise ValueError("feats must have one row per coordinate")
+    cin = f.shape[1]
+    cout = w.shape[0]
+    if w.shape != (cout, k, k, k, cin):
+        raise ValueError(f"weight must be KRSC [Cout, {k}, {k}, {k}, Cin={cin}], got {w.shape}")
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float64)
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    nrows = n if r is None else r.shape[0]
+    out = np.empty((nrows, cout), dtype=np.float64)
+    rc = _load().oracle_conv(_ptr(c), n, _ptr(g), _ptr(f), cin, _ptr(w), _ptr(b), cout, k,
+                             orientation, _ptr(r), nrows, _ptr(out), threads)
+    if rc:
+        raise OracleError(rc)
+    return out

@@ -1,0 +1,73 @@
+"""Planted mistakes: each is compiled into a throw-away copy of the oracle on
+the CPU, and the pins of test_oracle_pins must reject it.  This shows the pins
+are strong enough to catch the plausible slips they were chosen for."""
+import ctypes
+import os
+import subprocess
+import tempfile
+
+import numpy as np
+import pytest
+import torch
+
+from tests.test_oracle_pins import _random_case, _torch_dense_conv
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                   "oracle", "smc_oracle.cpp")
+
+MUTATIONS = {
+    "orientation_sign": ("c[1] + sign * delta[0], c[2] + sign * delta[1], c[3] + sign * delta[2]",
+                         "c[1] - sign * delta[0], c[2] - sign * delta[1], c[3] - sign * delta[2]"),
+    "axis_swap": ("delta[0] = kz - h;\n  delta[1] = ky - h;\n  delta[2] = kx - h;",
+                  "delta[0] = kx - h;\n  delta[1] = ky - h;\n  delta[2] = kz - h;"),
+    "weight_transposed": ("weight + (o * taps + d) * cin", "weight + (d * cout + o) * cin"),
+    "dropped_tap": ("const int64_t u = neighbour(index, coords + 4 * v, delta, orientation);\n      if (u < 0) continue;",
+                    "const int64_t u = neighbour(index, coords + 4 * v, delta, orientation);\n      if (u < 0 || d == 0) continue;"),
+    "batch_leak": ("Site s = {c[0], c[1] + sign", "Site s = {0, c[1] + sign"),
+    "bias_missing": ("acc[o] + (bias ? bias[o] : 0.0)", "acc[o]"),
+}
+
+
+def _build_mutant(name, tmpdir):
+    old, new = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation {name} no longer applies"
+    path = os.path.join(tmpdir, f"{name}.cpp")
+    with open(path, "w") as f:
+        f.write(src.replace(old, new))
+    lib = os.path.join(tmpdir, f"lib{name}.so")
+    subprocess.check_call(["g++", "-O1", "-std=c++17", "-shared", "-fPIC", path, "-o", lib])
+    dll = ctypes.CDLL(lib)
+    P, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    dll.oracle_conv.argtypes = [P, i64, P, P, i64, P, P, i64, i32, i32, P, i64, P, i32]
+    dll.oracle_conv.restype = ctypes.c_int
+    return dll
+
+
+def _run(dll, coords, grid, feats, w, b, k, s):
+    c = np.ascontiguousarray(coords, dtype=np.int32)
+    g = np.ascontiguousarray(grid, dtype=np.int32)
+    f = np.ascontiguousarray(feats, dtype=np.float64)
+    ww = np.ascontiguousarray(w, dtype=np.float64)
+    bb = np.ascontiguousarray(b, dtype=np.float64)
+    out = np.empty((len(c), ww.shape[0]))
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    rc = dll.oracle_conv(p(c), len(c), p(g), p(f), f.shape[1], p(ww), p(bb), ww.shape[0], k, s,
+                         None, len(c), p(out), 1)
+    assert rc == 0
+    return out
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_reject_planted_mistake(name):
+    with tempfile.TemporaryDirectory() as tmp:
+        dll = _build_mutant(name, tmp)
+        rng = np.random.default_rng(0)
+        grid, batch = (5, 6, 7), 2
+        coords, feats, w, b = _random_case(rng, grid, batch, 0.35, 3, 5)
+        caught = False
+        for s, wref in ((+1, w), (-1, w[:, ::-1, ::-1, ::-1, :])):
+            ref = _torch_dense_conv(coords, feats, wref, b, grid, batch, 3)
+            got = _run(dll, coords, grid, feats, w, b, 3, s)
+            caught |= not np.allclose(got, ref, rtol=1e-12, atol=1e-12)
+        assert caught, f"planted mistake {name!r} passed the dense-equivalence pin"
