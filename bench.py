@@ -1,0 +1,429 @@
+#!/usr/bin/env python
+"""Benchmark of the submanifold-convolution hot path on B200.
+
+One *step* is one pass of the whole path over one synthetic batch: build the
+neighbour map of the coordinate set (key generation and validation, hash
+build, 27-lookup map, per-offset pair lists, tile schedule) and run the k=3
+bf16 convolution over it (the map would then be reused by further layers).
+The default workload is the pages' benchmark shape: batch 1, 128^3 grid,
+128 -> 128 channels, bf16 with fp32 accumulation, union of 6 random sphere
+shells (seeded synthetic data; no dataset is involved).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  ``value`` is active voxels per second of the
+whole step (device-timed with CUDA events, L2 flushed before every step,
+max over ranks); the line also carries the conv's pair-TFLOP/s, the map
+build's GB/s, the roofline of the dominant kernel, an end-to-end figure
+through the public API with host buffers, the CPU oracle's throughput on a
+bounded sample, and the SM clocks seen during the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from submanifold_sparse_convolution_packed_b200 import synth as S  # noqa: E402
+
+METRIC = "SubMConv3d k=3 Mvoxels/s & pair-TFLOP/s @128^3/128ch bf16; map-build GB/s"
+UNIT = "Mvoxels/s"
+L2_FLUSH_BYTES = 256 << 20
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+CONV_SRC = os.path.join(ROOT, "submanifold_sparse_convolution_packed_b200", "csrc", "conv_tc.cu")
+
+
+# ---------------------------------------------------------------- helpers
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def init_dist(world: int, backend: str, timeout_s: float = 120.0):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return dist
+
+
+def reduce_max(x: float, world: int, device=None) -> float:
+    """Max of a float over ranks (identity on one rank)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def source_sha(path: str) -> str:
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        import torch
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.id = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            self.id = str(device_index)
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{device_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.id}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, val in zip(names, r[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "samples": len(rows),
+                "reasons": sorted(reasons)}
+
+
+def tap_efficiency(perm: np.ndarray, nbr: np.ndarray, tile: int = 128) -> float:
+    """Pairs / (taps issued x 128) of the tensor-core conv's tile schedule."""
+    n = len(perm)
+    hits = (nbr >= 0)
+    pairs = int(hits.sum())
+    issued = 0
+    for t0 in range(0, n, tile):
+        issued += int(hits[perm[t0:t0 + tile]].any(axis=0).sum()) * tile
+    return pairs / issued if issued else 0.0
+
+
+# ------------------------------------------------------------- workloads
+def get_workload(name: str) -> S.Workload:
+    return S.workload(name)
+
+
+def algorithmic_map_bytes(n: int, p: int) -> int:
+    """coords read (16 B) + map written (108 B) per voxel + pairs written (8 B)."""
+    return 16 * n + 108 * n + 8 * p
+
+
+def pair_flops(p: int, cin: int, cout: int) -> float:
+    return 2.0 * p * cin * cout
+
+
+# ------------------------------------------------------------- GPU arm
+def run_gpu(args):
+    import torch
+
+    import submanifold_sparse_convolution_packed_b200 as smc
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    smc.lib()
+    peaks = load_peaks()
+
+    w = get_workload(args.workload)
+    f, wt, b = S.layer_tensors(w, "bf16")
+    coords_d = torch.from_numpy(w.coords).to(dev)
+    feats_d = torch.from_numpy(f).to(torch.bfloat16).to(dev)
+    w_d = torch.from_numpy(wt).to(torch.bfloat16).to(dev)
+    b_d = torch.from_numpy(b).to(torch.bfloat16).to(dev)
+    out_d = torch.empty((w.n, w.cout), dtype=torch.bfloat16, device=dev)
+    batch = int(w.coords[:, 0].max()) + 1
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    smc.set_profiling(True)
+    launches0 = smc.kernel_launches()
+
+    def step(times, conv_times, map_times):
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        m = smc.build_map(coords_d, w.grid, batch=batch, stream=stream)
+        e1.record(stream)
+        smc.conv(m, feats_d, w_d, b_d, ksize=3, orientation=1, out=out_d, stream=stream)
+        e2.record(stream)
+        e2.synchronize()
+        times.append(e0.elapsed_time(e2))
+        conv_times.append(e1.elapsed_time(e2))
+        map_times.append(m.timing())
+        return m
+
+    # warm-up
+    for _ in range(args.warmup):
+        flush.zero_()
+        step([], [], []).free()
+    smc.status(stream)
+    # reference of the schedule quality (host-side, untimed)
+    m0 = smc.build_map(coords_d, w.grid, batch=batch, stream=stream)
+    P = m0.pairs_total
+    eff = tap_efficiency(m0.schedule().cpu().numpy(), m0.nbr().cpu().numpy())
+    m0.free()
+
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    t_wall0 = time.perf_counter()
+    times, conv_times, map_times = [], [], []
+    launches_before = smc.kernel_launches()
+    for _ in range(args.steps):
+        flush.zero_()
+        step(times, conv_times, map_times).free()
+    torch.cuda.synchronize()
+    launches = smc.kernel_launches() - launches_before
+    wall = time.perf_counter() - t_wall0
+    clk = clocks.stop()
+    barrier(world)
+    smc.status(stream)
+
+    total_ms = reduce_max(sum(times), world, dev)
+    conv_ms = reduce_max(sum(conv_times) / len(conv_times), world, dev)
+    mapk_ms = reduce_max(sum(t[0] for t in map_times) / len(map_times), world, dev)
+    sched_ms = reduce_max(sum(t[1] for t in map_times) / len(map_times), world, dev)
+    ms_per_step = total_ms / args.steps
+    value = world * w.n * args.steps / (total_ms * 1e-3) / 1e6
+    flops = pair_flops(P, w.cin, w.cout)
+    conv_tflops = flops / (conv_ms * 1e-3) / 1e12
+    map_bytes = algorithmic_map_bytes(w.n, P)
+    map_gbs = map_bytes / (mapk_ms * 1e-3) / 1e9
+
+    # traffic of the conv kernel from the committed ncu capture, if still current
+    traffic = None
+    if os.path.exists(PROFILE_TRAFFIC):
+        with open(PROFILE_TRAFFIC) as fh:
+            tr = json.load(fh).get("conv_tc", {})
+        if tr.get("source_sha") == source_sha(CONV_SRC) and tr.get("workload") == w.name:
+            traffic = tr.get("dram_bytes_per_launch")
+
+    # end to end through the public API: pinned host inputs in, result out
+    e2e = run_e2e(w, f, wt, b, batch, dev, stream, args)
+    e2e_v = reduce_max(e2e["ms"], world, dev)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        cpu = run_cpu_baseline(w, f, wt, b, budget_s=args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded union of 6 sphere shells; random-init KRSC weights)",
+            "config": {
+                "workload": f"{w.name}: {w.note}", "n_voxels": w.n, "pairs": P, "grid": list(w.grid),
+                "cin": w.cin, "cout": w.cout, "step": "build_map + conv k=3 s=+1 (map freed after)",
+                "l2": "flushed before every step (256 MB write, outside the timed events)",
+                "parallelism": f"replicas x{world} (no collective on the data path)",
+            },
+            "pair_tflops": round(conv_tflops, 2),
+            "map_build_gbs": round(map_gbs, 1),
+            "breakdown_ms": {"step": round(ms_per_step, 4), "map_kernels": round(mapk_ms, 4),
+                             "tile_schedule": round(sched_ms, 4), "conv": round(conv_ms, 4)},
+            "conv_mvoxels_per_s": round(w.n / (conv_ms * 1e-3) / 1e6, 2),
+            "conv_tap_efficiency": round(eff, 4),
+            "roofline": {"kernel": "k_conv_tc", "bound": "tensor", "achieved": round(conv_tflops, 2),
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": round(conv_tflops / peaks["bf16_tflops"], 4), "traffic": traffic,
+                         "peak_source": f"{peaks['source']} bf16 burst (kernel timed alone)",
+                         "algorithmic": "2 * pairs * Cin * Cout per launch"},
+            "map_roofline": {"kernels": "k_insert..k_pairs", "bound": "hbm", "achieved": round(map_gbs, 1),
+                             "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": round(map_gbs / peaks["hbm_gbs"], 4),
+                             "algorithmic": "16N coords + 108N map + 8P pairs"},
+            "e2e": {"value": round(world * w.n / (e2e_v * 1e-3) / 1e6, 3), "unit": UNIT,
+                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                    "ms_per_step": round(e2e_v, 4)},
+            "gpu_launches": int(launches),
+            "launches_per_step": launches / args.steps,
+            "wall_s": round(wall, 3),
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        if clk is not None:
+            line["clocks"] = clk
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(w, f, wt, b, batch, dev, stream, args):
+    """Same step through the public API, with the step's inputs copied from
+    pinned host memory and the result copied back inside the timed region."""
+    import torch
+
+    import submanifold_sparse_convolution_packed_b200 as smc
+    coords_h = torch.from_numpy(w.coords).pin_memory()
+    feats_h = torch.from_numpy(f).to(torch.bfloat16).pin_memory()
+    w_h = torch.from_numpy(wt).to(torch.bfloat16).pin_memory()
+    b_h = torch.from_numpy(b).to(torch.bfloat16).pin_memory()
+    out_h = torch.empty((w.n, w.cout), dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (coords_h, feats_h, w_h, b_h))
+    d2h = out_h.numel() * out_h.element_size()
+    times = []
+    n = max(3, min(args.steps, 50))
+    for i in range(n + 3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        c = coords_h.to(dev, non_blocking=True)
+        x = feats_h.to(dev, non_blocking=True)
+        ww = w_h.to(dev, non_blocking=True)
+        bb = b_h.to(dev, non_blocking=True)
+        m = smc.build_map(c, w.grid, batch=batch, stream=stream)
+        y = smc.conv(m, x, ww, bb, ksize=3, orientation=1, stream=stream)
+        out_h.copy_(y, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        m.free()
+        if i >= 3:
+            times.append(e0.elapsed_time(e1))
+    return {"ms": sum(times) / len(times), "h2d": h2d, "d2h": d2h}
+
+
+# ------------------------------------------------------------- CPU oracle
+def run_cpu_baseline(w, f, wt, b, budget_s: float = 20.0):
+    """The CPU oracle, as it stands, on a bounded sample of the same workload:
+    the full neighbour map plus the conv on a seeded sample of output rows;
+    throughput = voxels per second of (map cost per voxel + conv cost per row)."""
+    from oracle import oracle
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    oracle.neighbour_map(w.coords, w.grid)
+    t_map = time.perf_counter() - t0
+    rows_n = min(w.n, 2048)
+    rng = np.random.default_rng(0)
+    t_conv, done = 0.0, 0
+    while t_conv < budget_s * 0.5 and done < w.n:
+        rows = np.sort(rng.choice(w.n, size=rows_n, replace=False))
+        t1 = time.perf_counter()
+        oracle.conv(w.coords, w.grid, f, wt, b, 3, 1, rows=rows, threads=threads)
+        t_conv += time.perf_counter() - t1
+        done += rows_n
+    per_voxel = t_map / w.n + t_conv / done
+    return {"value": round(1.0 / per_voxel / 1e6, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"map over all {w.n} voxels ({t_map:.2f} s) + fp64 conv on {done} seeded rows "
+                      f"({t_conv:.2f} s, {threads} threads), per-voxel cost scaled to the metric"}
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle timed on the host cores (the pages
+    ship no runnable implementation of this path); rank 0 only.  Each step is
+    a bounded sample (full map + conv on seeded rows), sized so that the whole
+    run stays within a few minutes; steps that would not fit are not run and
+    the line reports the steps actually timed."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    w = get_workload(args.workload)
+    f, wt, b = S.layer_tensors(w, "bf16")
+    per_step = max(1.0, min(args.cpu_seconds, 150.0 / (args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        run_cpu_baseline(w, f, wt, b, budget_s=min(per_step, 2.0))
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(run_cpu_baseline(w, f, wt, b, budget_s=per_step))
+        if time.perf_counter() - t0 > 180.0:
+            break
+    elapsed = time.perf_counter() - t0
+    value = statistics.median(v["value"] for v in vals)
+    ms = w.n / (value * 1e6) * 1e3
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": len(vals),
+        "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": f"{w.name}: {w.note}", "n_voxels": w.n},
+        "cpu_baseline": vals[-1],
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": round(elapsed, 2),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1500)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="shells6",
+                    help="shells6 (default), full128, varlen4, shell2, decoder0..decoder3")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--skip-cpu", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

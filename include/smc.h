@@ -1,0 +1,172 @@
+/*
+ * smc.h -- C ABI of the B200 submanifold sparse convolution library (libsmc.so).
+ *
+ * The operation (LATO.2 MLX port README, summary and "The scope, once
+ * measured"; Pixal3D working notes, "Measured facts"): a submanifold 3x3x3
+ * convolution, stride 1, no padding (spconv's SubMConv3d).  Outputs exist only
+ * at the input's active voxels:
+ *
+ *     out[v] = bias + sum_{d=0}^{26} feats[nbr(v, d)] @ W[:, d, :]^T
+ *
+ * where nbr(v, d) is the active voxel at coordinate c_v + s*delta_d (missing
+ * or out-of-grid neighbours contribute nothing), delta_d = (kz-1, ky-1, kx-1)
+ * with d = 9*kz + 3*ky + kx, and W is in spconv's KRSC layout
+ * [Cout, kz, ky, kx, Cin] (LATO.2 README summary; Pixal3D commit log,
+ * converter paragraph).  The neighbour lookup is an "indice map" built once
+ * per coordinate set and reused by every conv on it, the way spconv's
+ * indice_key caches it (LATO.2 README summary).  s is the kernel orientation:
+ * +1 gathers feats[c+d] (cross-correlation), -1 gathers feats[c-d]; the
+ * README's "Correctness" section flags this choice as silent when wrong, so
+ * both are offered.  k = 1 is the centre tap alone, a per-voxel linear layer
+ * (LATO.2 README, "Status").
+ *
+ * Conventions for every entry point
+ *  - Pointers marked "device" are CUDA device pointers on the current device;
+ *    "host" pointers are ordinary host memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *  - Return value: SMC_OK (0) or a negative SMC_E_* code.  Nothing traps,
+ *    aborts or hangs: device-side problems are recorded in an error word and
+ *    surface as a return code.  A CUDA error from an earlier asynchronous
+ *    launch surfaces at the next call as SMC_E_CUDA.
+ *  - The caller owns every buffer it passes in; the library owns the map.
+ */
+#ifndef SMC_H_
+#define SMC_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SMC_API __attribute__((visibility("default")))
+#else
+#define SMC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque neighbour-map handle: library-owned, immutable after build. */
+typedef struct smc_map smc_map;
+
+/* Storage type of feats, weight, bias and out in smc_conv. */
+typedef enum { SMC_F32 = 0, SMC_BF16 = 1, SMC_F16 = 2 } smc_dtype;
+
+enum {
+  SMC_OK = 0,
+  SMC_E_ARG = -1,       /* null pointer, negative size, bad ksize/orientation/dtype value */
+  SMC_E_RANGE = -2,     /* a coordinate outside [0,batch) x [0,Z) x [0,Y) x [0,X) */
+  SMC_E_DUPLICATE = -3, /* the same (b,z,y,x) appears twice */
+  SMC_E_DTYPE = -4,     /* unsupported dtype for this call */
+  SMC_E_SHAPE = -5,     /* channel count or N does not match the map / limits */
+  SMC_E_ALIAS = -6,     /* out overlaps feats, weight or bias */
+  SMC_E_CAPACITY = -7,  /* hash table full after a bounded probe sequence */
+  SMC_E_OOM = -8,       /* device allocation failed */
+  SMC_E_CUDA = -9,      /* a CUDA runtime error (launch, copy, earlier async fault) */
+  SMC_E_TIMEOUT = -10,  /* a bounded device-side wait ran out; results are invalid */
+  SMC_E_ALIGN = -11     /* a device pointer lacks the alignment stated below */
+};
+
+/*
+ * smc_build_map -- build the neighbour map of one coordinate set.
+ *
+ * coords : device, int32 [n, 4], rows (b, z, y, x), contiguous, 16-byte aligned.
+ *          Row order is arbitrary; row v of the map corresponds to row v here.
+ * n      : number of active voxels (n >= 0; n == 0 gives an empty map).
+ * batch  : number of batch items; every b must lie in [0, batch).
+ * grid   : host, int32 [3] = (Z, Y, X); every coordinate must lie inside.
+ *          batch * Z * Y * X must be below 2^62.
+ * stream : work is enqueued on it; the call synchronises it once, at the end,
+ *          to read the per-offset counts and the error word.
+ * out    : receives the handle; left NULL on failure.
+ *
+ * Builds, on the device: 64-bit site keys, an open-addressing hash table of
+ * the sites, the int32 [n, 27] neighbour map (-1 = absent), the per-offset
+ * pair lists (stable compaction of each map column, ascending output row),
+ * and the tile schedule used by the tensor-core conv.  coords may be freed
+ * once the call returns.  Errors: SMC_E_ARG, SMC_E_ALIGN, SMC_E_RANGE,
+ * SMC_E_DUPLICATE, SMC_E_CAPACITY, SMC_E_OOM, SMC_E_CUDA.
+ */
+SMC_API int smc_build_map(const int32_t* coords, int64_t n, int32_t batch, const int32_t grid[3],
+                  void* stream, smc_map** out);
+
+/*
+ * smc_conv -- one submanifold convolution over a built map.
+ *
+ * feats  : device, [n, cin] row-major, dtype `dtype`.
+ * weight : device, KRSC [cout, k, k, k, cin] row-major, dtype `dtype`.
+ * bias   : device, [cout], dtype `dtype`, or NULL for no bias.
+ * out    : device, [n, cout] row-major, dtype `dtype`; fully overwritten.
+ *          Must not overlap feats, weight or bias.
+ * ksize  : 3 (27 taps through the map) or 1 (centre tap only; the map is used
+ *          only for n).
+ * orientation : +1 gathers feats[c+d], -1 gathers feats[c-d]; ignored for k=1.
+ * dtype  : SMC_F32 (exact fp32 FMA accumulation, no TF32), SMC_BF16 or
+ *          SMC_F16 (fp32 accumulation, bias added in fp32, output rounded to
+ *          nearest even).
+ *
+ * Asynchronous on `stream`; no synchronisation.  bf16/fp16 with cin a
+ * multiple of 16 and at least 64, cout a multiple of 16 and 16-byte aligned
+ * buffers run on the tcgen05 tensor-core kernel; every other shape runs on
+ * the FMA kernel.  A bounded device-side wait that runs out is reported by
+ * smc_status as SMC_E_TIMEOUT.
+ * Errors: SMC_E_ARG, SMC_E_SHAPE (cin, cout < 1), SMC_E_ALIAS, SMC_E_DTYPE,
+ * SMC_E_CUDA.
+ */
+SMC_API int smc_conv(const smc_map* map, const void* feats, int64_t cin, const void* weight,
+             const void* bias, void* out, int64_t cout, int32_t ksize, int32_t orientation,
+             int32_t dtype, void* stream);
+
+/* n and the per-offset pair counts counts[27] (host) of a map. */
+SMC_API int smc_map_info(const smc_map* map, int64_t* n, int64_t counts[27]);
+
+/* Device pointer to the int32 [n, 27] neighbour map (-1 = absent). */
+SMC_API int smc_map_nbr(const smc_map* map, const int32_t** nbr);
+
+/*
+ * Per-offset pair lists: device pointers in_idx[P], out_idx[P] (int32) and
+ * host offsets[28] (int64, offsets[0] = 0, offsets[27] = P).  Pairs of offset
+ * d occupy [offsets[d], offsets[d+1]) in ascending out_idx:
+ * (in_idx, out_idx) = (nbr[v][d], v) for every v with nbr[v][d] >= 0.
+ */
+SMC_API int smc_map_pairs(const smc_map* map, const int32_t** in_idx, const int32_t** out_idx,
+                  int64_t offsets[28]);
+
+/*
+ * Tile schedule of the tensor-core conv: device pointer to perm[n] (int32),
+ * the order in which output rows are grouped into tiles of 128 (a
+ * permutation of 0..n-1: rows with similar neighbour sets are adjacent, so
+ * each tile skips the offsets none of its rows has).
+ */
+SMC_API int smc_map_schedule(const smc_map* map, const int32_t** perm);
+
+/* Release a map.  Work on other streams that reads it must have completed. */
+SMC_API int smc_free_map(smc_map* map);
+
+/* Synchronise `stream`, then return and clear the device-side error word
+ * (SMC_E_TIMEOUT if a bounded wait in a conv kernel ran out), or SMC_OK. */
+SMC_API int smc_status(void* stream);
+
+/* Static description of an error code. */
+SMC_API const char* smc_strerror(int code);
+
+/*
+ * Test and measurement hooks.
+ * smc_set_hash_capacity: force the hash table to `slots` entries (rounded up
+ *   to a power of two, minimum 16) for later builds; 0 restores automatic
+ *   sizing (2^ceil(log2(2n))).  Used to exercise SMC_E_CAPACITY.
+ * smc_set_profiling: when on, smc_build_map records CUDA events on its stream
+ *   around its kernels; smc_map_timing then returns, in milliseconds,
+ *   ms[0] = hash insert + neighbour map + pair lists, ms[1] = tile schedule.
+ * smc_kernel_launches: number of CUDA kernels this library has launched in
+ *   the process so far (memsets and copies excluded).
+ */
+SMC_API int smc_set_hash_capacity(int64_t slots);
+SMC_API int smc_set_profiling(int32_t on);
+SMC_API int smc_map_timing(const smc_map* map, float ms[2]);
+SMC_API int smc_kernel_launches(int64_t* count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SMC_H_ */

@@ -1,0 +1,15 @@
+"""B200-native submanifold sparse convolution (SubMConv3d, stride 1).
+
+The computation lives in libsmc.so (hand-written sm_100a CUDA kernels behind
+the C ABI of include/smc.h); this package is its thin Python binding plus the
+seeded synthetic-workload generators (``synth``).
+
+    from submanifold_sparse_convolution_packed_b200 import build_map, conv
+    m = build_map(coords_int32_Nx4_cuda, grid=(Z, Y, X), key="level0")
+    out = conv(m, feats, weight_krsc, bias, ksize=3, orientation=+1)
+"""
+from ._binding import (  # noqa: F401
+    EXPORTS, LIB_PATH, Map, SmcError, build_map, clear_cache, conv, kernel_launches, lib,
+    set_hash_capacity,
+    set_profiling, status,
+)

@@ -1,0 +1,253 @@
+"""ctypes binding of libsmc.so (include/smc.h): argument marshalling only.
+
+Every step of the computation runs in the library's CUDA kernels; this module
+checks tensor dtypes and shapes, passes raw device pointers and the current
+CUDA stream, and turns negative return codes into ``SmcError``.  If the
+library has not been built, every call raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Hashable, Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsmc.so")
+
+SMC_F32, SMC_BF16, SMC_F16 = 0, 1, 2
+_DTYPES = {torch.float32: SMC_F32, torch.bfloat16: SMC_BF16, torch.float16: SMC_F16}
+
+ERROR_NAMES = {
+    -1: "SMC_E_ARG", -2: "SMC_E_RANGE", -3: "SMC_E_DUPLICATE", -4: "SMC_E_DTYPE",
+    -5: "SMC_E_SHAPE", -6: "SMC_E_ALIAS", -7: "SMC_E_CAPACITY", -8: "SMC_E_OOM",
+    -9: "SMC_E_CUDA", -10: "SMC_E_TIMEOUT", -11: "SMC_E_ALIGN",
+}
+
+EXPORTS = [
+    "smc_build_map", "smc_conv", "smc_map_info", "smc_map_nbr", "smc_map_pairs",
+    "smc_map_schedule", "smc_free_map", "smc_status", "smc_strerror",
+    "smc_set_hash_capacity", "smc_set_profiling", "smc_map_timing", "smc_kernel_launches",
+]
+
+
+class SmcError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        msg = lib().smc_strerror(code).decode() if _lib is not None else "error"
+        super().__init__(f"{what}: {ERROR_NAMES.get(code, code)} ({msg})")
+        self.code = code
+        self.name = ERROR_NAMES.get(code, str(code))
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libsmc.so.  Raises if it was not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m submanifold_sparse_convolution_packed_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+        L.smc_build_map.argtypes = [P, i64, i32, P, P, ctypes.POINTER(P)]
+        L.smc_conv.argtypes = [P, P, i64, P, P, P, i64, i32, i32, i32, P]
+        L.smc_map_info.argtypes = [P, P, P]
+        L.smc_map_nbr.argtypes = [P, ctypes.POINTER(P)]
+        L.smc_map_pairs.argtypes = [P, ctypes.POINTER(P), ctypes.POINTER(P), P]
+        L.smc_map_schedule.argtypes = [P, ctypes.POINTER(P)]
+        L.smc_free_map.argtypes = [P]
+        L.smc_status.argtypes = [P]
+        L.smc_strerror.argtypes = [ctypes.c_int]
+        L.smc_strerror.restype = ctypes.c_char_p
+        L.smc_set_hash_capacity.argtypes = [i64]
+        L.smc_set_profiling.argtypes = [i32]
+        L.smc_map_timing.argtypes = [P, P]
+        L.smc_kernel_launches.argtypes = [P]
+        for name in EXPORTS:
+            if name != "smc_strerror":
+                getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(code: int, what: str) -> None:
+    if code != 0:
+        raise SmcError(code, what)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[ctypes.c_void_p]:
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+class _DeviceView:
+    """__cuda_array_interface__ over library-owned memory (kept alive by `owner`)."""
+
+    def __init__(self, ptr: int, shape, typestr: str, owner):
+        self.owner = owner
+        self.__cuda_array_interface__ = {
+            "shape": tuple(shape), "typestr": typestr, "data": (ptr, False), "version": 3,
+            "strides": None, "stream": None,
+        }
+
+
+class Map:
+    """A built neighbour map (library-owned device buffers)."""
+
+    def __init__(self, handle: ctypes.c_void_p, n: int, batch: int, grid: Sequence[int], device):
+        self._h = handle
+        self.n = n
+        self.batch = batch
+        self.grid = tuple(int(g) for g in grid)
+        self.device = device
+        counts = (ctypes.c_int64 * 27)()
+        _check(lib().smc_map_info(self._h, None, counts), "smc_map_info")
+        self.counts = [int(c) for c in counts]
+        offs = (ctypes.c_int64 * 28)()
+        _check(lib().smc_map_pairs(self._h, None, None, offs), "smc_map_pairs")
+        self.offsets = [int(o) for o in offs]
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        if self._h is None:
+            raise RuntimeError("map already freed")
+        return self._h
+
+    @property
+    def pairs_total(self) -> int:
+        return self.offsets[-1]
+
+    def _view(self, ptr: int, shape, typestr="<i4") -> torch.Tensor:
+        if self.n == 0 or ptr is None:
+            return torch.empty(shape, dtype=torch.int32, device=self.device)
+        return torch.as_tensor(_DeviceView(ptr, shape, typestr, self), device=self.device)
+
+    def nbr(self) -> torch.Tensor:
+        """int32 [n, 27] device view of the neighbour map (-1 = absent)."""
+        p = ctypes.c_void_p()
+        _check(lib().smc_map_nbr(self.handle, ctypes.byref(p)), "smc_map_nbr")
+        return self._view(p.value, (self.n, 27))
+
+    def pairs(self):
+        """(in_idx, out_idx, offsets): int32 [P] device views and the 28 offsets."""
+        pi, po = ctypes.c_void_p(), ctypes.c_void_p()
+        _check(lib().smc_map_pairs(self.handle, ctypes.byref(pi), ctypes.byref(po), None), "smc_map_pairs")
+        P = self.pairs_total
+        return self._view(pi.value, (P,)), self._view(po.value, (P,)), list(self.offsets)
+
+    def schedule(self) -> torch.Tensor:
+        """int32 [n] device view of the tile order of the tensor-core conv."""
+        p = ctypes.c_void_p()
+        _check(lib().smc_map_schedule(self.handle, ctypes.byref(p)), "smc_map_schedule")
+        return self._view(p.value, (self.n,))
+
+    def timing(self):
+        ms = (ctypes.c_float * 2)()
+        _check(lib().smc_map_timing(self.handle, ms), "smc_map_timing")
+        return float(ms[0]), float(ms[1])
+
+    def free(self) -> None:
+        if self._h is not None:
+            _check(lib().smc_free_map(self._h), "smc_free_map")
+            self._h = None
+
+    def __del__(self):
+        try:
+            if self._h is not None and _lib is not None:
+                _lib.smc_free_map(self._h)
+                self._h = None
+        except Exception:
+            pass
+
+
+_cache: Dict[Hashable, Map] = {}
+
+
+def build_map(coords: torch.Tensor, grid: Sequence[int], batch: Optional[int] = None,
+              key: Optional[Hashable] = None, stream=None) -> Map:
+    """Build (or fetch from the cache under `key`) the map of int32 [N, 4]
+    (b, z, y, x) coordinates on a (Z, Y, X) grid.  Like spconv's indice_key,
+    `key` names a coordinate set so every conv on it reuses one map."""
+    if key is not None and key in _cache:
+        return _cache[key]
+    if coords.dtype != torch.int32 or coords.dim() != 2 or coords.shape[1] != 4:
+        raise ValueError("coords must be int32 [N, 4]")
+    if not coords.is_cuda:
+        raise ValueError("coords must be a CUDA tensor")
+    coords = coords.contiguous()
+    n = coords.shape[0]
+    if batch is None:
+        batch = int(coords[:, 0].max().item()) + 1 if n else 1
+    g = (ctypes.c_int32 * 3)(*[int(x) for x in grid])
+    h = ctypes.c_void_p()
+    with torch.cuda.device(coords.device):
+        _check(lib().smc_build_map(_ptr(coords), n, int(batch), g, _stream(stream), ctypes.byref(h)),
+               "smc_build_map")
+    m = Map(h, n, int(batch), grid, coords.device)
+    if key is not None:
+        _cache[key] = m
+    return m
+
+
+def clear_cache() -> None:
+    for m in _cache.values():
+        m.free()
+    _cache.clear()
+
+
+def conv(m: Map, feats: torch.Tensor, weight: torch.Tensor, bias: Optional[torch.Tensor] = None,
+         ksize: int = 3, orientation: int = 1, out: Optional[torch.Tensor] = None,
+         stream=None) -> torch.Tensor:
+    """Submanifold conv over map `m`: feats [N, Cin], KRSC weight [Cout, k, k, k, Cin]."""
+    if feats.dtype not in _DTYPES:
+        raise TypeError(f"unsupported dtype {feats.dtype}")
+    if weight.dtype != feats.dtype or (bias is not None and bias.dtype != feats.dtype):
+        raise TypeError("feats, weight and bias must share one dtype")
+    if feats.dim() != 2 or feats.shape[0] != m.n:
+        raise ValueError(f"feats must be [N={m.n}, Cin]")
+    cin = feats.shape[1]
+    cout = weight.shape[0]
+    if tuple(weight.shape) != (cout, ksize, ksize, ksize, cin):
+        raise ValueError(f"weight must be KRSC [Cout, {ksize}, {ksize}, {ksize}, {cin}]")
+    if bias is not None and tuple(bias.shape) != (cout,):
+        raise ValueError("bias must be [Cout]")
+    feats = feats.contiguous()
+    weight = weight.contiguous()
+    bias = None if bias is None else bias.contiguous()
+    if out is None:
+        out = torch.empty((m.n, cout), dtype=feats.dtype, device=feats.device)
+    elif out.shape != (m.n, cout) or out.dtype != feats.dtype or not out.is_contiguous():
+        raise ValueError("out must be a contiguous [N, Cout] tensor of the feats dtype")
+    with torch.cuda.device(feats.device):
+        _check(lib().smc_conv(m.handle, _ptr(feats), cin, _ptr(weight), _ptr(bias), _ptr(out), cout,
+                              ksize, orientation, _DTYPES[feats.dtype], _stream(stream)), "smc_conv")
+    return out
+
+
+def status(stream=None) -> None:
+    """Synchronise the stream and raise if a conv kernel reported a timeout."""
+    _check(lib().smc_status(_stream(stream)), "smc_status")
+
+
+def set_hash_capacity(slots: int) -> None:
+    _check(lib().smc_set_hash_capacity(int(slots)), "smc_set_hash_capacity")
+
+
+def kernel_launches() -> int:
+    """Kernels launched by libsmc in this process so far."""
+    c = ctypes.c_int64()
+    _check(lib().smc_kernel_launches(ctypes.byref(c)), "smc_kernel_launches")
+    return int(c.value)
+
+
+def set_profiling(on: bool) -> None:
+    _check(lib().smc_set_profiling(1 if on else 0), "smc_set_profiling")

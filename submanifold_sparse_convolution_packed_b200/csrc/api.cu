@@ -1,0 +1,402 @@
+// Host side of libsmc: the C ABI declared in include/smc.h.
+//
+// Owns the neighbour-map handle (device buffers allocated stream-ordered on
+// the build stream), validates every argument before anything is launched,
+// picks the conv kernel, and turns device error bits into SMC_E_* codes.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "../../include/smc.h"
+#include "common.cuh"
+#include "kernels.h"
+
+struct smc_map {
+  int device;
+  cudaStream_t stream;
+  int64_t n;
+  int32_t batch;
+  int32_t grid[3];
+  int64_t counts[27];
+  int64_t offsets[28];
+  int32_t* nbr;
+  int32_t* in_idx;
+  int32_t* out_idx;
+  int32_t* perm;
+  void* keep;  // one allocation holding nbr, pairs and perm
+  float ms[2];
+};
+
+namespace {
+
+std::atomic<int64_t> g_capacity_override{0};
+std::atomic<long long> g_launches{0};
+std::atomic<int32_t> g_profiling{0};
+
+// Per-device error word of the conv kernels (bounded-wait timeouts).
+constexpr int kMaxDevices = 64;
+uint32_t* g_status[kMaxDevices] = {};
+std::mutex g_status_mu;
+
+uint32_t* device_status(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  if (!g_status[dev]) {
+    void* p = nullptr;
+    if (cudaMalloc(&p, 256) != cudaSuccess) return nullptr;
+    if (cudaMemset(p, 0, 256) != cudaSuccess) return nullptr;
+    g_status[dev] = static_cast<uint32_t*>(p);
+  }
+  return g_status[dev];
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Bump allocator over one device allocation.
+struct Carve {
+  size_t off = 0;
+  template <typename T>
+  size_t take(size_t count) {
+    const size_t o = align_up(off, 256);
+    off = o + count * sizeof(T);
+    return o;
+  }
+};
+
+int pending_cuda_error() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SMC_OK : SMC_E_CUDA;
+}
+
+bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+}  // namespace
+
+namespace smc {
+void count_launches(int k) { g_launches.fetch_add(k, std::memory_order_relaxed); }
+}  // namespace smc
+
+extern "C" {
+
+const char* smc_strerror(int code) {
+  switch (code) {
+    case SMC_OK: return "ok";
+    case SMC_E_ARG: return "invalid argument";
+    case SMC_E_RANGE: return "coordinate outside the grid or batch range";
+    case SMC_E_DUPLICATE: return "duplicate coordinate";
+    case SMC_E_DTYPE: return "unsupported dtype";
+    case SMC_E_SHAPE: return "shape mismatch";
+    case SMC_E_ALIAS: return "output overlaps an input";
+    case SMC_E_CAPACITY: return "hash table capacity exhausted";
+    case SMC_E_OOM: return "device allocation failed";
+    case SMC_E_CUDA: return "CUDA error";
+    case SMC_E_TIMEOUT: return "device-side wait timed out";
+    case SMC_E_ALIGN: return "misaligned device pointer";
+    default: return "unknown error";
+  }
+}
+
+int smc_set_hash_capacity(int64_t slots) {
+  if (slots < 0) return SMC_E_ARG;
+  g_capacity_override.store(slots);
+  return SMC_OK;
+}
+
+int smc_set_profiling(int32_t on) {
+  g_profiling.store(on ? 1 : 0);
+  return SMC_OK;
+}
+
+int smc_build_map(const int32_t* coords, int64_t n, int32_t batch, const int32_t grid[3], void* stream,
+                  smc_map** out) {
+  if (!out) return SMC_E_ARG;
+  *out = nullptr;
+  if (!grid || n < 0 || batch < 1 || (n > 0 && !coords)) return SMC_E_ARG;
+  if (grid[0] < 1 || grid[1] < 1 || grid[2] < 1) return SMC_E_ARG;
+  if (n >= (1ll << 31) - 1) return SMC_E_ARG;  // rows are int32
+  if (n > 0 && (reinterpret_cast<uintptr_t>(coords) & 15u)) return SMC_E_ALIGN;
+  const double sites = static_cast<double>(batch) * grid[0] * grid[1] * grid[2];
+  if (sites >= 4.6e18) return SMC_E_ARG;
+  if (pending_cuda_error() != SMC_OK) return SMC_E_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  smc_map* m = new (std::nothrow) smc_map();
+  if (!m) return SMC_E_OOM;
+  std::memset(m, 0, sizeof(*m));
+  cudaGetDevice(&m->device);
+  m->stream = s;
+  m->n = n;
+  m->batch = batch;
+  for (int i = 0; i < 3; ++i) m->grid[i] = grid[i];
+  if (n == 0) {
+    *out = m;
+    return SMC_OK;
+  }
+
+  // ---- sizes
+  const bool wide = sites > 4294967294.0;  // packed slots need keys < 2^32 - 1
+  int lg = 4;
+  const int64_t forced = g_capacity_override.load();
+  const int64_t want = forced > 0 ? forced : 2 * n;
+  while ((1ll << lg) < want) ++lg;
+  const int64_t cap = 1ll << lg;
+  const int nb = smc::map_nblocks(n);
+  const int64_t Lmap = 27ll * nb;
+  const int nblk = smc::radix_nblocks(n);
+  const int64_t Lrad = static_cast<int64_t>(smc::radix_bins()) * nblk;
+  const int64_t pair_cap = 27ll * n;
+
+  Carve keep;
+  const size_t o_nbr = keep.take<int32_t>(27ull * n);
+  const size_t o_in = keep.take<int32_t>(pair_cap);
+  const size_t o_out = keep.take<int32_t>(pair_cap);
+  const size_t o_perm = keep.take<int32_t>(n);
+  Carve tmp;
+  const size_t o_table = tmp.take<unsigned long long>(wide ? 2 * cap : cap);
+  const size_t o_err = tmp.take<uint32_t>(1);
+  const size_t o_info = tmp.take<int64_t>(28);
+  const size_t o_total = tmp.take<int64_t>(1);
+  const size_t o_gkey = tmp.take<uint32_t>(n);
+  const size_t o_bc = tmp.take<int32_t>(Lmap);
+  const size_t o_bo = tmp.take<int64_t>(Lmap);
+  const size_t o_sp = tmp.take<int64_t>(smc::scan_partials_len(Lmap > Lrad ? Lmap : Lrad));
+  const size_t o_hist = tmp.take<int32_t>(Lrad);
+  const size_t o_hoff = tmp.take<int64_t>(Lrad);
+  const size_t o_ktmp = tmp.take<uint32_t>(n);
+  const size_t o_vtmp = tmp.take<int32_t>(n);
+
+  void* kp = nullptr;
+  void* tp = nullptr;
+  if (cudaMallocAsync(&kp, keep.off, s) != cudaSuccess) {
+    cudaGetLastError();
+    delete m;
+    return SMC_E_OOM;
+  }
+  if (cudaMallocAsync(&tp, tmp.off, s) != cudaSuccess) {
+    cudaGetLastError();
+    cudaFreeAsync(kp, s);
+    delete m;
+    return SMC_E_OOM;
+  }
+  char* K = static_cast<char*>(kp);
+  char* T = static_cast<char*>(tp);
+  m->keep = kp;
+  m->nbr = reinterpret_cast<int32_t*>(K + o_nbr);
+  m->in_idx = reinterpret_cast<int32_t*>(K + o_in);
+  m->out_idx = reinterpret_cast<int32_t*>(K + o_out);
+  m->perm = reinterpret_cast<int32_t*>(K + o_perm);
+
+  const bool prof = g_profiling.load() != 0;
+  cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};
+  if (prof)
+    for (auto& e : ev) cudaEventCreate(&e);
+
+  int rc = SMC_OK;
+  cudaError_t ce = cudaMemsetAsync(T + o_table, 0xFF, (wide ? 2 : 1) * cap * sizeof(unsigned long long), s);
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(T + o_err, 0, sizeof(uint32_t), s);
+  if (prof) cudaEventRecord(ev[0], s);
+  if (ce == cudaSuccess) {
+    smc::MapBuildArgs a;
+    a.coords = coords;
+    a.n = n;
+    a.batch = batch;
+    a.Z = grid[0];
+    a.Y = grid[1];
+    a.X = grid[2];
+    a.wide = wide;
+    a.table = reinterpret_cast<unsigned long long*>(T + o_table);
+    a.lg = lg;
+    a.err = reinterpret_cast<uint32_t*>(T + o_err);
+    a.nbr = m->nbr;
+    a.gkey = reinterpret_cast<uint32_t*>(T + o_gkey);
+    a.block_counts = reinterpret_cast<int32_t*>(T + o_bc);
+    a.block_offsets = reinterpret_cast<int64_t*>(T + o_bo);
+    a.scan_partials = reinterpret_cast<int64_t*>(T + o_sp);
+    a.total = reinterpret_cast<int64_t*>(T + o_total);
+    a.info = reinterpret_cast<int64_t*>(T + o_info);
+    a.in_idx = m->in_idx;
+    a.out_idx = m->out_idx;
+    ce = smc::launch_map_build(a, s);
+  }
+  if (prof) cudaEventRecord(ev[1], s);
+  if (ce == cudaSuccess) {
+    smc::ScheduleArgs b;
+    b.gkey = reinterpret_cast<uint32_t*>(T + o_gkey);
+    b.n = n;
+    b.hist = reinterpret_cast<int32_t*>(T + o_hist);
+    b.hoff = reinterpret_cast<int64_t*>(T + o_hoff);
+    b.scan_partials = reinterpret_cast<int64_t*>(T + o_sp);
+    b.key_tmp = reinterpret_cast<uint32_t*>(T + o_ktmp);
+    b.val_tmp = reinterpret_cast<int32_t*>(T + o_vtmp);
+    b.perm = m->perm;
+    ce = smc::launch_schedule(b, s);
+  }
+  if (prof) cudaEventRecord(ev[2], s);
+  // one device->host read: error bits and pair offsets
+  struct {
+    uint32_t err;
+    uint32_t pad;
+    int64_t info[28];
+  } h;
+  std::memset(&h, 0, sizeof(h));
+  if (ce == cudaSuccess) ce = cudaMemcpyAsync(&h.err, T + o_err, sizeof(uint32_t), cudaMemcpyDeviceToHost, s);
+  if (ce == cudaSuccess) ce = cudaMemcpyAsync(h.info, T + o_info, 28 * sizeof(int64_t), cudaMemcpyDeviceToHost, s);
+  cudaFreeAsync(tp, s);
+  if (ce == cudaSuccess) ce = cudaStreamSynchronize(s);
+  if (ce != cudaSuccess) {
+    cudaGetLastError();
+    rc = SMC_E_CUDA;
+  } else if (h.err & smc::kErrRange) {
+    rc = SMC_E_RANGE;
+  } else if (h.err & smc::kErrDuplicate) {
+    rc = SMC_E_DUPLICATE;
+  } else if (h.err & smc::kErrCapacity) {
+    rc = SMC_E_CAPACITY;
+  }
+  if (prof) {
+    if (rc == SMC_OK) {
+      cudaEventElapsedTime(&m->ms[0], ev[0], ev[1]);
+      cudaEventElapsedTime(&m->ms[1], ev[1], ev[2]);
+    }
+    for (auto& e : ev) cudaEventDestroy(e);
+  }
+  if (rc != SMC_OK) {
+    cudaFreeAsync(kp, s);
+    cudaStreamSynchronize(s);
+    cudaGetLastError();
+    delete m;
+    return rc;
+  }
+  for (int d = 0; d < 28; ++d) m->offsets[d] = h.info[d];
+  for (int d = 0; d < 27; ++d) m->counts[d] = h.info[d + 1] - h.info[d];
+  *out = m;
+  return SMC_OK;
+}
+
+int smc_conv(const smc_map* map, const void* feats, int64_t cin, const void* weight, const void* bias,
+             void* out, int64_t cout, int32_t ksize, int32_t orientation, int32_t dtype, void* stream) {
+  if (!map) return SMC_E_ARG;
+  if (ksize != 1 && ksize != 3) return SMC_E_ARG;
+  if (orientation != 1 && orientation != -1) return SMC_E_ARG;
+  if (dtype != SMC_F32 && dtype != SMC_BF16 && dtype != SMC_F16) return SMC_E_DTYPE;
+  if (cin < 1 || cout < 1 || cin > (1 << 24) || cout > (1 << 24)) return SMC_E_SHAPE;
+  const int64_t n = map->n;
+  if (n == 0) return SMC_OK;
+  if (!feats || !weight || !out) return SMC_E_ARG;
+  const size_t esz = dtype == SMC_F32 ? 4 : 2;
+  const int taps = ksize == 3 ? 27 : 1;
+  if (ranges_overlap(out, n * cout * esz, feats, n * cin * esz) ||
+      ranges_overlap(out, n * cout * esz, weight, static_cast<size_t>(cout) * taps * cin * esz) ||
+      ranges_overlap(out, n * cout * esz, bias, static_cast<size_t>(cout) * esz))
+    return SMC_E_ALIAS;
+  if (pending_cuda_error() != SMC_OK) return SMC_E_CUDA;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  uint32_t* st = device_status(dev);
+  if (!st) return SMC_E_OOM;
+  smc::ConvArgs a;
+  a.feats = feats;
+  a.weight = weight;
+  a.bias = bias;
+  a.out = out;
+  a.nbr = map->nbr;
+  a.perm = map->perm;
+  a.n = n;
+  a.cin = static_cast<int>(cin);
+  a.cout = static_cast<int>(cout);
+  a.taps = taps;
+  a.orientation = orientation;
+  a.dtype = dtype;
+  a.err = st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = smc::conv_tc_supported(a) ? smc::launch_conv_tc(a, s) : smc::launch_conv_simt(a, s);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return SMC_E_CUDA;
+  }
+  return SMC_OK;
+}
+
+int smc_map_info(const smc_map* map, int64_t* n, int64_t counts[27]) {
+  if (!map) return SMC_E_ARG;
+  if (n) *n = map->n;
+  if (counts)
+    for (int d = 0; d < 27; ++d) counts[d] = map->counts[d];
+  return SMC_OK;
+}
+
+int smc_map_nbr(const smc_map* map, const int32_t** nbr) {
+  if (!map || !nbr) return SMC_E_ARG;
+  *nbr = map->nbr;
+  return SMC_OK;
+}
+
+int smc_map_pairs(const smc_map* map, const int32_t** in_idx, const int32_t** out_idx, int64_t offsets[28]) {
+  if (!map) return SMC_E_ARG;
+  if (in_idx) *in_idx = map->in_idx;
+  if (out_idx) *out_idx = map->out_idx;
+  if (offsets)
+    for (int d = 0; d < 28; ++d) offsets[d] = map->offsets[d];
+  return SMC_OK;
+}
+
+int smc_map_schedule(const smc_map* map, const int32_t** perm) {
+  if (!map || !perm) return SMC_E_ARG;
+  *perm = map->perm;
+  return SMC_OK;
+}
+
+int smc_kernel_launches(int64_t* count) {
+  if (!count) return SMC_E_ARG;
+  *count = g_launches.load();
+  return SMC_OK;
+}
+
+int smc_map_timing(const smc_map* map, float ms[2]) {
+  if (!map || !ms) return SMC_E_ARG;
+  ms[0] = map->ms[0];
+  ms[1] = map->ms[1];
+  return SMC_OK;
+}
+
+int smc_free_map(smc_map* map) {
+  if (!map) return SMC_OK;
+  int rc = SMC_OK;
+  if (map->keep) {
+    int cur = 0;
+    cudaGetDevice(&cur);
+    if (cur != map->device) cudaSetDevice(map->device);
+    if (cudaFreeAsync(map->keep, map->stream) != cudaSuccess) {
+      cudaGetLastError();
+      rc = SMC_E_CUDA;
+    }
+    if (cur != map->device) cudaSetDevice(cur);
+  }
+  delete map;
+  return rc;
+}
+
+int smc_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return SMC_E_CUDA;
+  }
+  int dev = 0;
+  cudaGetDevice(&dev);
+  uint32_t* st = device_status(dev);
+  if (!st) return SMC_E_OOM;
+  uint32_t h = 0;
+  if (cudaMemcpy(&h, st, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return SMC_E_CUDA;
+  if (h) cudaMemset(st, 0, sizeof(uint32_t));
+  return (h & smc::kErrTimeout) ? SMC_E_TIMEOUT : SMC_OK;
+}
+
+}  // extern "C"

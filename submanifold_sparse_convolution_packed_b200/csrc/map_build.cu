@@ -1,0 +1,430 @@
+// Neighbour-map construction for submanifold convolution (sm_100a).
+//
+// The pages build a "sorted-key indice map" with 27 vectorised lookups per
+// voxel, cached per coordinate set (LATO.2 MLX port README, summary).  Here
+// the lookup structure is an open-addressing hash table in device memory:
+//   k_insert      one thread per voxel: validate (b,z,y,x), form the 64-bit
+//                 linear site key, insert (key,row) with atomicCAS and linear
+//                 probing; duplicates and a full table set error bits.
+//   k_neighbours  one thread per voxel: 27 lookups -> int32 [n,27] map row
+//                 (staged in shared memory, written coalesced), a 20-bit
+//                 grouping key for the tile schedule, per-block hit counts.
+//   scan          exclusive scan of the block counts in (offset, block) order.
+//   k_pairs       stable compaction of every map column into the per-offset
+//                 pair lists (ascending output row).
+//   radix sort    stable 2x10-bit LSD sort of rows by the grouping key: the
+//                 order in which the tensor-core conv forms 128-row tiles.
+#include <cstdint>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace smc {
+
+constexpr uint64_t kEmpty = ~0ull;
+constexpr uint64_t kFib = 0x9E3779B97F4A7C15ull;
+
+__device__ __forceinline__ uint64_t slot_of(uint64_t key, int lg) { return (key * kFib) >> (64 - lg); }
+
+__device__ __forceinline__ bool site_ok(int4 c, int32_t batch, int32_t Z, int32_t Y, int32_t X) {
+  return c.x >= 0 && c.x < batch && c.y >= 0 && c.y < Z && c.z >= 0 && c.z < Y && c.w >= 0 &&
+         c.w < X;
+}
+
+__device__ __forceinline__ uint64_t site_key(int4 c, int32_t Z, int32_t Y, int32_t X) {
+  return ((static_cast<uint64_t>(c.x) * Z + c.y) * Y + c.z) * X + c.w;
+}
+
+// Packed layout: one word per slot, (key << 32) | row, for keys < 2^32 - 1.
+// Wide layout: two words per slot, key then row.
+template <bool kWide>
+__global__ void __launch_bounds__(256) k_insert(const int4* __restrict__ coords, int64_t n, int32_t batch,
+                                                int32_t Z, int32_t Y, int32_t X,
+                                                unsigned long long* table, int lg, uint32_t* err) {
+  const uint64_t mask = (1ull << lg) - 1;
+  for (int64_t v = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; v < n;
+       v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int4 c = coords[v];
+    if (!site_ok(c, batch, Z, Y, X)) {
+      atomicOr(err, kErrRange);
+      continue;
+    }
+    const uint64_t key = site_key(c, Z, Y, X);
+    uint64_t s = slot_of(key, lg);
+    bool placed = false;
+    for (uint64_t probe = 0; probe <= mask; ++probe) {
+      if (!kWide) {
+        const unsigned long long want = (key << 32) | static_cast<uint32_t>(v);
+        const unsigned long long prev = atomicCAS(&table[s], kEmpty, want);
+        if (prev == kEmpty) { placed = true; break; }
+        if ((prev >> 32) == key) { atomicOr(err, kErrDuplicate); placed = true; break; }
+      } else {
+        const unsigned long long prev = atomicCAS(&table[2 * s], kEmpty, key);
+        if (prev == kEmpty) { table[2 * s + 1] = static_cast<uint64_t>(v); placed = true; break; }
+        if (prev == key) { atomicOr(err, kErrDuplicate); placed = true; break; }
+      }
+      s = (s + 1) & mask;
+    }
+    if (!placed) atomicOr(err, kErrCapacity);
+  }
+}
+
+template <bool kWide>
+__device__ __forceinline__ int32_t lookup(const unsigned long long* __restrict__ table, uint64_t mask,
+                                          int lg, uint64_t key) {
+  uint64_t s = slot_of(key, lg);
+  for (uint64_t probe = 0; probe <= mask; ++probe) {
+    if (!kWide) {
+      const uint64_t e = __ldg(&table[s]);
+      if (e == kEmpty) return -1;
+      if ((e >> 32) == key) return static_cast<int32_t>(e & 0xFFFFFFFFull);
+    } else {
+      const uint64_t k = __ldg(&table[2 * s]);
+      if (k == kEmpty) return -1;
+      if (k == key) return static_cast<int32_t>(__ldg(&table[2 * s + 1]));
+    }
+    s = (s + 1) & mask;
+  }
+  return -1;
+}
+
+// Grouping key of a 27-bit hit mask: the 8 corner offsets then the 12 edge
+// offsets, most significant first.  Rows whose rarer neighbours agree end up
+// adjacent after sorting, so a 128-row tile shares most of its absent taps.
+__device__ __forceinline__ uint32_t group_key(uint32_t m) {
+  constexpr int kOrder[20] = {0, 2, 6, 8, 18, 20, 24, 26, 1, 3, 5, 7, 9, 11, 15, 17, 19, 21, 23, 25};
+  uint32_t k = 0;
+#pragma unroll
+  for (int i = 0; i < 20; ++i) k |= ((m >> kOrder[i]) & 1u) << (19 - i);
+  return k;
+}
+
+constexpr int kMapBlock = 256;
+
+template <bool kWide>
+__global__ void __launch_bounds__(kMapBlock) k_neighbours(
+    const int4* __restrict__ coords, int64_t n, int32_t Z, int32_t Y, int32_t X,
+    const unsigned long long* __restrict__ table, int lg, int32_t* __restrict__ nbr,
+    uint32_t* __restrict__ gkey, int32_t* __restrict__ block_counts, int nblocks) {
+  __shared__ int32_t s_nbr[kMapBlock * kTaps];
+  __shared__ int32_t s_cnt[kMapBlock / 32][kTaps];
+  const uint64_t mask = (1ull << lg) - 1;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kMapBlock;
+  const int64_t v = base + tid;
+  uint32_t hits = 0;
+  if (v < n) {
+    const int4 c = coords[v];
+    const uint64_t key = site_key(c, Z, Y, X);
+    const int64_t sz = static_cast<int64_t>(Y) * X;
+#pragma unroll
+    for (int d = 0; d < kTaps; ++d) {
+      const int dz = d / 9 - 1, dy = (d / 3) % 3 - 1, dx = d % 3 - 1;
+      int32_t r = -1;
+      if (c.y + dz >= 0 && c.y + dz < Z && c.z + dy >= 0 && c.z + dy < Y && c.w + dx >= 0 &&
+          c.w + dx < X) {
+        const uint64_t nk = key + static_cast<uint64_t>(dz * sz + static_cast<int64_t>(dy) * X + dx);
+        r = lookup<kWide>(table, mask, lg, nk);
+      }
+      s_nbr[tid * kTaps + d] = r;
+      hits |= static_cast<uint32_t>(r >= 0) << d;
+    }
+    gkey[v] = group_key(hits);
+  }
+#pragma unroll
+  for (int d = 0; d < kTaps; ++d) {
+    const uint32_t b = __ballot_sync(0xffffffffu, (hits >> d) & 1u);
+    if (lane == 0) s_cnt[warp][d] = __popc(b);
+  }
+  __syncthreads();
+  const int64_t rows = n - base < kMapBlock ? n - base : kMapBlock;
+  const int total = static_cast<int>(rows) * kTaps;
+  int32_t* dst = nbr + base * kTaps;  // base*27*4 bytes is a multiple of 16
+  const int vec = total >> 2;
+  for (int i = tid; i < vec; i += kMapBlock)
+    reinterpret_cast<int4*>(dst)[i] = reinterpret_cast<const int4*>(s_nbr)[i];
+  for (int i = (vec << 2) + tid; i < total; i += kMapBlock) dst[i] = s_nbr[i];
+  if (tid < kTaps) {
+    int32_t s = 0;
+#pragma unroll
+    for (int w = 0; w < kMapBlock / 32; ++w) s += s_cnt[w][tid];
+    block_counts[static_cast<int64_t>(tid) * nblocks + blockIdx.x] = s;
+  }
+}
+
+__global__ void __launch_bounds__(kMapBlock) k_pairs(const int32_t* __restrict__ nbr, int64_t n,
+                                                     const int64_t* __restrict__ block_offsets,
+                                                     int nblocks, int32_t* __restrict__ in_idx,
+                                                     int32_t* __restrict__ out_idx) {
+  __shared__ int32_t s_nbr[kMapBlock * kTaps];
+  __shared__ int32_t s_pre[kMapBlock / 32][kTaps];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kMapBlock;
+  const int64_t rows = n - base < kMapBlock ? n - base : kMapBlock;
+  const int total = static_cast<int>(rows) * kTaps;
+  const int32_t* src = nbr + base * kTaps;
+  const int vec = total >> 2;
+  for (int i = tid; i < vec; i += kMapBlock)
+    reinterpret_cast<int4*>(s_nbr)[i] = reinterpret_cast<const int4*>(src)[i];
+  for (int i = (vec << 2) + tid; i < total; i += kMapBlock) s_nbr[i] = src[i];
+  __syncthreads();
+  const int64_t v = base + tid;
+  const bool live = tid < rows;
+#pragma unroll
+  for (int d = 0; d < kTaps; ++d) {
+    const bool hit = live && s_nbr[tid * kTaps + d] >= 0;
+    const uint32_t b = __ballot_sync(0xffffffffu, hit);
+    if (lane == 0) s_pre[warp][d] = __popc(b);
+  }
+  __syncthreads();
+  if (tid < kTaps) {
+    int32_t run = 0;
+#pragma unroll
+    for (int w = 0; w < kMapBlock / 32; ++w) {
+      const int32_t t = s_pre[w][tid];
+      s_pre[w][tid] = run;
+      run += t;
+    }
+  }
+  __syncthreads();
+  const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll 1
+  for (int d = 0; d < kTaps; ++d) {
+    const int32_t u = live ? s_nbr[tid * kTaps + d] : -1;
+    const uint32_t b = __ballot_sync(0xffffffffu, u >= 0);
+    if (u >= 0) {
+      const int64_t pos = block_offsets[static_cast<int64_t>(d) * nblocks + blockIdx.x] +
+                          s_pre[warp][d] + __popc(b & lt);
+      in_idx[pos] = u;
+      out_idx[pos] = static_cast<int32_t>(v);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ scan
+constexpr int kScanThreads = 1024;
+constexpr int kScanItems = 4;
+constexpr int kScanSeg = kScanThreads * kScanItems;
+
+__device__ __forceinline__ int64_t block_exclusive_scan(int64_t x, int64_t* s_warp, int64_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int64_t incl = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    int64_t w = lane < nw ? s_warp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < nw) s_warp[lane] = w;
+  }
+  __syncthreads();
+  const int64_t before = warp > 0 ? s_warp[warp - 1] : 0;
+  if (total) *total = s_warp[(blockDim.x >> 5) - 1];
+  __syncthreads();
+  return before + incl - x;
+}
+
+__global__ void __launch_bounds__(kScanThreads) k_scan_reduce(const int32_t* __restrict__ in, int64_t L,
+                                                              int64_t* __restrict__ partials) {
+  __shared__ int64_t s_warp[32];
+  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * kScanSeg;
+  int64_t s = 0;
+#pragma unroll
+  for (int i = 0; i < kScanItems; ++i) {
+    const int64_t j = b0 + static_cast<int64_t>(i) * kScanThreads + threadIdx.x;
+    if (j < L) s += in[j];
+  }
+  int64_t tot;
+  block_exclusive_scan(s, s_warp, &tot);
+  if (threadIdx.x == 0) partials[blockIdx.x] = tot;
+}
+
+// Exclusive scan of the segment partials in place (one block, any count).
+__global__ void __launch_bounds__(kScanThreads) k_scan_partials(int64_t* partials, int64_t nseg,
+                                                                int64_t* grand_total) {
+  __shared__ int64_t s_warp[32];
+  int64_t carry = 0;
+  for (int64_t c0 = 0; c0 < nseg; c0 += kScanThreads) {
+    const int64_t j = c0 + threadIdx.x;
+    const int64_t x = j < nseg ? partials[j] : 0;
+    int64_t tot;
+    const int64_t ex = block_exclusive_scan(x, s_warp, &tot);
+    if (j < nseg) partials[j] = carry + ex;
+    carry += tot;
+  }
+  if (threadIdx.x == 0 && grand_total) *grand_total = carry;
+}
+
+__global__ void __launch_bounds__(kScanThreads) k_scan_apply(const int32_t* __restrict__ in, int64_t L,
+                                                             const int64_t* __restrict__ partials,
+                                                             int64_t* __restrict__ out) {
+  __shared__ int64_t s_warp[32];
+  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * kScanSeg + threadIdx.x * kScanItems;
+  int32_t v[kScanItems];
+  int64_t s = 0;
+#pragma unroll
+  for (int i = 0; i < kScanItems; ++i) {
+    v[i] = b0 + i < L ? in[b0 + i] : 0;
+    s += v[i];
+  }
+  int64_t run = partials[blockIdx.x] + block_exclusive_scan(s, s_warp, nullptr);
+#pragma unroll
+  for (int i = 0; i < kScanItems; ++i) {
+    if (b0 + i < L) out[b0 + i] = run;
+    run += v[i];
+  }
+}
+
+// Per-offset totals: counts[d] and offsets[0..27] of the pair lists from the
+// scanned block counts.
+__global__ void k_pair_info(const int64_t* __restrict__ block_offsets, int nblocks,
+                            const int64_t* __restrict__ total, int64_t* __restrict__ info) {
+  const int d = threadIdx.x;
+  if (d < kTaps) info[d] = block_offsets[static_cast<int64_t>(d) * nblocks];
+  if (d == kTaps) info[kTaps] = *total;
+}
+
+// ------------------------------------------------------------ radix sort
+constexpr int kRadixBits = 10;
+constexpr int kRadixBins = 1 << kRadixBits;
+constexpr int kRadixThreads = 256;
+constexpr int kRadixRounds = 8;
+constexpr int kRadixChunk = kRadixThreads * kRadixRounds;
+
+__global__ void __launch_bounds__(kRadixThreads) k_radix_hist(const uint32_t* __restrict__ keys, int64_t n,
+                                                              int shift, int32_t* __restrict__ hist,
+                                                              int nblk) {
+  __shared__ int32_t s_h[kRadixBins];
+  for (int i = threadIdx.x; i < kRadixBins; i += kRadixThreads) s_h[i] = 0;
+  __syncthreads();
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kRadixChunk;
+  for (int i = threadIdx.x; i < kRadixChunk; i += kRadixThreads) {
+    const int64_t j = c0 + i;
+    if (j < n) atomicAdd(&s_h[(keys[j] >> shift) & (kRadixBins - 1)], 1);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kRadixBins; i += kRadixThreads)
+    hist[static_cast<int64_t>(i) * nblk + blockIdx.x] = s_h[i];
+}
+
+// Stable scatter of one radix pass.  The chunk of a block is visited in
+// rounds of 256 consecutive elements; inside a round, an element's rank is
+// (elements of its digit in earlier rounds) + (in earlier warps of this
+// round) + (in earlier lanes of its warp), so the input order is kept.
+__global__ void __launch_bounds__(kRadixThreads) k_radix_scatter(
+    const uint32_t* __restrict__ keys_in, const int32_t* __restrict__ vals_in, int64_t n, int shift,
+    const int64_t* __restrict__ offsets, int nblk, uint32_t* __restrict__ keys_out,
+    int32_t* __restrict__ vals_out) {
+  __shared__ unsigned long long s_base[kRadixBins];
+  __shared__ int32_t s_wcnt[kRadixThreads / 32][kRadixBins];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < kRadixBins; i += kRadixThreads)
+    s_base[i] = static_cast<unsigned long long>(offsets[static_cast<int64_t>(i) * nblk + blockIdx.x]);
+  for (int i = tid; i < (kRadixThreads / 32) * kRadixBins; i += kRadixThreads)
+    (&s_wcnt[0][0])[i] = 0;
+  __syncthreads();
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kRadixChunk;
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int round = 0; round < kRadixRounds; ++round) {
+    const int64_t j = c0 + static_cast<int64_t>(round) * kRadixThreads + tid;
+    const bool valid = j < n;
+    const uint32_t key = valid ? keys_in[j] : 0u;
+    const int32_t val = valid ? (vals_in ? vals_in[j] : static_cast<int32_t>(j)) : 0;
+    const uint32_t digit = (key >> shift) & (kRadixBins - 1);
+    const uint32_t peers = __match_any_sync(0xffffffffu, valid ? digit : 0xFFFFFFFFu);
+    const bool leader = valid && (__ffs(peers) - 1) == lane;
+    if (leader) s_wcnt[warp][digit] = __popc(peers);
+    __syncthreads();
+    if (valid) {
+      long long pos = static_cast<long long>(s_base[digit]) + __popc(peers & lt);
+      for (int w = 0; w < warp; ++w) pos += s_wcnt[w][digit];
+      if (keys_out) keys_out[pos] = key;
+      vals_out[pos] = val;
+    }
+    __syncthreads();
+    if (leader) {
+      atomicAdd(&s_base[digit], static_cast<unsigned long long>(__popc(peers)));
+      s_wcnt[warp][digit] = 0;
+    }
+    __syncwarp();
+  }
+}
+
+// ------------------------------------------------------------ launchers
+static cudaError_t scan_i32(const int32_t* in, int64_t L, int64_t* out, int64_t* partials,
+                            int64_t* grand_total, cudaStream_t s) {
+  const int64_t nseg = (L + kScanSeg - 1) / kScanSeg;
+  if (nseg == 0) return cudaSuccess;
+  k_scan_reduce<<<static_cast<unsigned>(nseg), kScanThreads, 0, s>>>(in, L, partials);
+  k_scan_partials<<<1, kScanThreads, 0, s>>>(partials, nseg, grand_total);
+  k_scan_apply<<<static_cast<unsigned>(nseg), kScanThreads, 0, s>>>(in, L, partials, out);
+  count_launches(3);
+  return cudaGetLastError();
+}
+
+int64_t scan_partials_len(int64_t L) { return (L + kScanSeg - 1) / kScanSeg + 1; }
+int map_nblocks(int64_t n) { return static_cast<int>((n + kMapBlock - 1) / kMapBlock); }
+int radix_nblocks(int64_t n) { return static_cast<int>((n + kRadixChunk - 1) / kRadixChunk); }
+int radix_bins() { return kRadixBins; }
+
+cudaError_t launch_map_build(const MapBuildArgs& a, cudaStream_t s) {
+  const int64_t n = a.n;
+  if (n == 0) return cudaSuccess;
+  const int nb = map_nblocks(n);
+  const int grid_ins = static_cast<int>((n + 255) / 256);
+  if (a.wide) {
+    k_insert<true><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.batch,
+                                            a.Z, a.Y, a.X, a.table, a.lg, a.err);
+    k_neighbours<true><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.Z,
+                                                a.Y, a.X, a.table, a.lg, a.nbr, a.gkey,
+                                                a.block_counts, nb);
+  } else {
+    k_insert<false><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.batch,
+                                             a.Z, a.Y, a.X, a.table, a.lg, a.err);
+    k_neighbours<false><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.Z,
+                                                 a.Y, a.X, a.table, a.lg, a.nbr, a.gkey,
+                                                 a.block_counts, nb);
+  }
+  count_launches(2);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t L = static_cast<int64_t>(kTaps) * nb;
+  e = scan_i32(a.block_counts, L, a.block_offsets, a.scan_partials, a.total, s);
+  if (e != cudaSuccess) return e;
+  k_pair_info<<<1, 32, 0, s>>>(a.block_offsets, nb, a.total, a.info);
+  k_pairs<<<nb, kMapBlock, 0, s>>>(a.nbr, n, a.block_offsets, nb, a.in_idx, a.out_idx);
+  count_launches(2);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_schedule(const ScheduleArgs& a, cudaStream_t s) {
+  const int64_t n = a.n;
+  if (n == 0) return cudaSuccess;
+  const int nblk = radix_nblocks(n);
+  const int64_t L = static_cast<int64_t>(kRadixBins) * nblk;
+  // pass 1: low 10 bits, rows in input order
+  k_radix_hist<<<nblk, kRadixThreads, 0, s>>>(a.gkey, n, 0, a.hist, nblk);
+  cudaError_t e = scan_i32(a.hist, L, a.hoff, a.scan_partials, nullptr, s);
+  if (e != cudaSuccess) return e;
+  k_radix_scatter<<<nblk, kRadixThreads, 0, s>>>(a.gkey, nullptr, n, 0, a.hoff, nblk, a.key_tmp,
+                                                 a.val_tmp);
+  // pass 2: high 10 bits
+  k_radix_hist<<<nblk, kRadixThreads, 0, s>>>(a.key_tmp, n, kRadixBits, a.hist, nblk);
+  e = scan_i32(a.hist, L, a.hoff, a.scan_partials, nullptr, s);
+  if (e != cudaSuccess) return e;
+  k_radix_scatter<<<nblk, kRadixThreads, 0, s>>>(a.key_tmp, a.val_tmp, n, kRadixBits, a.hoff, nblk,
+                                                 nullptr, a.perm);
+  count_launches(4);
+  return cudaGetLastError();
+}
+
+}  // namespace smc

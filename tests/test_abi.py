@@ -1,0 +1,52 @@
+"""CPU checks of the C ABI: the library loads and exports exactly the entry
+points include/smc.h declares (no compute call is made without a GPU)."""
+import os
+import re
+import subprocess
+
+import submanifold_sparse_convolution_packed_b200 as smc
+from submanifold_sparse_convolution_packed_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared():
+    src = open(os.path.join(ROOT, "include", "smc.h")).read()
+    return sorted(set(re.findall(r"SMC_API\s+[\w\s\*]+?\b(smc_\w+)\s*\(", src)))
+
+
+def test_header_declares_binding_exports():
+    assert declared() == sorted(smc.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    B.build()
+    lib = smc.lib()
+    for name in declared():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB], capture_output=True, text=True).stdout
+    exported = sorted(l.split()[-1] for l in out.splitlines() if " T " in l)
+    assert exported == declared()
+
+
+def test_strerror_without_gpu():
+    lib = smc.lib()
+    assert lib.smc_strerror(0) == b"ok"
+    assert lib.smc_strerror(-3) == b"duplicate coordinate"
+    assert lib.smc_set_hash_capacity(-1) == -1
+    assert lib.smc_set_hash_capacity(0) == 0
+
+
+def test_argument_errors_without_gpu():
+    """Validation happens before any device work, so these run on a CPU machine."""
+    import ctypes
+    lib = smc.lib()
+    h = ctypes.c_void_p()
+    grid = (ctypes.c_int32 * 3)(4, 4, 4)
+    assert lib.smc_build_map(None, 5, 1, grid, None, ctypes.byref(h)) == -1   # null coords
+    assert lib.smc_build_map(None, -1, 1, grid, None, ctypes.byref(h)) == -1  # n < 0
+    assert lib.smc_build_map(None, 0, 0, grid, None, ctypes.byref(h)) == -1   # batch 0
+    assert lib.smc_build_map(ctypes.c_void_p(8), 3, 1, grid, None, ctypes.byref(h)) == -11  # misaligned
+    assert h.value is None
+    assert lib.smc_conv(None, None, 1, None, None, None, 1, 3, 1, 0, None) == -1
+    assert lib.smc_free_map(None) == 0

@@ -1,0 +1,306 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle.
+
+Every case draws seeded inputs from ``synth`` and feeds the same values to
+both sides.  Bars:
+* neighbour map, pair lists: bit-exact;
+* fp32 conv: max|gpu - oracle| <= 1e-5 * max|oracle|;
+* bf16 / fp16 conv: max|gpu - oracle| <= 5e-3 * max|oracle|, the oracle run
+  in fp64 on the identically rounded inputs;
+* small-integer inputs: bit-exact in every dtype.
+Large workloads are checked on a seeded sample of output rows.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import submanifold_sparse_convolution_packed_b200 as smc
+from submanifold_sparse_convolution_packed_b200 import synth as S
+
+pytestmark = pytest.mark.gpu
+
+TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}
+TOL = {"f32": 1e-5, "bf16": 5e-3, "f16": 5e-3}
+THREADS = min(32, os.cpu_count() or 1)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    smc.lib()
+    yield
+    smc.clear_cache()
+
+
+_WL = {}
+
+
+def workload(name):
+    if name not in _WL:
+        _WL[name] = S.workload(name)
+    return _WL[name]
+
+
+def dev(x, dtype="f32"):
+    return torch.from_numpy(np.ascontiguousarray(x)).to(TORCH_DT[dtype]).cuda()
+
+
+def host(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def build(w, **kw):
+    coords = torch.from_numpy(w.coords).cuda()
+    batch = int(w.coords[:, 0].max()) + 1 if w.n else 1
+    return smc.build_map(coords, w.grid, batch=batch, **kw)
+
+
+def check_close(got, ref, dtype, what=""):
+    err = float(np.abs(got - ref).max()) if ref.size else 0.0
+    scale = float(np.abs(ref).max()) if ref.size else 0.0
+    assert err <= TOL[dtype] * scale, f"{what}: max err {err:.3e} vs bound {TOL[dtype] * scale:.3e}"
+
+
+def sample_rows(n, k, seed):
+    if n <= k:
+        return None
+    return np.sort(np.random.default_rng(seed).choice(n, size=k, replace=False))
+
+
+# ------------------------------------------------------------------ map
+MAP_CASES = ["tiny", "shell2", "shells6", "varlen4", "decoder0", "decoder3", "full128"]
+
+
+@pytest.mark.parametrize("name", MAP_CASES)
+def test_map_bit_exact(oracle_mod, name):
+    w = workload(name)
+    m = build(w)
+    nbr = m.nbr().cpu().numpy()
+    ref = oracle_mod.neighbour_map(w.coords, w.grid)
+    np.testing.assert_array_equal(nbr, ref)
+    counts, offsets, in_idx, out_idx = oracle_mod.pair_lists(ref)
+    assert m.counts == counts.tolist()
+    assert m.offsets == offsets.tolist()
+    gi, go, _ = m.pairs()
+    np.testing.assert_array_equal(gi.cpu().numpy(), in_idx)
+    np.testing.assert_array_equal(go.cpu().numpy(), out_idx)
+    perm = m.schedule().cpu().numpy()
+    assert np.array_equal(np.sort(perm), np.arange(w.n))
+
+
+def test_map_shuffled_rows(oracle_mod):
+    w = workload("shell2")
+    rng = np.random.default_rng(1)
+    coords = w.coords[rng.permutation(w.n)]
+    m = smc.build_map(torch.from_numpy(coords).cuda(), w.grid, batch=2)
+    np.testing.assert_array_equal(m.nbr().cpu().numpy(), oracle_mod.neighbour_map(coords, w.grid))
+
+
+def test_map_wide_keys(oracle_mod):
+    """batch * Z * Y * X above 2^32 takes the two-word hash slots."""
+    rng = np.random.default_rng(2)
+    grid = (2048, 2048, 2048)
+    base = rng.integers(1, 2040, size=(300, 3))
+    pts = {tuple(p + o) for p in base for o in np.argwhere(np.ones((2, 2, 2)))}
+    zyx = np.array(sorted(pts), dtype=np.int32)
+    coords = np.concatenate([np.zeros((len(zyx), 1), np.int32), zyx], axis=1)
+    coords = np.concatenate([coords, coords + np.array([1, 0, 0, 0], np.int32)])
+    m = smc.build_map(torch.from_numpy(coords).cuda(), grid, batch=2)
+    np.testing.assert_array_equal(m.nbr().cpu().numpy(), oracle_mod.neighbour_map(coords, grid))
+
+
+def test_map_empty_and_single():
+    m = smc.build_map(torch.zeros((0, 4), dtype=torch.int32, device="cuda"), (4, 4, 4), batch=1)
+    assert m.n == 0 and m.counts == [0] * 27
+    out = smc.conv(m, torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda"),
+                   torch.zeros((64, 3, 3, 3, 64), dtype=torch.bfloat16, device="cuda"))
+    assert out.shape == (0, 64)
+    one = smc.build_map(torch.tensor([[0, 2, 2, 2]], dtype=torch.int32, device="cuda"), (5, 5, 5), batch=1)
+    nbr = one.nbr().cpu().numpy()
+    assert nbr[0, 13] == 0 and (np.delete(nbr[0], 13) == -1).all()
+
+
+def test_map_errors():
+    def err_of(coords, grid=(8, 8, 8), batch=1):
+        with pytest.raises(smc.SmcError) as e:
+            smc.build_map(torch.tensor(coords, dtype=torch.int32, device="cuda"), grid, batch=batch)
+        return e.value.name
+
+    assert err_of([[0, 1, 1, 1], [0, 2, 2, 2], [0, 1, 1, 1]]) == "SMC_E_DUPLICATE"
+    assert err_of([[0, 8, 0, 0]]) == "SMC_E_RANGE"
+    assert err_of([[0, 0, -1, 0]]) == "SMC_E_RANGE"
+    assert err_of([[1, 0, 0, 0]], batch=1) == "SMC_E_RANGE"
+    coords = [[0, z, y, x] for z in range(4) for y in range(4) for x in range(4)]
+    smc.set_hash_capacity(16)
+    try:
+        assert err_of(coords) == "SMC_E_CAPACITY"
+    finally:
+        smc.set_hash_capacity(0)
+    m = smc.build_map(torch.tensor(coords, dtype=torch.int32, device="cuda"), (8, 8, 8), batch=1)
+    assert m.counts[13] == 64
+    smc.status()
+
+
+# ------------------------------------------------------------------ conv
+def _layer(w, dtype, layer=0, ksize=3, cin=None, cout=None):
+    return S.layer_tensors(w, dtype, layer, ksize, cin, cout)
+
+
+def _conv_pair(oracle_mod, w, m, dtype, f, wt, b, ksize, orientation, rows=None):
+    out = smc.conv(m, dev(f, dtype), dev(wt, dtype), dev(b, dtype), ksize=ksize, orientation=orientation)
+    smc.status()
+    got = host(out)
+    ref = oracle_mod.conv(w.coords, w.grid, f, wt, b, ksize, orientation, rows=rows, threads=THREADS)
+    return (got if rows is None else got[rows]), ref
+
+
+@pytest.mark.parametrize("ksize,orientation", [(3, 1), (3, -1), (1, 1)])
+def test_conv_tiny_f32(oracle_mod, ksize, orientation):
+    w = workload("tiny")
+    m = build(w)
+    f, wt, b = _layer(w, "f32", 0, ksize)
+    got, ref = _conv_pair(oracle_mod, w, m, "f32", f, wt, b, ksize, orientation)
+    check_close(got, ref, "f32", f"tiny k={ksize} s={orientation}")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_conv_shell2_stacked(oracle_mod, dtype):
+    """One map reused by 4 stacked k=3 layers; each layer is checked against
+    the oracle fed the GPU's own (rounded) input to that layer."""
+    w = workload("shell2")
+    m = build(w, key=("shell2", dtype))
+    assert build(w, key=("shell2", dtype)) is m
+    x = _layer(w, dtype, 0)[0]
+    for layer in range(4):
+        _, wt, b = _layer(w, dtype, layer)
+        xt = dev(x, dtype)
+        out = smc.conv(m, xt, dev(wt, dtype), dev(b, dtype))
+        got = host(out)
+        ref = oracle_mod.conv(w.coords, w.grid, x, wt, b, 3, 1, threads=THREADS)
+        check_close(got, ref, dtype, f"shell2 {dtype} layer {layer}")
+        x = got.astype(np.float32)
+    smc.status()
+
+
+@pytest.mark.parametrize("orientation", [1, -1])
+def test_conv_shells6_bf16(oracle_mod, orientation):
+    w = workload("shells6")
+    m = build(w)
+    f, wt, b = _layer(w, "bf16")
+    rows = sample_rows(w.n, 8192, 3)
+    got, ref = _conv_pair(oracle_mod, w, m, "bf16", f, wt, b, 3, orientation, rows)
+    check_close(got, ref, "bf16", f"shells6 s={orientation}")
+
+
+def test_conv_full128_bf16_sampled(oracle_mod):
+    w = workload("full128")
+    m = build(w)
+    f, wt, b = _layer(w, "bf16")
+    rows = sample_rows(w.n, 4096, 4)
+    got, ref = _conv_pair(oracle_mod, w, m, "bf16", f, wt, b, 3, 1, rows)
+    check_close(got, ref, "bf16", "full128")
+
+
+def test_conv_varlen4_f16_k3_then_k1(oracle_mod):
+    w = workload("varlen4")
+    m = build(w, key="varlen4")
+    f, wt, b = _layer(w, "f16", 0, 3)
+    rows = sample_rows(w.n, 4096, 5)
+    out3 = smc.conv(m, dev(f, "f16"), dev(wt, "f16"), dev(b, "f16"), ksize=3)
+    got3 = host(out3)
+    ref3 = oracle_mod.conv(w.coords, w.grid, f, wt, b, 3, 1, rows=rows, threads=THREADS)
+    check_close(got3[rows], ref3, "f16", "varlen4 k=3")
+    x = got3.astype(np.float32)
+    _, w1, b1 = _layer(w, "f16", 1, 1)
+    out1 = smc.conv(build(w, key="varlen4"), out3, dev(w1, "f16"), dev(b1, "f16"), ksize=1)
+    ref1 = oracle_mod.conv(w.coords, w.grid, x, w1, b1, 1, 1, rows=rows, threads=THREADS)
+    check_close(host(out1)[rows], ref1, "f16", "varlen4 k=1")
+    smc.status()
+
+
+@pytest.mark.parametrize("stage", [0, 1, 2, 3])
+def test_conv_decoder_stage(oracle_mod, stage):
+    """Decoder stack: 10 stacked bf16 k=3 layers on one map; sampled rows of
+    every layer checked against the oracle on that layer's actual input."""
+    w = workload(f"decoder{stage}")
+    m = build(w)
+    rows = sample_rows(w.n, 1024 if w.cin >= 256 else 2048, 10 + stage)
+    x = _layer(w, "bf16", 0)[0]
+    xt = dev(x, "bf16")
+    for layer in range(10):
+        _, wt, b = _layer(w, "bf16", layer)
+        out = smc.conv(m, xt, dev(wt, "bf16"), dev(b, "bf16"))
+        if layer in (0, 4, 9):
+            ref = oracle_mod.conv(w.coords, w.grid, host(xt), wt, b, 3, 1, rows=rows, threads=THREADS)
+            got = host(out)
+            check_close(got if rows is None else got[rows], ref, "bf16", f"decoder{stage} layer {layer}")
+        xt = out
+    smc.status()
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("orientation", [1, -1])
+def test_conv_small_integers_bit_exact(oracle_mod, dtype, orientation):
+    """Inputs in {-1, 0, 1}: every partial sum is a small integer, so the
+    result is exact in any accumulation order and must match bit for bit."""
+    w = workload("shell2")
+    m = build(w)
+    rng = np.random.default_rng(21)
+    cin, cout = 64, 64
+    f = S.small_integer_values((w.n, cin), rng) * (rng.random((w.n, cin)) < 0.3)
+    wt = S.small_integer_values((cout, 3, 3, 3, cin), rng) * (rng.random((cout, 3, 3, 3, cin)) < 0.3)
+    b = S.small_integer_values((cout,), rng)
+    got, ref = _conv_pair(oracle_mod, w, m, dtype, f.astype(np.float32), wt.astype(np.float32),
+                          b.astype(np.float32), 3, orientation)
+    assert np.abs(ref).max() <= 256
+    np.testing.assert_array_equal(got, ref)
+
+
+@pytest.mark.parametrize("cin,cout", [(64, 16), (64, 512), (96, 48), (48, 64), (200, 24), (128, 272)])
+def test_conv_channel_shapes_bf16(oracle_mod, cin, cout):
+    """Tensor-core path with ragged K blocks, narrow and split N tiles; shapes
+    outside its limits run on the FMA kernel; all must meet the same bar."""
+    w = workload("shell2")
+    m = build(w)
+    f, wt, b = _layer(w, "bf16", 7, 3, cin, cout)
+    rows = sample_rows(w.n, 3000, 6)
+    for s in (1, -1):
+        got, ref = _conv_pair(oracle_mod, w, m, "bf16", f, wt, b, 3, s, rows)
+        check_close(got, ref, "bf16", f"cin={cin} cout={cout} s={s}")
+
+
+def test_conv_ragged_tail_and_no_bias(oracle_mod):
+    w = workload("shell2")
+    coords = w.coords[: 128 * 5 + 37]
+    sub = S.Workload("ragged", coords, w.grid, 64, 64, ("bf16",))
+    m = build(sub)
+    f, wt, _ = _layer(sub, "bf16", 3)
+    for dtype in ("bf16", "f32"):
+        out = smc.conv(m, dev(f, dtype), dev(wt, dtype), None)
+        ref = oracle_mod.conv(coords, w.grid, f, wt, None, 3, 1)
+        check_close(host(out), ref, dtype, f"ragged {dtype}")
+    smc.status()
+
+
+def test_conv_errors():
+    w = workload("tiny")
+    m = build(w)
+    f = torch.zeros((w.n, 16), device="cuda")
+    wt = torch.zeros((16, 3, 3, 3, 16), device="cuda")
+    with pytest.raises(smc.SmcError) as e:
+        smc.conv(m, f, wt, out=f)
+    assert e.value.name == "SMC_E_ALIAS"
+    lib = smc.lib()
+    import ctypes
+    rc = lib.smc_conv(m.handle, ctypes.c_void_p(f.data_ptr()), 16, ctypes.c_void_p(wt.data_ptr()), None,
+                      ctypes.c_void_p(f.data_ptr() + 10 ** 6), 16, 2, 1, 0, None)
+    assert rc == -1  # ksize 2
+    rc = lib.smc_conv(m.handle, ctypes.c_void_p(f.data_ptr()), 16, ctypes.c_void_p(wt.data_ptr()), None,
+                      ctypes.c_void_p(f.data_ptr() + 10 ** 6), 16, 3, 0, 0, None)
+    assert rc == -1  # orientation 0
+    rc = lib.smc_conv(m.handle, ctypes.c_void_p(f.data_ptr()), 16, ctypes.c_void_p(wt.data_ptr()), None,
+                      ctypes.c_void_p(f.data_ptr() + 10 ** 6), 16, 3, 1, 7, None)
+    assert rc == -4  # dtype
+    smc.status()
