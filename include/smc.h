@@ -83,11 +83,29 @@ enum {
  * the sites, the int32 [n, 27] neighbour map (-1 = absent), the per-offset
  * pair lists (stable compaction of each map column, ascending output row),
  * and the tile schedule used by the tensor-core conv.  coords may be freed
- * once the call returns.  Errors: SMC_E_ARG, SMC_E_ALIGN, SMC_E_RANGE,
+ * once the call returns.  Device memory comes from a per-device
+ * stream-ordered pool owned by the library that keeps freed memory for
+ * later builds.  Errors: SMC_E_ARG, SMC_E_ALIGN, SMC_E_RANGE,
  * SMC_E_DUPLICATE, SMC_E_CAPACITY, SMC_E_OOM, SMC_E_CUDA.
  */
 SMC_API int smc_build_map(const int32_t* coords, int64_t n, int32_t batch, const int32_t grid[3],
                   void* stream, smc_map** out);
+
+/*
+ * smc_build_map_async -- the same build with no synchronisation: every step
+ * is enqueued on `stream` and the handle returns at once.  Argument errors
+ * are returned immediately; errors found on the device (SMC_E_RANGE,
+ * SMC_E_DUPLICATE, SMC_E_CAPACITY) are returned by smc_map_wait and by every
+ * later smc_map_* query, and smc_conv refuses a map known to have failed.
+ * A conv enqueued before the outcome is known reads a map whose entries are
+ * always -1 or valid rows, so it stays memory-safe.  coords must stay valid
+ * until the build has run on `stream`.
+ */
+SMC_API int smc_build_map_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t grid[3],
+                        void* stream, smc_map** out);
+
+/* Block until the map's build has finished; return its outcome. */
+SMC_API int smc_map_wait(const smc_map* map);
 
 /*
  * smc_conv -- one submanifold convolution over a built map.
@@ -104,7 +122,9 @@ SMC_API int smc_build_map(const int32_t* coords, int64_t n, int32_t batch, const
  *          SMC_F16 (fp32 accumulation, bias added in fp32, output rounded to
  *          nearest even).
  *
- * Asynchronous on `stream`; no synchronisation.  bf16/fp16 with cin a
+ * Asynchronous on `stream`; no synchronisation.  When `stream` is not the
+ * stream the map was built on, the conv first waits (on the device) for the
+ * build to finish.  bf16/fp16 with cin a
  * multiple of 16 and at least 64, cout a multiple of 16 and 16-byte aligned
  * buffers run on the tcgen05 tensor-core kernel; every other shape runs on
  * the FMA kernel.  A bounded device-side wait that runs out is reported by
@@ -139,7 +159,9 @@ SMC_API int smc_map_pairs(const smc_map* map, const int32_t** in_idx, const int3
  */
 SMC_API int smc_map_schedule(const smc_map* map, const int32_t** perm);
 
-/* Release a map.  Work on other streams that reads it must have completed. */
+/* Release a map (its memory returns to the library's pool, ordered on the
+ * build stream).  Work on other streams that reads the map must have
+ * completed. */
 SMC_API int smc_free_map(smc_map* map);
 
 /* Synchronise `stream`, then return and clear the device-side error word

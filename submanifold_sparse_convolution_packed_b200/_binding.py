@@ -29,6 +29,7 @@ EXPORTS = [
     "smc_build_map", "smc_conv", "smc_map_info", "smc_map_nbr", "smc_map_pairs",
     "smc_map_schedule", "smc_free_map", "smc_status", "smc_strerror",
     "smc_set_hash_capacity", "smc_set_profiling", "smc_map_timing", "smc_kernel_launches",
+    "smc_build_map_async", "smc_map_wait",
 ]
 
 
@@ -54,6 +55,8 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         P, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
         L.smc_build_map.argtypes = [P, i64, i32, P, P, ctypes.POINTER(P)]
+        L.smc_build_map_async.argtypes = [P, i64, i32, P, P, ctypes.POINTER(P)]
+        L.smc_map_wait.argtypes = [P]
         L.smc_conv.argtypes = [P, P, i64, P, P, P, i64, i32, i32, i32, P]
         L.smc_map_info.argtypes = [P, P, P]
         L.smc_map_nbr.argtypes = [P, ctypes.POINTER(P)]
@@ -109,12 +112,29 @@ class Map:
         self.batch = batch
         self.grid = tuple(int(g) for g in grid)
         self.device = device
-        counts = (ctypes.c_int64 * 27)()
-        _check(lib().smc_map_info(self._h, None, counts), "smc_map_info")
-        self.counts = [int(c) for c in counts]
-        offs = (ctypes.c_int64 * 28)()
-        _check(lib().smc_map_pairs(self._h, None, None, offs), "smc_map_pairs")
-        self.offsets = [int(o) for o in offs]
+        self._counts = None
+        self._offsets = None
+
+    def wait(self) -> "Map":
+        """Block until the build has finished; raise SmcError if it failed."""
+        _check(lib().smc_map_wait(self.handle), "smc_build_map")
+        return self
+
+    @property
+    def counts(self):
+        if self._counts is None:
+            c = (ctypes.c_int64 * 27)()
+            _check(lib().smc_map_info(self.handle, None, c), "smc_map_info")
+            self._counts = [int(x) for x in c]
+        return self._counts
+
+    @property
+    def offsets(self):
+        if self._offsets is None:
+            o = (ctypes.c_int64 * 28)()
+            _check(lib().smc_map_pairs(self.handle, None, None, o), "smc_map_pairs")
+            self._offsets = [int(x) for x in o]
+        return self._offsets
 
     @property
     def handle(self) -> ctypes.c_void_p:
@@ -173,10 +193,12 @@ _cache: Dict[Hashable, Map] = {}
 
 
 def build_map(coords: torch.Tensor, grid: Sequence[int], batch: Optional[int] = None,
-              key: Optional[Hashable] = None, stream=None) -> Map:
+              key: Optional[Hashable] = None, stream=None, sync: bool = True) -> Map:
     """Build (or fetch from the cache under `key`) the map of int32 [N, 4]
     (b, z, y, x) coordinates on a (Z, Y, X) grid.  Like spconv's indice_key,
-    `key` names a coordinate set so every conv on it reuses one map."""
+    `key` names a coordinate set so every conv on it reuses one map.  With
+    sync=False the build is only enqueued (smc_build_map_async); device-side
+    input errors then surface at Map.wait() or the first query."""
     if key is not None and key in _cache:
         return _cache[key]
     if coords.dtype != torch.int32 or coords.dim() != 2 or coords.shape[1] != 4:
@@ -189,9 +211,9 @@ def build_map(coords: torch.Tensor, grid: Sequence[int], batch: Optional[int] = 
         batch = int(coords[:, 0].max().item()) + 1 if n else 1
     g = (ctypes.c_int32 * 3)(*[int(x) for x in grid])
     h = ctypes.c_void_p()
+    fn = lib().smc_build_map if sync else lib().smc_build_map_async
     with torch.cuda.device(coords.device):
-        _check(lib().smc_build_map(_ptr(coords), n, int(batch), g, _stream(stream), ctypes.byref(h)),
-               "smc_build_map")
+        _check(fn(_ptr(coords), n, int(batch), g, _stream(stream), ctypes.byref(h)), "smc_build_map")
     m = Map(h, n, int(batch), grid, coords.device)
     if key is not None:
         _cache[key] = m

@@ -10,10 +10,18 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <vector>
 
-#include "../../include/smc.h"
+#include "smc.h"
 #include "common.cuh"
 #include "kernels.h"
+
+// Status block a build copies back to the host: error bits and pair offsets.
+struct HostSlot {
+  uint32_t err;
+  uint32_t pad;
+  int64_t info[28];
+};
 
 struct smc_map {
   int device;
@@ -21,14 +29,22 @@ struct smc_map {
   int64_t n;
   int32_t batch;
   int32_t grid[3];
-  int64_t counts[27];
-  int64_t offsets[28];
   int32_t* nbr;
   int32_t* in_idx;
   int32_t* out_idx;
   int32_t* perm;
-  void* keep;  // one allocation holding nbr, pairs and perm
-  float ms[2];
+  uint32_t* tile_mask;
+  void* keep;           // one allocation holding nbr, pairs, schedule and tile masks
+  cudaEvent_t done;     // recorded after the status block is copied back
+  cudaEvent_t prof[3];  // optional timing events
+  HostSlot* slot;       // pinned status block
+  // filled in when the build is first waited on
+  mutable std::mutex mu;
+  mutable bool resolved;
+  mutable int status;
+  mutable int64_t counts[27];
+  mutable int64_t offsets[28];
+  mutable float ms[2];
 };
 
 namespace {
@@ -37,14 +53,19 @@ std::atomic<int64_t> g_capacity_override{0};
 std::atomic<long long> g_launches{0};
 std::atomic<int32_t> g_profiling{0};
 
-// Per-device error word of the conv kernels (bounded-wait timeouts).
 constexpr int kMaxDevices = 64;
+
+// Per-device error word of the conv kernels (bounded-wait timeouts).
 uint32_t* g_status[kMaxDevices] = {};
-std::mutex g_status_mu;
+// Per-device stream-ordered memory pool that keeps its memory between builds
+// (the default pool returns memory to the driver at every synchronisation,
+// which made each build re-map its buffers).
+cudaMemPool_t g_pool[kMaxDevices] = {};
+std::mutex g_dev_mu;
 
 uint32_t* device_status(int dev) {
   if (dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lk(g_status_mu);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
   if (!g_status[dev]) {
     void* p = nullptr;
     if (cudaMalloc(&p, 256) != cudaSuccess) return nullptr;
@@ -52,6 +73,47 @@ uint32_t* device_status(int dev) {
     g_status[dev] = static_cast<uint32_t*>(p);
   }
   return g_status[dev];
+}
+
+cudaMemPool_t device_pool(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_pool[dev]) {
+    cudaMemPoolProps props;
+    std::memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
+    uint64_t keep_all = ~0ull;
+    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep_all);
+    g_pool[dev] = pool;
+  }
+  return g_pool[dev];
+}
+
+// Pinned host status blocks, handed out from chunks of 256.
+std::mutex g_slot_mu;
+std::vector<HostSlot*> g_free_slots;
+
+HostSlot* take_slot() {
+  std::lock_guard<std::mutex> lk(g_slot_mu);
+  if (g_free_slots.empty()) {
+    void* p = nullptr;
+    if (cudaMallocHost(&p, 256 * sizeof(HostSlot)) != cudaSuccess) return nullptr;
+    HostSlot* s = static_cast<HostSlot*>(p);
+    for (int i = 0; i < 256; ++i) g_free_slots.push_back(s + i);
+  }
+  HostSlot* s = g_free_slots.back();
+  g_free_slots.pop_back();
+  return s;
+}
+
+void give_slot(HostSlot* s) {
+  if (!s) return;
+  std::lock_guard<std::mutex> lk(g_slot_mu);
+  g_free_slots.push_back(s);
 }
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -76,6 +138,197 @@ bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
   if (!a || !b || na == 0 || nb == 0) return false;
   const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
   return a0 < b0 + nb && b0 < a0 + na;
+}
+
+void release_map(smc_map* m) {
+  if (!m) return;
+  int cur = 0;
+  cudaGetDevice(&cur);
+  if (cur != m->device) cudaSetDevice(m->device);
+  if (m->done) cudaEventSynchronize(m->done);  // the status copy must land before the slot is reused
+  if (m->keep) cudaFreeAsync(m->keep, m->stream);
+  if (m->done) cudaEventDestroy(m->done);
+  for (auto& e : m->prof)
+    if (e) cudaEventDestroy(e);
+  give_slot(m->slot);
+  if (cur != m->device) cudaSetDevice(cur);
+  cudaGetLastError();
+  delete m;
+}
+
+// Wait for a build to finish and record its outcome (once).
+int resolve(const smc_map* m) {
+  std::lock_guard<std::mutex> lk(m->mu);
+  if (m->resolved) return m->status;
+  int rc = SMC_OK;
+  if (m->done && cudaEventSynchronize(m->done) != cudaSuccess) {
+    cudaGetLastError();
+    rc = SMC_E_CUDA;
+  } else if (m->slot) {
+    const uint32_t err = m->slot->err;
+    if (err & smc::kErrRange) rc = SMC_E_RANGE;
+    else if (err & smc::kErrDuplicate) rc = SMC_E_DUPLICATE;
+    else if (err & smc::kErrCapacity) rc = SMC_E_CAPACITY;
+    for (int d = 0; d < 28; ++d) m->offsets[d] = m->slot->info[d];
+    for (int d = 0; d < 27; ++d) m->counts[d] = m->slot->info[d + 1] - m->slot->info[d];
+  }
+  if (rc == SMC_OK && m->prof[0]) {
+    cudaEventElapsedTime(&m->ms[0], m->prof[0], m->prof[1]);
+    cudaEventElapsedTime(&m->ms[1], m->prof[1], m->prof[2]);
+  }
+  m->status = rc;
+  m->resolved = true;
+  return rc;
+}
+
+// Enqueue a whole map build on `s`; no synchronisation.
+int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t grid[3], cudaStream_t s,
+                smc_map** out) {
+  if (!out) return SMC_E_ARG;
+  *out = nullptr;
+  if (!grid || n < 0 || batch < 1 || (n > 0 && !coords)) return SMC_E_ARG;
+  if (grid[0] < 1 || grid[1] < 1 || grid[2] < 1) return SMC_E_ARG;
+  if (n >= (1ll << 31) - 1) return SMC_E_ARG;  // rows are int32
+  if (n > 0 && (reinterpret_cast<uintptr_t>(coords) & 15u)) return SMC_E_ALIGN;
+  const double sites = static_cast<double>(batch) * grid[0] * grid[1] * grid[2];
+  if (sites >= 4.6e18) return SMC_E_ARG;
+  if (pending_cuda_error() != SMC_OK) return SMC_E_CUDA;
+
+  smc_map* m = new (std::nothrow) smc_map();
+  if (!m) return SMC_E_OOM;
+  cudaGetDevice(&m->device);
+  m->stream = s;
+  m->n = n;
+  m->batch = batch;
+  for (int i = 0; i < 3; ++i) m->grid[i] = grid[i];
+  if (n == 0) {
+    m->resolved = true;
+    *out = m;
+    return SMC_OK;
+  }
+  cudaMemPool_t pool = device_pool(m->device);
+  m->slot = take_slot();
+  if (!pool || !m->slot || cudaEventCreateWithFlags(&m->done, cudaEventDisableTiming) != cudaSuccess) {
+    cudaGetLastError();
+    release_map(m);
+    return SMC_E_OOM;
+  }
+
+  // ---- sizes
+  const bool wide = sites > 4294967294.0;  // packed slots need keys < 2^32 - 1
+  int lg = 4;
+  const int64_t forced = g_capacity_override.load();
+  const int64_t want = forced > 0 ? forced : 2 * n;
+  while ((1ll << lg) < want) ++lg;
+  const int64_t cap = 1ll << lg;
+  const int nb = smc::map_nblocks(n);
+  const int64_t Lmap = 27ll * nb;
+  const int nblk = smc::radix_nblocks(n);
+  const int64_t Lrad = static_cast<int64_t>(smc::radix_bins()) * nblk;
+  const int64_t pair_cap = 27ll * n;
+
+  Carve keep;
+  const size_t o_nbr = keep.take<int32_t>(27ull * n);
+  const size_t o_in = keep.take<int32_t>(pair_cap);
+  const size_t o_out = keep.take<int32_t>(pair_cap);
+  const size_t o_perm = keep.take<int32_t>(n);
+  const size_t o_tmask = keep.take<uint32_t>((n + smc::kTileRows - 1) / smc::kTileRows);
+  Carve tmp;
+  const size_t o_table = tmp.take<unsigned long long>(wide ? 2 * cap : cap);
+  const size_t o_err = tmp.take<uint32_t>(1);
+  const size_t o_info = tmp.take<int64_t>(28);
+  const size_t o_total = tmp.take<int64_t>(1);
+  const size_t o_gkey = tmp.take<uint32_t>(n);
+  const size_t o_hmask = tmp.take<uint32_t>(n);
+  const size_t o_bc = tmp.take<int32_t>(Lmap);
+  const size_t o_bo = tmp.take<int64_t>(Lmap);
+  const size_t o_sp = tmp.take<int64_t>(smc::scan_partials_len(Lmap > Lrad ? Lmap : Lrad));
+  const size_t o_hist = tmp.take<int32_t>(Lrad);
+  const size_t o_hoff = tmp.take<int64_t>(Lrad);
+  const size_t o_ktmp = tmp.take<uint32_t>(n);
+  const size_t o_vtmp = tmp.take<int32_t>(n);
+
+  void* tp = nullptr;
+  if (cudaMallocFromPoolAsync(&m->keep, keep.off, pool, s) != cudaSuccess) {
+    cudaGetLastError();
+    m->keep = nullptr;
+    release_map(m);
+    return SMC_E_OOM;
+  }
+  if (cudaMallocFromPoolAsync(&tp, tmp.off, pool, s) != cudaSuccess) {
+    cudaGetLastError();
+    release_map(m);
+    return SMC_E_OOM;
+  }
+  char* K = static_cast<char*>(m->keep);
+  char* T = static_cast<char*>(tp);
+  m->nbr = reinterpret_cast<int32_t*>(K + o_nbr);
+  m->in_idx = reinterpret_cast<int32_t*>(K + o_in);
+  m->out_idx = reinterpret_cast<int32_t*>(K + o_out);
+  m->perm = reinterpret_cast<int32_t*>(K + o_perm);
+  m->tile_mask = reinterpret_cast<uint32_t*>(K + o_tmask);
+
+  if (g_profiling.load() != 0)
+    for (auto& e : m->prof) cudaEventCreate(&e);
+
+  cudaError_t ce = cudaMemsetAsync(T + o_table, 0xFF, (wide ? 2 : 1) * cap * sizeof(unsigned long long), s);
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(T + o_err, 0, sizeof(uint32_t), s);
+  if (m->prof[0]) cudaEventRecord(m->prof[0], s);
+  if (ce == cudaSuccess) {
+    smc::MapBuildArgs a;
+    a.coords = coords;
+    a.n = n;
+    a.batch = batch;
+    a.Z = grid[0];
+    a.Y = grid[1];
+    a.X = grid[2];
+    a.wide = wide;
+    a.table = reinterpret_cast<unsigned long long*>(T + o_table);
+    a.lg = lg;
+    a.err = reinterpret_cast<uint32_t*>(T + o_err);
+    a.nbr = m->nbr;
+    a.gkey = reinterpret_cast<uint32_t*>(T + o_gkey);
+    a.hmask = reinterpret_cast<uint32_t*>(T + o_hmask);
+    a.block_counts = reinterpret_cast<int32_t*>(T + o_bc);
+    a.block_offsets = reinterpret_cast<int64_t*>(T + o_bo);
+    a.scan_partials = reinterpret_cast<int64_t*>(T + o_sp);
+    a.total = reinterpret_cast<int64_t*>(T + o_total);
+    a.info = reinterpret_cast<int64_t*>(T + o_info);
+    a.in_idx = m->in_idx;
+    a.out_idx = m->out_idx;
+    ce = smc::launch_map_build(a, s);
+  }
+  if (m->prof[1]) cudaEventRecord(m->prof[1], s);
+  if (ce == cudaSuccess) {
+    smc::ScheduleArgs b;
+    b.gkey = reinterpret_cast<uint32_t*>(T + o_gkey);
+    b.n = n;
+    b.hist = reinterpret_cast<int32_t*>(T + o_hist);
+    b.hoff = reinterpret_cast<int64_t*>(T + o_hoff);
+    b.scan_partials = reinterpret_cast<int64_t*>(T + o_sp);
+    b.key_tmp = reinterpret_cast<uint32_t*>(T + o_ktmp);
+    b.val_tmp = reinterpret_cast<int32_t*>(T + o_vtmp);
+    b.perm = m->perm;
+    b.hmask = reinterpret_cast<uint32_t*>(T + o_hmask);
+    b.tile_mask = m->tile_mask;
+    ce = smc::launch_schedule(b, s);
+  }
+  if (m->prof[2]) cudaEventRecord(m->prof[2], s);
+  // the only device->host traffic: error bits and pair offsets, into pinned memory
+  if (ce == cudaSuccess) ce = cudaMemcpyAsync(&m->slot->err, T + o_err, sizeof(uint32_t), cudaMemcpyDeviceToHost, s);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpyAsync(m->slot->info, T + o_info, 28 * sizeof(int64_t), cudaMemcpyDeviceToHost, s);
+  cudaFreeAsync(tp, s);
+  if (ce == cudaSuccess) ce = cudaEventRecord(m->done, s);
+  if (ce != cudaSuccess) {
+    cudaGetLastError();
+    cudaStreamSynchronize(s);
+    cudaGetLastError();
+    release_map(m);
+    return SMC_E_CUDA;
+  }
+  *out = m;
+  return SMC_OK;
 }
 
 }  // namespace
@@ -115,168 +368,26 @@ int smc_set_profiling(int32_t on) {
   return SMC_OK;
 }
 
+int smc_build_map_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t grid[3], void* stream,
+                        smc_map** out) {
+  return build_async(coords, n, batch, grid, static_cast<cudaStream_t>(stream), out);
+}
+
+int smc_map_wait(const smc_map* map) {
+  if (!map) return SMC_E_ARG;
+  return resolve(map);
+}
+
 int smc_build_map(const int32_t* coords, int64_t n, int32_t batch, const int32_t grid[3], void* stream,
                   smc_map** out) {
-  if (!out) return SMC_E_ARG;
-  *out = nullptr;
-  if (!grid || n < 0 || batch < 1 || (n > 0 && !coords)) return SMC_E_ARG;
-  if (grid[0] < 1 || grid[1] < 1 || grid[2] < 1) return SMC_E_ARG;
-  if (n >= (1ll << 31) - 1) return SMC_E_ARG;  // rows are int32
-  if (n > 0 && (reinterpret_cast<uintptr_t>(coords) & 15u)) return SMC_E_ALIGN;
-  const double sites = static_cast<double>(batch) * grid[0] * grid[1] * grid[2];
-  if (sites >= 4.6e18) return SMC_E_ARG;
-  if (pending_cuda_error() != SMC_OK) return SMC_E_CUDA;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-
-  smc_map* m = new (std::nothrow) smc_map();
-  if (!m) return SMC_E_OOM;
-  std::memset(m, 0, sizeof(*m));
-  cudaGetDevice(&m->device);
-  m->stream = s;
-  m->n = n;
-  m->batch = batch;
-  for (int i = 0; i < 3; ++i) m->grid[i] = grid[i];
-  if (n == 0) {
-    *out = m;
-    return SMC_OK;
-  }
-
-  // ---- sizes
-  const bool wide = sites > 4294967294.0;  // packed slots need keys < 2^32 - 1
-  int lg = 4;
-  const int64_t forced = g_capacity_override.load();
-  const int64_t want = forced > 0 ? forced : 2 * n;
-  while ((1ll << lg) < want) ++lg;
-  const int64_t cap = 1ll << lg;
-  const int nb = smc::map_nblocks(n);
-  const int64_t Lmap = 27ll * nb;
-  const int nblk = smc::radix_nblocks(n);
-  const int64_t Lrad = static_cast<int64_t>(smc::radix_bins()) * nblk;
-  const int64_t pair_cap = 27ll * n;
-
-  Carve keep;
-  const size_t o_nbr = keep.take<int32_t>(27ull * n);
-  const size_t o_in = keep.take<int32_t>(pair_cap);
-  const size_t o_out = keep.take<int32_t>(pair_cap);
-  const size_t o_perm = keep.take<int32_t>(n);
-  Carve tmp;
-  const size_t o_table = tmp.take<unsigned long long>(wide ? 2 * cap : cap);
-  const size_t o_err = tmp.take<uint32_t>(1);
-  const size_t o_info = tmp.take<int64_t>(28);
-  const size_t o_total = tmp.take<int64_t>(1);
-  const size_t o_gkey = tmp.take<uint32_t>(n);
-  const size_t o_bc = tmp.take<int32_t>(Lmap);
-  const size_t o_bo = tmp.take<int64_t>(Lmap);
-  const size_t o_sp = tmp.take<int64_t>(smc::scan_partials_len(Lmap > Lrad ? Lmap : Lrad));
-  const size_t o_hist = tmp.take<int32_t>(Lrad);
-  const size_t o_hoff = tmp.take<int64_t>(Lrad);
-  const size_t o_ktmp = tmp.take<uint32_t>(n);
-  const size_t o_vtmp = tmp.take<int32_t>(n);
-
-  void* kp = nullptr;
-  void* tp = nullptr;
-  if (cudaMallocAsync(&kp, keep.off, s) != cudaSuccess) {
-    cudaGetLastError();
-    delete m;
-    return SMC_E_OOM;
-  }
-  if (cudaMallocAsync(&tp, tmp.off, s) != cudaSuccess) {
-    cudaGetLastError();
-    cudaFreeAsync(kp, s);
-    delete m;
-    return SMC_E_OOM;
-  }
-  char* K = static_cast<char*>(kp);
-  char* T = static_cast<char*>(tp);
-  m->keep = kp;
-  m->nbr = reinterpret_cast<int32_t*>(K + o_nbr);
-  m->in_idx = reinterpret_cast<int32_t*>(K + o_in);
-  m->out_idx = reinterpret_cast<int32_t*>(K + o_out);
-  m->perm = reinterpret_cast<int32_t*>(K + o_perm);
-
-  const bool prof = g_profiling.load() != 0;
-  cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};
-  if (prof)
-    for (auto& e : ev) cudaEventCreate(&e);
-
-  int rc = SMC_OK;
-  cudaError_t ce = cudaMemsetAsync(T + o_table, 0xFF, (wide ? 2 : 1) * cap * sizeof(unsigned long long), s);
-  if (ce == cudaSuccess) ce = cudaMemsetAsync(T + o_err, 0, sizeof(uint32_t), s);
-  if (prof) cudaEventRecord(ev[0], s);
-  if (ce == cudaSuccess) {
-    smc::MapBuildArgs a;
-    a.coords = coords;
-    a.n = n;
-    a.batch = batch;
-    a.Z = grid[0];
-    a.Y = grid[1];
-    a.X = grid[2];
-    a.wide = wide;
-    a.table = reinterpret_cast<unsigned long long*>(T + o_table);
-    a.lg = lg;
-    a.err = reinterpret_cast<uint32_t*>(T + o_err);
-    a.nbr = m->nbr;
-    a.gkey = reinterpret_cast<uint32_t*>(T + o_gkey);
-    a.block_counts = reinterpret_cast<int32_t*>(T + o_bc);
-    a.block_offsets = reinterpret_cast<int64_t*>(T + o_bo);
-    a.scan_partials = reinterpret_cast<int64_t*>(T + o_sp);
-    a.total = reinterpret_cast<int64_t*>(T + o_total);
-    a.info = reinterpret_cast<int64_t*>(T + o_info);
-    a.in_idx = m->in_idx;
-    a.out_idx = m->out_idx;
-    ce = smc::launch_map_build(a, s);
-  }
-  if (prof) cudaEventRecord(ev[1], s);
-  if (ce == cudaSuccess) {
-    smc::ScheduleArgs b;
-    b.gkey = reinterpret_cast<uint32_t*>(T + o_gkey);
-    b.n = n;
-    b.hist = reinterpret_cast<int32_t*>(T + o_hist);
-    b.hoff = reinterpret_cast<int64_t*>(T + o_hoff);
-    b.scan_partials = reinterpret_cast<int64_t*>(T + o_sp);
-    b.key_tmp = reinterpret_cast<uint32_t*>(T + o_ktmp);
-    b.val_tmp = reinterpret_cast<int32_t*>(T + o_vtmp);
-    b.perm = m->perm;
-    ce = smc::launch_schedule(b, s);
-  }
-  if (prof) cudaEventRecord(ev[2], s);
-  // one device->host read: error bits and pair offsets
-  struct {
-    uint32_t err;
-    uint32_t pad;
-    int64_t info[28];
-  } h;
-  std::memset(&h, 0, sizeof(h));
-  if (ce == cudaSuccess) ce = cudaMemcpyAsync(&h.err, T + o_err, sizeof(uint32_t), cudaMemcpyDeviceToHost, s);
-  if (ce == cudaSuccess) ce = cudaMemcpyAsync(h.info, T + o_info, 28 * sizeof(int64_t), cudaMemcpyDeviceToHost, s);
-  cudaFreeAsync(tp, s);
-  if (ce == cudaSuccess) ce = cudaStreamSynchronize(s);
-  if (ce != cudaSuccess) {
-    cudaGetLastError();
-    rc = SMC_E_CUDA;
-  } else if (h.err & smc::kErrRange) {
-    rc = SMC_E_RANGE;
-  } else if (h.err & smc::kErrDuplicate) {
-    rc = SMC_E_DUPLICATE;
-  } else if (h.err & smc::kErrCapacity) {
-    rc = SMC_E_CAPACITY;
-  }
-  if (prof) {
-    if (rc == SMC_OK) {
-      cudaEventElapsedTime(&m->ms[0], ev[0], ev[1]);
-      cudaEventElapsedTime(&m->ms[1], ev[1], ev[2]);
-    }
-    for (auto& e : ev) cudaEventDestroy(e);
-  }
+  smc_map* m = nullptr;
+  int rc = build_async(coords, n, batch, grid, static_cast<cudaStream_t>(stream), &m);
+  if (rc != SMC_OK) return rc;
+  rc = resolve(m);
   if (rc != SMC_OK) {
-    cudaFreeAsync(kp, s);
-    cudaStreamSynchronize(s);
-    cudaGetLastError();
-    delete m;
+    release_map(m);
     return rc;
   }
-  for (int d = 0; d < 28; ++d) m->offsets[d] = h.info[d];
-  for (int d = 0; d < 27; ++d) m->counts[d] = h.info[d + 1] - h.info[d];
   *out = m;
   return SMC_OK;
 }
@@ -291,6 +402,10 @@ int smc_conv(const smc_map* map, const void* feats, int64_t cin, const void* wei
   const int64_t n = map->n;
   if (n == 0) return SMC_OK;
   if (!feats || !weight || !out) return SMC_E_ARG;
+  {
+    std::lock_guard<std::mutex> lk(map->mu);
+    if (map->resolved && map->status != SMC_OK) return map->status;
+  }
   const size_t esz = dtype == SMC_F32 ? 4 : 2;
   const int taps = ksize == 3 ? 27 : 1;
   if (ranges_overlap(out, n * cout * esz, feats, n * cin * esz) ||
@@ -309,6 +424,7 @@ int smc_conv(const smc_map* map, const void* feats, int64_t cin, const void* wei
   a.out = out;
   a.nbr = map->nbr;
   a.perm = map->perm;
+  a.tile_mask = map->tile_mask;
   a.n = n;
   a.cin = static_cast<int>(cin);
   a.cout = static_cast<int>(cout);
@@ -317,6 +433,11 @@ int smc_conv(const smc_map* map, const void* feats, int64_t cin, const void* wei
   a.dtype = dtype;
   a.err = st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dev != map->device) return SMC_E_ARG;
+  if (s != map->stream && map->done && cudaStreamWaitEvent(s, map->done, 0) != cudaSuccess) {
+    cudaGetLastError();
+    return SMC_E_CUDA;
+  }
   const cudaError_t e = smc::conv_tc_supported(a) ? smc::launch_conv_tc(a, s) : smc::launch_conv_simt(a, s);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -327,6 +448,8 @@ int smc_conv(const smc_map* map, const void* feats, int64_t cin, const void* wei
 
 int smc_map_info(const smc_map* map, int64_t* n, int64_t counts[27]) {
   if (!map) return SMC_E_ARG;
+  const int rc = resolve(map);
+  if (rc != SMC_OK) return rc;
   if (n) *n = map->n;
   if (counts)
     for (int d = 0; d < 27; ++d) counts[d] = map->counts[d];
@@ -341,6 +464,8 @@ int smc_map_nbr(const smc_map* map, const int32_t** nbr) {
 
 int smc_map_pairs(const smc_map* map, const int32_t** in_idx, const int32_t** out_idx, int64_t offsets[28]) {
   if (!map) return SMC_E_ARG;
+  const int rc = resolve(map);
+  if (rc != SMC_OK) return rc;
   if (in_idx) *in_idx = map->in_idx;
   if (out_idx) *out_idx = map->out_idx;
   if (offsets)
@@ -362,6 +487,8 @@ int smc_kernel_launches(int64_t* count) {
 
 int smc_map_timing(const smc_map* map, float ms[2]) {
   if (!map || !ms) return SMC_E_ARG;
+  const int rc = resolve(map);
+  if (rc != SMC_OK) return rc;
   ms[0] = map->ms[0];
   ms[1] = map->ms[1];
   return SMC_OK;
@@ -369,19 +496,8 @@ int smc_map_timing(const smc_map* map, float ms[2]) {
 
 int smc_free_map(smc_map* map) {
   if (!map) return SMC_OK;
-  int rc = SMC_OK;
-  if (map->keep) {
-    int cur = 0;
-    cudaGetDevice(&cur);
-    if (cur != map->device) cudaSetDevice(map->device);
-    if (cudaFreeAsync(map->keep, map->stream) != cudaSuccess) {
-      cudaGetLastError();
-      rc = SMC_E_CUDA;
-    }
-    if (cur != map->device) cudaSetDevice(cur);
-  }
-  delete map;
-  return rc;
+  release_map(map);
+  return SMC_OK;
 }
 
 int smc_status(void* stream) {

@@ -16,6 +16,7 @@ struct MapBuildArgs {
   uint32_t* err;               // error bits
   int32_t* nbr;                // [n, 27]
   uint32_t* gkey;              // [n] grouping key of the tile schedule
+  uint32_t* hmask;             // [n] 27-bit neighbour hit mask of every row
   int32_t* block_counts;       // [27, nblocks]
   int64_t* block_offsets;      // [27, nblocks]
   int64_t* scan_partials;      // scan_partials_len(27 * nblocks)
@@ -33,8 +34,12 @@ struct ScheduleArgs {
   int64_t* scan_partials; // scan_partials_len(bins * nblk)
   uint32_t* key_tmp;      // [n]
   int32_t* val_tmp;       // [n]
-  int32_t* perm;          // [n] result
+  int32_t* perm;          // [n] result: tile order
+  const uint32_t* hmask;  // [n] hit masks
+  uint32_t* tile_mask;    // [ceil(n/128)] result: OR of the hit masks of each tile's rows
 };
+
+constexpr int kTileRows = 128;  // output rows per tensor-core tile
 
 // Running count of kernels this library has launched (measurement hook).
 void count_launches(int k);
@@ -57,6 +62,7 @@ struct ConvArgs {
   void* out;            // [n, cout]
   const int32_t* nbr;   // [n, 27] (taps == 27)
   const int32_t* perm;  // [n] tile order (tensor-core kernel, taps == 27) or null
+  const uint32_t* tile_mask;  // [ceil(n/128)] taps present in each tile (taps == 27)
   int64_t n;
   int cin, cout, taps, orientation, dtype;
   uint32_t* err;

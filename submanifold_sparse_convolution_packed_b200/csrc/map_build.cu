@@ -69,11 +69,12 @@ __global__ void __launch_bounds__(256) k_insert(const int4* __restrict__ coords,
   }
 }
 
+// Linear probing from slot s (the home slot has been checked already when
+// called from the neighbour kernel); at most one pass over the table.
 template <bool kWide>
-__device__ __forceinline__ int32_t lookup(const unsigned long long* __restrict__ table, uint64_t mask,
-                                          int lg, uint64_t key) {
-  uint64_t s = slot_of(key, lg);
-  for (uint64_t probe = 0; probe <= mask; ++probe) {
+__device__ __noinline__ int32_t lookup_from(const unsigned long long* __restrict__ table, uint64_t mask,
+                                            uint64_t s, uint64_t key) {
+  for (uint64_t probe = 0; probe < mask; ++probe) {
     if (!kWide) {
       const uint64_t e = __ldg(&table[s]);
       if (e == kEmpty) return -1;
@@ -105,7 +106,8 @@ template <bool kWide>
 __global__ void __launch_bounds__(kMapBlock) k_neighbours(
     const int4* __restrict__ coords, int64_t n, int32_t Z, int32_t Y, int32_t X,
     const unsigned long long* __restrict__ table, int lg, int32_t* __restrict__ nbr,
-    uint32_t* __restrict__ gkey, int32_t* __restrict__ block_counts, int nblocks) {
+    uint32_t* __restrict__ gkey, uint32_t* __restrict__ hmask, int32_t* __restrict__ block_counts,
+    int nblocks) {
   __shared__ int32_t s_nbr[kMapBlock * kTaps];
   __shared__ int32_t s_cnt[kMapBlock / 32][kTaps];
   const uint64_t mask = (1ull << lg) - 1;
@@ -117,19 +119,48 @@ __global__ void __launch_bounds__(kMapBlock) k_neighbours(
     const int4 c = coords[v];
     const uint64_t key = site_key(c, Z, Y, X);
     const int64_t sz = static_cast<int64_t>(Y) * X;
+    // Per kernel plane (dz), the first probes of its 9 lookups are issued
+    // together (most resolve there); the rare displaced entries continue
+    // with the probing loop.
 #pragma unroll
-    for (int d = 0; d < kTaps; ++d) {
-      const int dz = d / 9 - 1, dy = (d / 3) % 3 - 1, dx = d % 3 - 1;
-      int32_t r = -1;
-      if (c.y + dz >= 0 && c.y + dz < Z && c.z + dy >= 0 && c.z + dy < Y && c.w + dx >= 0 &&
-          c.w + dx < X) {
+    for (int pz = 0; pz < 3; ++pz) {
+      uint64_t first[9];
+      uint32_t inside = 0;
+#pragma unroll
+      for (int j = 0; j < 9; ++j) {
+        const int d = 9 * pz + j;
+        const int dz = pz - 1, dy = j / 3 - 1, dx = j % 3 - 1;
+        const bool in = c.y + dz >= 0 && c.y + dz < Z && c.z + dy >= 0 && c.z + dy < Y && c.w + dx >= 0 &&
+                        c.w + dx < X;
         const uint64_t nk = key + static_cast<uint64_t>(dz * sz + static_cast<int64_t>(dy) * X + dx);
-        r = lookup<kWide>(table, mask, lg, nk);
+        first[j] = in ? __ldg(&table[kWide ? 2 * slot_of(nk, lg) : slot_of(nk, lg)]) : kEmpty;
+        inside |= static_cast<uint32_t>(in) << j;
+        (void)d;
       }
-      s_nbr[tid * kTaps + d] = r;
-      hits |= static_cast<uint32_t>(r >= 0) << d;
+#pragma unroll
+      for (int j = 0; j < 9; ++j) {
+        const int d = 9 * pz + j;
+        const int dz = pz - 1, dy = j / 3 - 1, dx = j % 3 - 1;
+        const uint64_t nk = key + static_cast<uint64_t>(dz * sz + static_cast<int64_t>(dy) * X + dx);
+        int32_t r = -1;
+        if ((inside >> j) & 1u) {
+          const uint64_t e = first[j];
+          if (e == kEmpty) {
+            r = -1;
+          } else if (!kWide && (e >> 32) == nk) {
+            r = static_cast<int32_t>(e & 0xFFFFFFFFull);
+          } else if (kWide && e == nk) {
+            r = static_cast<int32_t>(__ldg(&table[2 * slot_of(nk, lg) + 1]));
+          } else {
+            r = lookup_from<kWide>(table, mask, (slot_of(nk, lg) + 1) & mask, nk);
+          }
+        }
+        s_nbr[tid * kTaps + d] = r;
+        hits |= static_cast<uint32_t>(r >= 0) << d;
+      }
     }
     gkey[v] = group_key(hits);
+    hmask[v] = hits;
   }
 #pragma unroll
   for (int d = 0; d < kTaps; ++d) {
@@ -359,6 +390,24 @@ __global__ void __launch_bounds__(kRadixThreads) k_radix_scatter(
   }
 }
 
+// Taps present in each 128-row tile of the schedule: OR of its rows' masks.
+// One warp per tile.
+__global__ void __launch_bounds__(256) k_tile_masks(const int32_t* __restrict__ perm,
+                                                    const uint32_t* __restrict__ hmask, int64_t n,
+                                                    uint32_t* __restrict__ tile_mask, int64_t ntiles) {
+  const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (t >= ntiles) return;
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < kTileRows / 32; ++i) {
+    const int64_t g = t * kTileRows + i * 32 + lane;
+    if (g < n) m |= hmask[perm[g]];
+  }
+  m = __reduce_or_sync(0xffffffffu, m);
+  if (lane == 0) tile_mask[t] = m;
+}
+
 // ------------------------------------------------------------ launchers
 static cudaError_t scan_i32(const int32_t* in, int64_t L, int64_t* out, int64_t* partials,
                             int64_t* grand_total, cudaStream_t s) {
@@ -386,13 +435,13 @@ cudaError_t launch_map_build(const MapBuildArgs& a, cudaStream_t s) {
                                             a.Z, a.Y, a.X, a.table, a.lg, a.err);
     k_neighbours<true><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.Z,
                                                 a.Y, a.X, a.table, a.lg, a.nbr, a.gkey,
-                                                a.block_counts, nb);
+                                                a.hmask, a.block_counts, nb);
   } else {
     k_insert<false><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.batch,
                                              a.Z, a.Y, a.X, a.table, a.lg, a.err);
     k_neighbours<false><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.Z,
                                                  a.Y, a.X, a.table, a.lg, a.nbr, a.gkey,
-                                                 a.block_counts, nb);
+                                                 a.hmask, a.block_counts, nb);
   }
   count_launches(2);
   cudaError_t e = cudaGetLastError();
@@ -423,7 +472,9 @@ cudaError_t launch_schedule(const ScheduleArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   k_radix_scatter<<<nblk, kRadixThreads, 0, s>>>(a.key_tmp, a.val_tmp, n, kRadixBits, a.hoff, nblk,
                                                  nullptr, a.perm);
-  count_launches(4);
+  const int64_t ntiles = (n + kTileRows - 1) / kTileRows;
+  k_tile_masks<<<static_cast<unsigned>((ntiles + 7) / 8), 256, 0, s>>>(a.perm, a.hmask, n, a.tile_mask, ntiles);
+  count_launches(5);
   return cudaGetLastError();
 }
 
