@@ -45,6 +45,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -159,23 +163,38 @@ __device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Shared-memory matrix descriptor of a K-major operand stored in the
-// 128-byte-swizzled canonical layout: rows of 128 bytes, 8-row groups 1024
-// bytes apart (stride byte offset), descriptor version 1 (tcgen05).
-__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);     // start address
-  d |= static_cast<uint64_t>(1u) << 16;                       // leading byte offset (unused)
-  d |= static_cast<uint64_t>(1024u >> 4) << 32;               // stride byte offset
-  d |= static_cast<uint64_t>(1u) << 46;                       // version
-  d |= static_cast<uint64_t>(2u) << 61;                       // 128-byte swizzle
-  return d;
-}
-
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator, A and B
 // both bf16 (ab_bf16 = 1) or both fp16 (0), both K-major, M = 128, N = n.
 __host__ __device__ constexpr uint32_t idesc_f16(uint32_t ab_bf16, uint32_t n) {
   return (1u << 4) | (ab_bf16 << 7) | (ab_bf16 << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24);
 }
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(tmap), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+// Shared-memory descriptor of a K-major operand in the canonical swizzled
+// layout: rows of `row_bytes` (64 or 128), 8-row groups 8*row_bytes apart,
+// descriptor version 1, layout 64-byte (4) or 128-byte (2) swizzle.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t smem_addr, uint32_t row_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>((8u * row_bytes) >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(row_bytes == 128 ? 2u : 4u) << 61;
+  return d;
+}
+
+// Bits of a 27-bit tap mask mirrored (d -> 26 - d): the taps of orientation -1.
+__device__ __forceinline__ uint32_t mirror27(uint32_t m) { return __brev(m) >> 5; }
 
 }  // namespace smc

@@ -52,34 +52,6 @@ __host__ __device__ inline TcSmemLayout tc_layout(int stages, int bn, int kb_ele
   return L;
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int32_t x, int32_t y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-      "l"(tmap), "r"(bar), "r"(x), "r"(y)
-      : "memory");
-}
-
-// Shared-memory descriptor of a K-major operand in the canonical swizzled
-// layout: rows of `row_bytes` (64 or 128), 8-row groups 8*row_bytes apart,
-// descriptor version 1, layout 64-byte (4) or 128-byte (2) swizzle.
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t smem_addr, uint32_t row_bytes) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>(1u) << 16;
-  d |= static_cast<uint64_t>((8u * row_bytes) >> 4) << 32;
-  d |= static_cast<uint64_t>(1u) << 46;
-  d |= static_cast<uint64_t>(row_bytes == 128 ? 2u : 4u) << 61;
-  return d;
-}
-
-// Bits of a 27-bit tap mask mirrored (d -> 26 - d): the taps of orientation -1.
-__device__ __forceinline__ uint32_t mirror27(uint32_t m) { return __brev(m) >> 5; }
-
 struct TcParams {
   const int32_t* nbr;
   const int32_t* perm;
@@ -282,12 +254,7 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
 }
 
 // ------------------------------------------------------------------ host
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
-                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                  CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn() {
+EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
   if (!fn) {
     void* ptr = nullptr;

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace smc {
@@ -68,10 +69,18 @@ struct ConvArgs {
   uint32_t* err;
 };
 
+// cuTensorMapEncodeTiled, fetched from the driver through the runtime.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn();
+
 // FMA kernel: every dtype, every shape.
 cudaError_t launch_conv_simt(const ConvArgs& a, cudaStream_t s);
 // tcgen05 kernel: bf16/fp16, cin % 16 == 0 and cin >= 64, cout % 16 == 0, 16-byte aligned.
 bool conv_tc_supported(const ConvArgs& a);
 cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s);
+
 
 }  // namespace smc
