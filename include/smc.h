@@ -175,7 +175,8 @@ SMC_API const char* smc_strerror(int code);
  * Test and measurement hooks.
  * smc_set_hash_capacity: force the hash table to `slots` entries (rounded up
  *   to a power of two, minimum 16) for later builds; 0 restores automatic
- *   sizing (2^ceil(log2(2n))).  Used to exercise SMC_E_CAPACITY.
+ *   sizing (2^ceil(log2(4n)), or 2^ceil(log2(2n)) for keys of 32 bits or
+ *   more).  Used to exercise SMC_E_CAPACITY.
  * smc_set_profiling: when on, smc_build_map records CUDA events on its stream
  *   around its kernels; smc_map_timing then returns, in milliseconds,
  *   ms[0] = hash insert + neighbour map + pair lists, ms[1] = tile schedule.

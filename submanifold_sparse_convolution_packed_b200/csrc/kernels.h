@@ -21,7 +21,6 @@ struct MapBuildArgs {
   int32_t* block_counts;       // [27, nblocks]
   int64_t* block_offsets;      // [27, nblocks]
   int64_t* scan_partials;      // scan_partials_len(27 * nblocks)
-  int64_t* total;              // [1]
   int64_t* info;               // [28]: offsets of the per-offset pair lists
   int32_t* in_idx;             // [27 n] capacity
   int32_t* out_idx;            // [27 n] capacity

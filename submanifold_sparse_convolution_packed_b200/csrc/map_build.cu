@@ -69,12 +69,11 @@ __global__ void __launch_bounds__(256) k_insert(const int4* __restrict__ coords,
   }
 }
 
-// Linear probing from slot s (the home slot has been checked already when
-// called from the neighbour kernel); at most one pass over the table.
+// Linear probing from slot s; at most one pass over the table.
 template <bool kWide>
 __device__ __noinline__ int32_t lookup_from(const unsigned long long* __restrict__ table, uint64_t mask,
                                             uint64_t s, uint64_t key) {
-  for (uint64_t probe = 0; probe < mask; ++probe) {
+  for (uint64_t probe = 0; probe <= mask; ++probe) {
     if (!kWide) {
       const uint64_t e = __ldg(&table[s]);
       if (e == kEmpty) return -1;
@@ -119,45 +118,80 @@ __global__ void __launch_bounds__(kMapBlock) k_neighbours(
     const int4 c = coords[v];
     const uint64_t key = site_key(c, Z, Y, X);
     const int64_t sz = static_cast<int64_t>(Y) * X;
-    // Per kernel plane (dz), the first probes of its 9 lookups are issued
-    // together (most resolve there); the rare displaced entries continue
-    // with the probing loop.
-#pragma unroll
-    for (int pz = 0; pz < 3; ++pz) {
-      uint64_t first[9];
-      uint32_t inside = 0;
-#pragma unroll
-      for (int j = 0; j < 9; ++j) {
-        const int d = 9 * pz + j;
-        const int dz = pz - 1, dy = j / 3 - 1, dx = j % 3 - 1;
-        const bool in = c.y + dz >= 0 && c.y + dz < Z && c.z + dy >= 0 && c.z + dy < Y && c.w + dx >= 0 &&
-                        c.w + dx < X;
-        const uint64_t nk = key + static_cast<uint64_t>(dz * sz + static_cast<int64_t>(dy) * X + dx);
-        first[j] = in ? __ldg(&table[kWide ? 2 * slot_of(nk, lg) : slot_of(nk, lg)]) : kEmpty;
-        inside |= static_cast<uint32_t>(in) << j;
-        (void)d;
-      }
-#pragma unroll
-      for (int j = 0; j < 9; ++j) {
-        const int d = 9 * pz + j;
-        const int dz = pz - 1, dy = j / 3 - 1, dx = j % 3 - 1;
-        const uint64_t nk = key + static_cast<uint64_t>(dz * sz + static_cast<int64_t>(dy) * X + dx);
+    if (kWide) {
+      // two-word slots: plain linear probing per lookup
+#pragma unroll 1
+      for (int d = 0; d < kTaps; ++d) {
+        const int dz = d / 9 - 1, dy = (d / 3) % 3 - 1, dx = d % 3 - 1;
         int32_t r = -1;
-        if ((inside >> j) & 1u) {
-          const uint64_t e = first[j];
-          if (e == kEmpty) {
-            r = -1;
-          } else if (!kWide && (e >> 32) == nk) {
-            r = static_cast<int32_t>(e & 0xFFFFFFFFull);
-          } else if (kWide && e == nk) {
-            r = static_cast<int32_t>(__ldg(&table[2 * slot_of(nk, lg) + 1]));
-          } else {
-            r = lookup_from<kWide>(table, mask, (slot_of(nk, lg) + 1) & mask, nk);
-          }
+        if (c.y + dz >= 0 && c.y + dz < Z && c.z + dy >= 0 && c.z + dy < Y && c.w + dx >= 0 && c.w + dx < X) {
+          const uint64_t nk = key + static_cast<uint64_t>(dz * sz + static_cast<int64_t>(dy) * X + dx);
+          r = lookup_from<true>(table, mask, slot_of(nk, lg), nk);
         }
         s_nbr[tid * kTaps + d] = r;
         hits |= static_cast<uint32_t>(r >= 0) << d;
       }
+    } else {
+    // Per kernel plane (dz) the 9 lookups run in lockstep: each round loads,
+    // for every still-unresolved lookup, the aligned 2-slot group (16 bytes)
+    // holding its next probe position and scans it in probing order.  With
+    // the table at <= 1/4 load almost every lookup resolves in the first round.
+#pragma unroll
+    for (int pz = 0; pz < 3; ++pz) {
+      const uint64_t pkey = key + static_cast<uint64_t>((pz - 1) * sz);  // key of the (dz, 0, 0) neighbour
+      auto nkey = [&](int j) -> uint64_t {
+        return pkey + static_cast<uint64_t>(static_cast<int64_t>(j / 3 - 1) * X + (j % 3 - 1));
+      };
+      uint64_t pos[9];
+      int32_t res[9];
+      uint32_t pend = 0, odd = 0;
+#pragma unroll
+      for (int j = 0; j < 9; ++j) {
+        const int dz = pz - 1, dy = j / 3 - 1, dx = j % 3 - 1;
+        const bool in = c.y + dz >= 0 && c.y + dz < Z && c.z + dy >= 0 && c.z + dy < Y && c.w + dx >= 0 &&
+                        c.w + dx < X;
+        const uint64_t h = slot_of(nkey(j), lg);
+        pos[j] = h & ~static_cast<uint64_t>(1);
+        odd |= static_cast<uint32_t>(h & 1u) << j;  // probing starts at the group's second slot
+        res[j] = -1;
+        pend |= static_cast<uint32_t>(in) << j;
+      }
+      for (uint64_t round = 0; pend != 0 && round <= (mask >> 1); ++round) {
+        ulonglong2 g[9];
+#pragma unroll
+        for (int j = 0; j < 9; ++j)
+          if ((pend >> j) & 1u) g[j] = __ldg(reinterpret_cast<const ulonglong2*>(table + pos[j]));
+#pragma unroll
+        for (int j = 0; j < 9; ++j) {
+          if (!((pend >> j) & 1u)) continue;
+          bool done = false;
+          if (!((odd >> j) & 1u)) {
+            if (g[j].x == kEmpty) {
+              done = true;
+            } else if ((g[j].x >> 32) == nkey(j)) {
+              res[j] = static_cast<int32_t>(g[j].x & 0xFFFFFFFFull);
+              done = true;
+            }
+          }
+          if (!done) {
+            if (g[j].y == kEmpty) {
+              done = true;
+            } else if ((g[j].y >> 32) == nkey(j)) {
+              res[j] = static_cast<int32_t>(g[j].y & 0xFFFFFFFFull);
+              done = true;
+            }
+          }
+          if (done) pend &= ~(1u << j);
+          else pos[j] = (pos[j] + 2) & mask;
+        }
+        odd = 0;
+      }
+#pragma unroll
+      for (int j = 0; j < 9; ++j) {
+        s_nbr[tid * kTaps + 9 * pz + j] = res[j];
+        hits |= static_cast<uint32_t>(res[j] >= 0) << (9 * pz + j);
+      }
+    }
     }
     gkey[v] = group_key(hits);
     hmask[v] = hits;
@@ -189,11 +223,13 @@ __global__ void __launch_bounds__(kMapBlock) k_pairs(const int32_t* __restrict__
                                                      int32_t* __restrict__ out_idx) {
   __shared__ int32_t s_nbr[kMapBlock * kTaps];
   __shared__ int32_t s_pre[kMapBlock / 32][kTaps];
+  __shared__ int64_t s_off[kTaps];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t base = static_cast<int64_t>(blockIdx.x) * kMapBlock;
   const int64_t rows = n - base < kMapBlock ? n - base : kMapBlock;
   const int total = static_cast<int>(rows) * kTaps;
   const int32_t* src = nbr + base * kTaps;
+  if (tid < kTaps) s_off[tid] = block_offsets[static_cast<int64_t>(tid) * nblocks + blockIdx.x];
   const int vec = total >> 2;
   for (int i = tid; i < vec; i += kMapBlock)
     reinterpret_cast<int4*>(s_nbr)[i] = reinterpret_cast<const int4*>(src)[i];
@@ -224,8 +260,7 @@ __global__ void __launch_bounds__(kMapBlock) k_pairs(const int32_t* __restrict__
     const int32_t u = live ? s_nbr[tid * kTaps + d] : -1;
     const uint32_t b = __ballot_sync(0xffffffffu, u >= 0);
     if (u >= 0) {
-      const int64_t pos = block_offsets[static_cast<int64_t>(d) * nblocks + blockIdx.x] +
-                          s_pre[warp][d] + __popc(b & lt);
+      const int64_t pos = s_off[d] + s_pre[warp][d] + __popc(b & lt);
       in_idx[pos] = u;
       out_idx[pos] = static_cast<int32_t>(v);
     }
@@ -279,26 +314,19 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_reduce(const int32_t* __r
   if (threadIdx.x == 0) partials[blockIdx.x] = tot;
 }
 
-// Exclusive scan of the segment partials in place (one block, any count).
-__global__ void __launch_bounds__(kScanThreads) k_scan_partials(int64_t* partials, int64_t nseg,
-                                                                int64_t* grand_total) {
-  __shared__ int64_t s_warp[32];
-  int64_t carry = 0;
-  for (int64_t c0 = 0; c0 < nseg; c0 += kScanThreads) {
-    const int64_t j = c0 + threadIdx.x;
-    const int64_t x = j < nseg ? partials[j] : 0;
-    int64_t tot;
-    const int64_t ex = block_exclusive_scan(x, s_warp, &tot);
-    if (j < nseg) partials[j] = carry + ex;
-    carry += tot;
-  }
-  if (threadIdx.x == 0 && grand_total) *grand_total = carry;
-}
-
+// Exclusive scan of one segment, offset by the sum of all earlier segments'
+// totals (summed by this block: segments are few).  When `info` is given, the
+// values at positions d * stride (d < 27) -- the starts of the per-offset pair
+// lists -- and the grand total go to info[0..27].
 __global__ void __launch_bounds__(kScanThreads) k_scan_apply(const int32_t* __restrict__ in, int64_t L,
-                                                             const int64_t* __restrict__ partials,
-                                                             int64_t* __restrict__ out) {
+                                                             const int64_t* __restrict__ partials, int64_t nseg,
+                                                             int64_t* __restrict__ out, int64_t* __restrict__ info,
+                                                             int64_t stride) {
   __shared__ int64_t s_warp[32];
+  int64_t pre = 0;
+  for (int64_t j = threadIdx.x; j < blockIdx.x; j += kScanThreads) pre += partials[j];
+  int64_t carry;
+  block_exclusive_scan(pre, s_warp, &carry);  // carry = sum of partials[0 .. blockIdx.x)
   const int64_t b0 = static_cast<int64_t>(blockIdx.x) * kScanSeg + threadIdx.x * kScanItems;
   int32_t v[kScanItems];
   int64_t s = 0;
@@ -307,21 +335,18 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_apply(const int32_t* __re
     v[i] = b0 + i < L ? in[b0 + i] : 0;
     s += v[i];
   }
-  int64_t run = partials[blockIdx.x] + block_exclusive_scan(s, s_warp, nullptr);
+  int64_t tot;
+  int64_t run = carry + block_exclusive_scan(s, s_warp, &tot);
 #pragma unroll
   for (int i = 0; i < kScanItems; ++i) {
-    if (b0 + i < L) out[b0 + i] = run;
+    const int64_t j = b0 + i;
+    if (j < L) {
+      out[j] = run;
+      if (info && j % stride == 0 && j / stride < kTaps) info[j / stride] = run;
+    }
     run += v[i];
   }
-}
-
-// Per-offset totals: counts[d] and offsets[0..27] of the pair lists from the
-// scanned block counts.
-__global__ void k_pair_info(const int64_t* __restrict__ block_offsets, int nblocks,
-                            const int64_t* __restrict__ total, int64_t* __restrict__ info) {
-  const int d = threadIdx.x;
-  if (d < kTaps) info[d] = block_offsets[static_cast<int64_t>(d) * nblocks];
-  if (d == kTaps) info[kTaps] = *total;
+  if (info && blockIdx.x == nseg - 1 && threadIdx.x == 0) info[kTaps] = carry + tot;
 }
 
 // ------------------------------------------------------------ radix sort
@@ -365,11 +390,20 @@ __global__ void __launch_bounds__(kRadixThreads) k_radix_scatter(
   __syncthreads();
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kRadixChunk;
   const uint32_t lt = (1u << lane) - 1u;
+  uint32_t keys[kRadixRounds];
+  int32_t vals[kRadixRounds];
+#pragma unroll
+  for (int round = 0; round < kRadixRounds; ++round) {
+    const int64_t j = c0 + static_cast<int64_t>(round) * kRadixThreads + tid;
+    keys[round] = j < n ? keys_in[j] : 0u;
+    vals[round] = j < n ? (vals_in ? vals_in[j] : static_cast<int32_t>(j)) : 0;
+  }
+#pragma unroll
   for (int round = 0; round < kRadixRounds; ++round) {
     const int64_t j = c0 + static_cast<int64_t>(round) * kRadixThreads + tid;
     const bool valid = j < n;
-    const uint32_t key = valid ? keys_in[j] : 0u;
-    const int32_t val = valid ? (vals_in ? vals_in[j] : static_cast<int32_t>(j)) : 0;
+    const uint32_t key = keys[round];
+    const int32_t val = vals[round];
     const uint32_t digit = (key >> shift) & (kRadixBins - 1);
     const uint32_t peers = __match_any_sync(0xffffffffu, valid ? digit : 0xFFFFFFFFu);
     const bool leader = valid && (__ffs(peers) - 1) == lane;
@@ -409,14 +443,13 @@ __global__ void __launch_bounds__(256) k_tile_masks(const int32_t* __restrict__ 
 }
 
 // ------------------------------------------------------------ launchers
-static cudaError_t scan_i32(const int32_t* in, int64_t L, int64_t* out, int64_t* partials,
-                            int64_t* grand_total, cudaStream_t s) {
+static cudaError_t scan_i32(const int32_t* in, int64_t L, int64_t* out, int64_t* partials, int64_t* info,
+                            int64_t stride, cudaStream_t s) {
   const int64_t nseg = (L + kScanSeg - 1) / kScanSeg;
   if (nseg == 0) return cudaSuccess;
   k_scan_reduce<<<static_cast<unsigned>(nseg), kScanThreads, 0, s>>>(in, L, partials);
-  k_scan_partials<<<1, kScanThreads, 0, s>>>(partials, nseg, grand_total);
-  k_scan_apply<<<static_cast<unsigned>(nseg), kScanThreads, 0, s>>>(in, L, partials, out);
-  count_launches(3);
+  k_scan_apply<<<static_cast<unsigned>(nseg), kScanThreads, 0, s>>>(in, L, partials, nseg, out, info, stride);
+  count_launches(2);
   return cudaGetLastError();
 }
 
@@ -447,11 +480,10 @@ cudaError_t launch_map_build(const MapBuildArgs& a, cudaStream_t s) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t L = static_cast<int64_t>(kTaps) * nb;
-  e = scan_i32(a.block_counts, L, a.block_offsets, a.scan_partials, a.total, s);
+  e = scan_i32(a.block_counts, L, a.block_offsets, a.scan_partials, a.info, nb, s);
   if (e != cudaSuccess) return e;
-  k_pair_info<<<1, 32, 0, s>>>(a.block_offsets, nb, a.total, a.info);
   k_pairs<<<nb, kMapBlock, 0, s>>>(a.nbr, n, a.block_offsets, nb, a.in_idx, a.out_idx);
-  count_launches(2);
+  count_launches(1);
   return cudaGetLastError();
 }
 
@@ -462,13 +494,13 @@ cudaError_t launch_schedule(const ScheduleArgs& a, cudaStream_t s) {
   const int64_t L = static_cast<int64_t>(kRadixBins) * nblk;
   // pass 1: low 10 bits, rows in input order
   k_radix_hist<<<nblk, kRadixThreads, 0, s>>>(a.gkey, n, 0, a.hist, nblk);
-  cudaError_t e = scan_i32(a.hist, L, a.hoff, a.scan_partials, nullptr, s);
+  cudaError_t e = scan_i32(a.hist, L, a.hoff, a.scan_partials, nullptr, 1, s);
   if (e != cudaSuccess) return e;
   k_radix_scatter<<<nblk, kRadixThreads, 0, s>>>(a.gkey, nullptr, n, 0, a.hoff, nblk, a.key_tmp,
                                                  a.val_tmp);
   // pass 2: high 10 bits
   k_radix_hist<<<nblk, kRadixThreads, 0, s>>>(a.key_tmp, n, kRadixBits, a.hist, nblk);
-  e = scan_i32(a.hist, L, a.hoff, a.scan_partials, nullptr, s);
+  e = scan_i32(a.hist, L, a.hoff, a.scan_partials, nullptr, 1, s);
   if (e != cudaSuccess) return e;
   k_radix_scatter<<<nblk, kRadixThreads, 0, s>>>(a.key_tmp, a.val_tmp, n, kRadixBits, a.hoff, nblk,
                                                  nullptr, a.perm);
