@@ -183,6 +183,36 @@ SMC_API const char* smc_strerror(int code);
  * smc_kernel_launches: number of CUDA kernels this library has launched in
  *   the process so far (memsets and copies excluded).
  */
+/*
+ * smc_neighbour_map_noalloc -- the int32 [n, 27] neighbour map of smc_build_map
+ * (same values: nbr[v][d] = row of the site at c_v + delta_d, -1 if absent),
+ * written into caller memory without allocating any device memory.  The pages
+ * have no counterpart; this serves callers that may not allocate device memory
+ * while they run: applications that reserve a fixed device-memory budget up
+ * front and forbid allocation in their steady-state loop (an allocation can
+ * stall, synchronise the device or fail part-way through), and plug-ins inside
+ * a host framework that owns the device allocator.
+ *
+ * coords : device, int32 [n, 4] (b, z, y, x), 16-byte aligned.
+ * nbr    : device, int32 [n, 27], 16-byte aligned; fully overwritten.
+ * n      : at most 262144 (SMC_E_SHAPE above that).
+ * batch, grid : as for smc_build_map; batch * Z * Y * X must be below
+ *          2^32 - 1 (SMC_E_ARG otherwise).
+ * stream : work is enqueued on it and the call synchronises it once, to read
+ *          the error word (SMC_E_RANGE, SMC_E_DUPLICATE as for smc_build_map).
+ *
+ * Scratch: one file-scope device array of about 10.1 MB, which every GPU that
+ * loads the library holds until the process exits; no cudaMalloc, cudaFree or
+ * other allocating call is made.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture.  Every call shares the
+ * array and clears what it reads; calls whose work overlaps on the GPU
+ * (different streams or host threads) race on it and must be serialised by
+ * the caller.  No pair lists or tile schedule are produced.
+ */
+SMC_API int smc_neighbour_map_noalloc(const int32_t* coords, int64_t n, int32_t batch, const int32_t grid[3],
+                              int32_t* nbr, void* stream);
+
 SMC_API int smc_set_hash_capacity(int64_t slots);
 SMC_API int smc_set_profiling(int32_t on);
 SMC_API int smc_map_timing(const smc_map* map, float ms[2]);

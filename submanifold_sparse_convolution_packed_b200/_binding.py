@@ -29,7 +29,7 @@ EXPORTS = [
     "smc_build_map", "smc_conv", "smc_map_info", "smc_map_nbr", "smc_map_pairs",
     "smc_map_schedule", "smc_free_map", "smc_status", "smc_strerror",
     "smc_set_hash_capacity", "smc_set_profiling", "smc_map_timing", "smc_kernel_launches",
-    "smc_build_map_async", "smc_map_wait",
+    "smc_build_map_async", "smc_map_wait", "smc_neighbour_map_noalloc",
 ]
 
 
@@ -57,6 +57,7 @@ def lib() -> ctypes.CDLL:
         L.smc_build_map.argtypes = [P, i64, i32, P, P, ctypes.POINTER(P)]
         L.smc_build_map_async.argtypes = [P, i64, i32, P, P, ctypes.POINTER(P)]
         L.smc_map_wait.argtypes = [P]
+        L.smc_neighbour_map_noalloc.argtypes = [P, i64, i32, P, P, P]
         L.smc_conv.argtypes = [P, P, i64, P, P, P, i64, i32, i32, i32, P]
         L.smc_map_info.argtypes = [P, P, P]
         L.smc_map_nbr.argtypes = [P, ctypes.POINTER(P)]
@@ -218,6 +219,34 @@ def build_map(coords: torch.Tensor, grid: Sequence[int], batch: Optional[int] = 
     if key is not None:
         _cache[key] = m
     return m
+
+
+NOALLOC_MAX_N = 1 << 18
+
+
+def neighbour_map_noalloc(coords: torch.Tensor, grid: Sequence[int], batch: Optional[int] = None,
+                          out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """int32 [N, 27] neighbour map computed without any device allocation by
+    the library (its scratch is a fixed static device array; see
+    smc_neighbour_map_noalloc in include/smc.h).  For callers that reserve
+    device memory up front and may not allocate while they run: pass `out`
+    preallocated.  N is limited to NOALLOC_MAX_N."""
+    if coords.dtype != torch.int32 or coords.dim() != 2 or coords.shape[1] != 4 or not coords.is_cuda:
+        raise ValueError("coords must be an int32 [N, 4] CUDA tensor")
+    if not coords.is_contiguous():
+        raise ValueError("coords must be contiguous")
+    n = coords.shape[0]
+    if batch is None:
+        batch = int(coords[:, 0].max().item()) + 1 if n else 1
+    if out is None:
+        out = torch.empty((n, 27), dtype=torch.int32, device=coords.device)
+    elif out.shape != (n, 27) or out.dtype != torch.int32 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous int32 [N, 27] tensor")
+    g = (ctypes.c_int32 * 3)(*[int(x) for x in grid])
+    with torch.cuda.device(coords.device):
+        _check(lib().smc_neighbour_map_noalloc(_ptr(coords), n, int(batch), g, _ptr(out), _stream(stream)),
+               "smc_neighbour_map_noalloc")
+    return out
 
 
 def clear_cache() -> None:

@@ -50,6 +50,9 @@ int radix_bins();
 int64_t scan_partials_len(int64_t L);
 
 cudaError_t launch_map_build(const MapBuildArgs& a, cudaStream_t s);
+cudaError_t launch_neighbour_map_only(const int32_t* coords, int64_t n, int32_t batch, int32_t Z, int32_t Y,
+                                      int32_t X, unsigned long long* table, int lg, uint32_t* err, int32_t* nbr,
+                                      uint32_t* gkey, uint32_t* hmask, int32_t* block_counts, cudaStream_t s);
 cudaError_t launch_schedule(const ScheduleArgs& a, cudaStream_t s);
 
 // dtype codes as in smc.h

@@ -487,6 +487,21 @@ cudaError_t launch_map_build(const MapBuildArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// Hash insert and the 27-lookup neighbour kernel alone (one-word slots), for
+// the entry point that writes the map into caller memory with fixed scratch.
+cudaError_t launch_neighbour_map_only(const int32_t* coords, int64_t n, int32_t batch, int32_t Z, int32_t Y,
+                                      int32_t X, unsigned long long* table, int lg, uint32_t* err, int32_t* nbr,
+                                      uint32_t* gkey, uint32_t* hmask, int32_t* block_counts, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  const int nb = map_nblocks(n);
+  const int grid_ins = static_cast<int>((n + 255) / 256);
+  k_insert<false><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(coords), n, batch, Z, Y, X, table, lg, err);
+  k_neighbours<false><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(coords), n, Z, Y, X, table, lg, nbr,
+                                               gkey, hmask, block_counts, nb);
+  count_launches(2);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_schedule(const ScheduleArgs& a, cudaStream_t s) {
   const int64_t n = a.n;
   if (n == 0) return cudaSuccess;
