@@ -304,3 +304,32 @@ def test_conv_errors():
                       ctypes.c_void_p(f.data_ptr() + 10 ** 6), 16, 3, 1, 7, None)
     assert rc == -4  # dtype
     smc.status()
+
+
+def test_async_build_matches_sync(oracle_mod):
+    """The asynchronous build enqueues everything on the stream; a conv queued
+    right behind it must see the finished map."""
+    w = workload("shells6")
+    coords = torch.from_numpy(w.coords).cuda()
+    f, wt, b = _layer(w, "bf16")
+    ma = smc.build_map(coords, w.grid, batch=1, sync=False)
+    out_a = smc.conv(ma, dev(f, "bf16"), dev(wt, "bf16"), dev(b, "bf16"))
+    ma.wait()
+    ms = smc.build_map(coords, w.grid, batch=1)
+    out_s = smc.conv(ms, dev(f, "bf16"), dev(wt, "bf16"), dev(b, "bf16"))
+    torch.testing.assert_close(out_a, out_s, rtol=0, atol=0)
+    np.testing.assert_array_equal(ma.nbr().cpu().numpy(), ms.nbr().cpu().numpy())
+    assert ma.counts == ms.counts
+
+
+def test_async_build_reports_errors_late():
+    coords = torch.tensor([[0, 1, 1, 1], [0, 2, 2, 2], [0, 1, 1, 1]], dtype=torch.int32, device="cuda")
+    m = smc.build_map(coords, (8, 8, 8), batch=1, sync=False)
+    with pytest.raises(smc.SmcError) as e:
+        m.wait()
+    assert e.value.name == "SMC_E_DUPLICATE"
+    with pytest.raises(smc.SmcError) as e:
+        smc.conv(m, torch.zeros((3, 16), device="cuda"), torch.zeros((16, 3, 3, 3, 16), device="cuda"))
+    assert e.value.name == "SMC_E_DUPLICATE"
+    m.free()
+    smc.status()
