@@ -86,16 +86,22 @@ enum {
  * once the call returns.  Device memory comes from a per-device
  * stream-ordered pool owned by the library that keeps freed memory for
  * later builds.  Errors: SMC_E_ARG, SMC_E_ALIGN, SMC_E_RANGE,
- * SMC_E_DUPLICATE, SMC_E_CAPACITY, SMC_E_OOM, SMC_E_CUDA.
+ * SMC_E_DUPLICATE, SMC_E_CAPACITY, SMC_E_OOM, SMC_E_CUDA, and SMC_E_TIMEOUT
+ * if a bounded wait of the single-pass scans ran out (not expected: a scan
+ * block waits only on blocks that started before it).
  */
 SMC_API int smc_build_map(const int32_t* coords, int64_t n, int32_t batch, const int32_t grid[3],
                   void* stream, smc_map** out);
 
 /*
- * smc_build_map_async -- the same build with no synchronisation: every step
- * is enqueued on `stream` and the handle returns at once.  Argument errors
+ * smc_build_map_async -- the same build with no synchronisation: the work is
+ * enqueued and the handle returns at once.  Work enqueued on `stream` after
+ * the call is ordered after the neighbour map and the tile schedule.  The
+ * pair lists are built on a library-owned stream, concurrently with the tile
+ * schedule, and are complete once smc_map_wait, smc_map_info or smc_map_pairs
+ * has returned.  Argument errors
  * are returned immediately; errors found on the device (SMC_E_RANGE,
- * SMC_E_DUPLICATE, SMC_E_CAPACITY) are returned by smc_map_wait and by every
+ * SMC_E_DUPLICATE, SMC_E_CAPACITY, SMC_E_TIMEOUT) are returned by smc_map_wait and by every
  * later smc_map_* query, and smc_conv refuses a map known to have failed.
  * A conv enqueued before the outcome is known reads a map whose entries are
  * always -1 or valid rows, so it stays memory-safe.  coords must stay valid
@@ -179,7 +185,9 @@ SMC_API const char* smc_strerror(int code);
  *   more).  Used to exercise SMC_E_CAPACITY.
  * smc_set_profiling: when on, smc_build_map records CUDA events on its stream
  *   around its kernels; smc_map_timing then returns, in milliseconds,
- *   ms[0] = hash insert + neighbour map + pair lists, ms[1] = tile schedule.
+ *   ms[0] = hash insert + neighbour lookups, ms[1] = tile schedule, and
+ *   ms[2] = pair lists (built on a library-owned side stream, concurrently
+ *   with the tile schedule; measured from the end of the lookups).
  * smc_kernel_launches: number of CUDA kernels this library has launched in
  *   the process so far (memsets and copies excluded).
  */
@@ -201,7 +209,7 @@ SMC_API const char* smc_strerror(int code);
  * stream : work is enqueued on it and the call synchronises it once, to read
  *          the error word (SMC_E_RANGE, SMC_E_DUPLICATE as for smc_build_map).
  *
- * Scratch: one file-scope device array of about 10.1 MB, which every GPU that
+ * Scratch: one file-scope device array of about 9.5 MB, which every GPU that
  * loads the library holds until the process exits; no cudaMalloc, cudaFree or
  * other allocating call is made.  The first call on a device looks up the
  * array's device address (cudaGetSymbolAddress) with that device current;
@@ -215,7 +223,7 @@ SMC_API int smc_neighbour_map_noalloc(const int32_t* coords, int64_t n, int32_t 
 
 SMC_API int smc_set_hash_capacity(int64_t slots);
 SMC_API int smc_set_profiling(int32_t on);
-SMC_API int smc_map_timing(const smc_map* map, float ms[2]);
+SMC_API int smc_map_timing(const smc_map* map, float ms[3]);
 SMC_API int smc_kernel_launches(int64_t* count);
 
 #ifdef __cplusplus

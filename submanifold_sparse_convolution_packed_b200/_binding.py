@@ -172,9 +172,12 @@ class Map:
         return self._view(p.value, (self.n,))
 
     def timing(self):
-        ms = (ctypes.c_float * 2)()
+        """(lookups, tile schedule, pair lists) device times in ms of a build
+        made with profiling on; the pair lists run concurrently with the
+        schedule."""
+        ms = (ctypes.c_float * 3)()
         _check(lib().smc_map_timing(self.handle, ms), "smc_map_timing")
-        return float(ms[0]), float(ms[1])
+        return float(ms[0]), float(ms[1]), float(ms[2])
 
     def free(self) -> None:
         if self._h is not None:

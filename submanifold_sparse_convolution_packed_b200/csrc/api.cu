@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cstddef>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -36,7 +37,7 @@ struct smc_map {
   uint32_t* tile_mask;
   void* keep;           // one allocation holding nbr, pairs, schedule and tile masks
   cudaEvent_t done;     // recorded after the status block is copied back
-  cudaEvent_t prof[3];  // optional timing events
+  cudaEvent_t prof[4];  // optional timing events
   HostSlot* slot;       // pinned status block
   // filled in when the build is first waited on
   mutable std::mutex mu;
@@ -44,7 +45,7 @@ struct smc_map {
   mutable int status;
   mutable int64_t counts[27];
   mutable int64_t offsets[28];
-  mutable float ms[2];
+  mutable float ms[3];
 };
 
 namespace {
@@ -91,6 +92,51 @@ cudaMemPool_t device_pool(int dev) {
     g_pool[dev] = pool;
   }
   return g_pool[dev];
+}
+
+// Per-device side stream: the pair lists are built there, concurrently with
+// the tile schedule on the build stream (the conv needs the schedule, not the
+// pair lists).
+cudaStream_t g_side[kMaxDevices] = {};
+
+cudaStream_t side_stream(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_side[dev] && cudaStreamCreateWithFlags(&g_side[dev], cudaStreamNonBlocking) != cudaSuccess) {
+    cudaGetLastError();
+    g_side[dev] = nullptr;
+  }
+  return g_side[dev];
+}
+
+// Per-device pool of timing-free events (fork/join points and the maps'
+// completion events), reused instead of created per build.
+std::mutex g_ev_mu;
+std::vector<cudaEvent_t> g_events[kMaxDevices];
+
+cudaEvent_t take_event(int dev) {
+  {
+    std::lock_guard<std::mutex> lk(g_ev_mu);
+    if (!g_events[dev].empty()) {
+      cudaEvent_t e = g_events[dev].back();
+      g_events[dev].pop_back();
+      return e;
+    }
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return e;
+}
+
+// An event may go back once every wait on it has been enqueued (a wait binds
+// to the record made before it) or, for a completion event, once it is done.
+void give_event(int dev, cudaEvent_t e) {
+  if (!e) return;
+  std::lock_guard<std::mutex> lk(g_ev_mu);
+  g_events[dev].push_back(e);
 }
 
 // Pinned host status blocks, handed out from chunks of 256.
@@ -147,7 +193,7 @@ void release_map(smc_map* m) {
   if (cur != m->device) cudaSetDevice(m->device);
   if (m->done) cudaEventSynchronize(m->done);  // the status copy must land before the slot is reused
   if (m->keep) cudaFreeAsync(m->keep, m->stream);
-  if (m->done) cudaEventDestroy(m->done);
+  give_event(m->device, m->done);
   for (auto& e : m->prof)
     if (e) cudaEventDestroy(e);
   give_slot(m->slot);
@@ -169,12 +215,14 @@ int resolve(const smc_map* m) {
     if (err & smc::kErrRange) rc = SMC_E_RANGE;
     else if (err & smc::kErrDuplicate) rc = SMC_E_DUPLICATE;
     else if (err & smc::kErrCapacity) rc = SMC_E_CAPACITY;
+    else if (err & smc::kErrTimeout) rc = SMC_E_TIMEOUT;
     for (int d = 0; d < 28; ++d) m->offsets[d] = m->slot->info[d];
     for (int d = 0; d < 27; ++d) m->counts[d] = m->slot->info[d + 1] - m->slot->info[d];
   }
   if (rc == SMC_OK && m->prof[0]) {
     cudaEventElapsedTime(&m->ms[0], m->prof[0], m->prof[1]);
     cudaEventElapsedTime(&m->ms[1], m->prof[1], m->prof[2]);
+    cudaEventElapsedTime(&m->ms[2], m->prof[1], m->prof[3]);
   }
   m->status = rc;
   m->resolved = true;
@@ -208,8 +256,12 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   }
   cudaMemPool_t pool = device_pool(m->device);
   m->slot = take_slot();
-  if (!pool || !m->slot || cudaEventCreateWithFlags(&m->done, cudaEventDisableTiming) != cudaSuccess) {
-    cudaGetLastError();
+  cudaStream_t side = side_stream(m->device);
+  m->done = take_event(m->device);
+  cudaEvent_t ev_fork = take_event(m->device), ev_sched = take_event(m->device);
+  if (!pool || !m->slot || !side || !m->done || !ev_fork || !ev_sched) {
+    give_event(m->device, ev_fork);
+    give_event(m->device, ev_sched);
     release_map(m);
     return SMC_E_OOM;
   }
@@ -238,27 +290,36 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   const size_t o_tmask = keep.take<uint32_t>((n + smc::kTileRows - 1) / smc::kTileRows);
   Carve tmp;
   const size_t o_table = tmp.take<unsigned long long>(wide ? 2 * cap : cap);
-  const size_t o_err = tmp.take<uint32_t>(1);
-  const size_t o_info = tmp.take<int64_t>(28);
   const size_t o_gkey = tmp.take<uint32_t>(n);
-  const size_t o_hmask = tmp.take<uint32_t>(n);
   const size_t o_bc = tmp.take<int32_t>(Lmap);
   const size_t o_bo = tmp.take<int64_t>(Lmap);
-  const size_t o_sp = tmp.take<int64_t>(smc::scan_partials_len(Lmap > Lrad ? Lmap : Lrad));
-  const size_t o_hist = tmp.take<int32_t>(Lrad);
   const size_t o_hoff = tmp.take<int64_t>(Lrad);
   const size_t o_ktmp = tmp.take<uint32_t>(n);
   const size_t o_vtmp = tmp.take<int32_t>(n);
+  // zeroed by one memset: the device image of the status block (error word,
+  // pair offsets), scan tickets and statuses, histograms
+  const size_t o_err = tmp.take<HostSlot>(1);
+  const size_t o_tick = tmp.take<uint32_t>(3);
+  const size_t o_st0 = tmp.take<unsigned long long>(smc::scan_status_len(Lmap));
+  const size_t o_st1 = tmp.take<unsigned long long>(smc::scan_status_len(Lrad));
+  const size_t o_st2 = tmp.take<unsigned long long>(smc::scan_status_len(Lrad));
+  const size_t o_h1 = tmp.take<int32_t>(Lrad);
+  const size_t o_h2 = tmp.take<int32_t>(Lrad);
+  const size_t zero_bytes = tmp.off - o_err;
 
   void* tp = nullptr;
   if (cudaMallocFromPoolAsync(&m->keep, keep.off, pool, s) != cudaSuccess) {
     cudaGetLastError();
     m->keep = nullptr;
+    give_event(m->device, ev_fork);
+    give_event(m->device, ev_sched);
     release_map(m);
     return SMC_E_OOM;
   }
   if (cudaMallocFromPoolAsync(&tp, tmp.off, pool, s) != cudaSuccess) {
     cudaGetLastError();
+    give_event(m->device, ev_fork);
+    give_event(m->device, ev_sched);
     release_map(m);
     return SMC_E_OOM;
   }
@@ -273,61 +334,79 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   if (g_profiling.load() != 0)
     for (auto& e : m->prof) cudaEventCreate(&e);
 
+  uint32_t* err = reinterpret_cast<uint32_t*>(T + o_err + offsetof(HostSlot, err));
+  uint32_t* tickets = reinterpret_cast<uint32_t*>(T + o_tick);
+  smc::MapBuildArgs a;
+  a.coords = coords;
+  a.n = n;
+  a.batch = batch;
+  a.Z = grid[0];
+  a.Y = grid[1];
+  a.X = grid[2];
+  a.wide = wide;
+  a.table = reinterpret_cast<unsigned long long*>(T + o_table);
+  a.lg = lg;
+  a.err = err;
+  a.zero = m->tile_mask;
+  a.nzero = (n + smc::kTileRows - 1) / smc::kTileRows;
+  a.nbr = m->nbr;
+  a.gkey = reinterpret_cast<uint32_t*>(T + o_gkey);
+  a.block_counts = reinterpret_cast<int32_t*>(T + o_bc);
+  a.block_offsets = reinterpret_cast<int64_t*>(T + o_bo);
+  a.scan_status = reinterpret_cast<unsigned long long*>(T + o_st0);
+  a.scan_ticket = tickets;
+  a.hist1 = reinterpret_cast<int32_t*>(T + o_h1);
+  a.info = reinterpret_cast<int64_t*>(T + o_err + offsetof(HostSlot, info));
+  a.in_idx = m->in_idx;
+  a.out_idx = m->out_idx;
+  smc::ScheduleArgs b;
+  b.gkey = a.gkey;
+  b.n = n;
+  b.hist1 = a.hist1;
+  b.hist2 = reinterpret_cast<int32_t*>(T + o_h2);
+  b.hoff = reinterpret_cast<int64_t*>(T + o_hoff);
+  b.status1 = reinterpret_cast<unsigned long long*>(T + o_st1);
+  b.status2 = reinterpret_cast<unsigned long long*>(T + o_st2);
+  b.tickets = tickets + 1;
+  b.key_tmp = reinterpret_cast<uint32_t*>(T + o_ktmp);
+  b.val_tmp = reinterpret_cast<int32_t*>(T + o_vtmp);
+  b.perm = m->perm;
+  b.tile_mask = m->tile_mask;
+  b.err = err;
+
+  // Build stream s: clear, insert + lookups, then the tile schedule.  Side
+  // stream: the pair lists (forked after the lookups), then -- once the
+  // schedule is done too -- the status copy, the completion event and the
+  // release of the scratch.  A conv enqueued on s behind the build waits for
+  // the schedule only, and overlaps the pair lists.
   cudaError_t ce = cudaMemsetAsync(T + o_table, 0xFF, (wide ? 2 : 1) * cap * sizeof(unsigned long long), s);
-  if (ce == cudaSuccess) ce = cudaMemsetAsync(T + o_err, 0, sizeof(uint32_t), s);
-  if (m->prof[0]) cudaEventRecord(m->prof[0], s);
-  if (ce == cudaSuccess) {
-    smc::MapBuildArgs a;
-    a.coords = coords;
-    a.n = n;
-    a.batch = batch;
-    a.Z = grid[0];
-    a.Y = grid[1];
-    a.X = grid[2];
-    a.wide = wide;
-    a.table = reinterpret_cast<unsigned long long*>(T + o_table);
-    a.lg = lg;
-    a.err = reinterpret_cast<uint32_t*>(T + o_err);
-    a.nbr = m->nbr;
-    a.gkey = reinterpret_cast<uint32_t*>(T + o_gkey);
-    a.hmask = reinterpret_cast<uint32_t*>(T + o_hmask);
-    a.block_counts = reinterpret_cast<int32_t*>(T + o_bc);
-    a.block_offsets = reinterpret_cast<int64_t*>(T + o_bo);
-    a.scan_partials = reinterpret_cast<int64_t*>(T + o_sp);
-    a.info = reinterpret_cast<int64_t*>(T + o_info);
-    a.in_idx = m->in_idx;
-    a.out_idx = m->out_idx;
-    ce = smc::launch_map_build(a, s);
-  }
-  if (m->prof[1]) cudaEventRecord(m->prof[1], s);
-  if (ce == cudaSuccess) {
-    smc::ScheduleArgs b;
-    b.gkey = reinterpret_cast<uint32_t*>(T + o_gkey);
-    b.n = n;
-    b.hist = reinterpret_cast<int32_t*>(T + o_hist);
-    b.hoff = reinterpret_cast<int64_t*>(T + o_hoff);
-    b.scan_partials = reinterpret_cast<int64_t*>(T + o_sp);
-    b.key_tmp = reinterpret_cast<uint32_t*>(T + o_ktmp);
-    b.val_tmp = reinterpret_cast<int32_t*>(T + o_vtmp);
-    b.perm = m->perm;
-    b.hmask = reinterpret_cast<uint32_t*>(T + o_hmask);
-    b.tile_mask = m->tile_mask;
-    ce = smc::launch_schedule(b, s);
-  }
-  if (m->prof[2]) cudaEventRecord(m->prof[2], s);
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(T + o_err, 0, zero_bytes, s);
+  if (ce == cudaSuccess && m->prof[0]) ce = cudaEventRecord(m->prof[0], s);
+  if (ce == cudaSuccess) ce = smc::launch_map_lookups(a, s);
+  if (ce == cudaSuccess && m->prof[1]) ce = cudaEventRecord(m->prof[1], s);
+  if (ce == cudaSuccess) ce = cudaEventRecord(ev_fork, s);
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(side, ev_fork, 0);
+  if (ce == cudaSuccess) ce = smc::launch_pair_lists(a, side);
+  if (ce == cudaSuccess && m->prof[3]) ce = cudaEventRecord(m->prof[3], side);
+  if (ce == cudaSuccess) ce = smc::launch_schedule(b, s);
+  if (ce == cudaSuccess && m->prof[2]) ce = cudaEventRecord(m->prof[2], s);
+  if (ce == cudaSuccess) ce = cudaEventRecord(ev_sched, s);
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(side, ev_sched, 0);
   // the only device->host traffic: error bits and pair offsets, into pinned memory
-  if (ce == cudaSuccess) ce = cudaMemcpyAsync(&m->slot->err, T + o_err, sizeof(uint32_t), cudaMemcpyDeviceToHost, s);
-  if (ce == cudaSuccess)
-    ce = cudaMemcpyAsync(m->slot->info, T + o_info, 28 * sizeof(int64_t), cudaMemcpyDeviceToHost, s);
-  cudaFreeAsync(tp, s);
-  if (ce == cudaSuccess) ce = cudaEventRecord(m->done, s);
+  if (ce == cudaSuccess) ce = cudaMemcpyAsync(m->slot, T + o_err, sizeof(HostSlot), cudaMemcpyDeviceToHost, side);
+  if (ce == cudaSuccess) ce = cudaEventRecord(m->done, side);
+  give_event(m->device, ev_fork);  // their waits are enqueued
+  give_event(m->device, ev_sched);
   if (ce != cudaSuccess) {
     cudaGetLastError();
     cudaStreamSynchronize(s);
+    cudaStreamSynchronize(side);
     cudaGetLastError();
+    cudaFreeAsync(tp, s);
     release_map(m);
     return SMC_E_CUDA;
   }
+  cudaFreeAsync(tp, side);
   *out = m;
   return SMC_OK;
 }
@@ -486,12 +565,13 @@ int smc_kernel_launches(int64_t* count) {
   return SMC_OK;
 }
 
-int smc_map_timing(const smc_map* map, float ms[2]) {
+int smc_map_timing(const smc_map* map, float ms[3]) {
   if (!map || !ms) return SMC_E_ARG;
   const int rc = resolve(map);
   if (rc != SMC_OK) return rc;
   ms[0] = map->ms[0];
   ms[1] = map->ms[1];
+  ms[2] = map->ms[2];
   return SMC_OK;
 }
 

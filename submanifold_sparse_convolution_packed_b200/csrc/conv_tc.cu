@@ -165,7 +165,8 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
     const int q = warp & 3;       // TMEM lane quarter of warps 2..5
     const int r = q * 32 + lane;  // tile row
     const int64_t g = tile * kTileRows + r;
-    const int32_t v = g < p.n ? (k3 ? __ldg(p.perm + g) : static_cast<int32_t>(g)) : -1;
+    int32_t v = g < p.n ? (k3 ? __ldg(p.perm + g) : static_cast<int32_t>(g)) : -1;
+    if (v >= p.n) v = -1;  // a schedule left incomplete by a failed build is skipped, never followed
     // ---------------------------------------------------------- A gather (k=3)
     if (k3) {
       int32_t nb[kTaps];

@@ -14,13 +14,16 @@ struct MapBuildArgs {
   bool wide;                   // two-word hash slots (keys >= 2^32 - 1)
   unsigned long long* table;   // 2^lg slots, pre-filled with ~0
   int lg;
-  uint32_t* err;               // error bits
+  uint32_t* err;               // error bits (zeroed)
+  uint32_t* zero;              // [nzero] words k_insert clears (the tile tap masks)
+  int64_t nzero;
   int32_t* nbr;                // [n, 27]
-  uint32_t* gkey;              // [n] grouping key of the tile schedule
-  uint32_t* hmask;             // [n] 27-bit neighbour hit mask of every row
+  uint32_t* gkey;              // [n] schedule key of every row (carries the 27-bit hit mask)
   int32_t* block_counts;       // [27, nblocks]
   int64_t* block_offsets;      // [27, nblocks]
-  int64_t* scan_partials;      // scan_partials_len(27 * nblocks)
+  unsigned long long* scan_status;  // [scan_status_len(27 * nblocks)], zeroed
+  uint32_t* scan_ticket;       // zeroed
+  int32_t* hist1;              // [bins, radix nblk], zeroed: first schedule digit per chunk
   int64_t* info;               // [28]: offsets of the per-offset pair lists
   int32_t* in_idx;             // [27 n] capacity
   int32_t* out_idx;            // [27 n] capacity
@@ -29,14 +32,17 @@ struct MapBuildArgs {
 struct ScheduleArgs {
   const uint32_t* gkey;   // [n]
   int64_t n;
-  int32_t* hist;          // [bins, nblk]
+  int32_t* hist1;         // [bins, nblk] filled by the neighbour kernel
+  int32_t* hist2;         // [bins, nblk] zeroed
   int64_t* hoff;          // [bins, nblk]
-  int64_t* scan_partials; // scan_partials_len(bins * nblk)
+  unsigned long long* status1;  // [scan_status_len(bins * nblk)] each, zeroed
+  unsigned long long* status2;
+  uint32_t* tickets;      // [2], zeroed
   uint32_t* key_tmp;      // [n]
   int32_t* val_tmp;       // [n]
   int32_t* perm;          // [n] result: tile order
-  const uint32_t* hmask;  // [n] hit masks
-  uint32_t* tile_mask;    // [ceil(n/128)] result: OR of the hit masks of each tile's rows
+  uint32_t* tile_mask;    // [ceil(n/128)] result, zeroed: OR of the hit masks of each tile's rows
+  uint32_t* err;          // error bits
 };
 
 constexpr int kTileRows = 128;  // output rows per tensor-core tile
@@ -47,12 +53,15 @@ void count_launches(int k);
 int map_nblocks(int64_t n);
 int radix_nblocks(int64_t n);
 int radix_bins();
-int64_t scan_partials_len(int64_t L);
+int64_t scan_status_len(int64_t L);
 
-cudaError_t launch_map_build(const MapBuildArgs& a, cudaStream_t s);
+// Hash insert + neighbour lookups (map, schedule keys, block counts, first
+// radix histogram), then, on any stream ordered after them, the pair lists.
+cudaError_t launch_map_lookups(const MapBuildArgs& a, cudaStream_t s);
+cudaError_t launch_pair_lists(const MapBuildArgs& a, cudaStream_t s);
 cudaError_t launch_neighbour_map_only(const int32_t* coords, int64_t n, int32_t batch, int32_t Z, int32_t Y,
                                       int32_t X, unsigned long long* table, int lg, uint32_t* err, int32_t* nbr,
-                                      uint32_t* gkey, uint32_t* hmask, int32_t* block_counts, cudaStream_t s);
+                                      uint32_t* gkey, int32_t* block_counts, cudaStream_t s);
 cudaError_t launch_schedule(const ScheduleArgs& a, cudaStream_t s);
 
 // dtype codes as in smc.h

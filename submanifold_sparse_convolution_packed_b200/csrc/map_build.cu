@@ -7,13 +7,18 @@
 //                 linear site key, insert (key,row) with atomicCAS and linear
 //                 probing; duplicates and a full table set error bits.
 //   k_neighbours  one thread per voxel: 27 lookups -> int32 [n,27] map row
-//                 (staged in shared memory, written coalesced), a 20-bit
-//                 grouping key for the tile schedule, per-block hit counts.
-//   scan          exclusive scan of the block counts in (offset, block) order.
+//                 (staged in shared memory, written coalesced), the row's
+//                 schedule key, per-block hit counts and the histogram of the
+//                 first radix digit of the schedule keys.
+//   scan          single-pass exclusive scan (decoupled look-back) of the
+//                 block counts in (offset, block) order.
 //   k_pairs       stable compaction of every map column into the per-offset
 //                 pair lists (ascending output row).
-//   radix sort    stable 2x10-bit LSD sort of rows by the grouping key: the
+//   radix sort    stable 2x10-bit LSD sort of rows by the schedule key: the
 //                 order in which the tensor-core conv forms 128-row tiles.
+//                 Each pass is one look-back scan of its histogram plus one
+//                 scatter; the first scatter also counts the second digit,
+//                 the second one ORs the tile tap masks.
 #include <cstdint>
 
 #include "common.cuh"
@@ -22,6 +27,13 @@
 namespace smc {
 
 constexpr uint64_t kEmpty = ~0ull;
+constexpr int kMapBlock = 256;       // rows per neighbour / pair block
+constexpr int kRadixBits = 10;
+constexpr int kRadixBins = 1 << kRadixBits;
+constexpr int kRadixThreads = 256;
+constexpr int kRadixRounds = 8;
+constexpr int kRadixChunk = kRadixThreads * kRadixRounds;  // rows per radix block
+static_assert(kRadixChunk % kMapBlock == 0, "a radix chunk is a whole number of map blocks");
 constexpr uint64_t kFib = 0x9E3779B97F4A7C15ull;
 
 __device__ __forceinline__ uint64_t slot_of(uint64_t key, int lg) { return (key * kFib) >> (64 - lg); }
@@ -40,8 +52,13 @@ __device__ __forceinline__ uint64_t site_key(int4 c, int32_t Z, int32_t Y, int32
 template <bool kWide>
 __global__ void __launch_bounds__(256) k_insert(const int4* __restrict__ coords, int64_t n, int32_t batch,
                                                 int32_t Z, int32_t Y, int32_t X,
-                                                unsigned long long* table, int lg, uint32_t* err) {
+                                                unsigned long long* table, int lg, uint32_t* err,
+                                                uint32_t* __restrict__ zero, int64_t nzero) {
   const uint64_t mask = (1ull << lg) - 1;
+  // words later kernels accumulate into (the tile tap masks)
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nzero;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    zero[i] = 0u;
   for (int64_t v = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; v < n;
        v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int4 c = coords[v];
@@ -88,32 +105,48 @@ __device__ __noinline__ int32_t lookup_from(const unsigned long long* __restrict
   return -1;
 }
 
-// Grouping key of a 27-bit hit mask: the 8 corner offsets then the 12 edge
-// offsets, most significant first.  Rows whose rarer neighbours agree end up
-// adjacent after sorting, so a 128-row tile shares most of its absent taps.
+// Schedule key of a row, from its 27-bit hit mask.  Bits 19..0 hold the 8
+// corner offsets then the 12 edge offsets, most significant first: rows whose
+// rarer neighbours agree sort next to each other, so a 128-row tile shares
+// most of its absent taps.  Bits 26..20 carry the other 7 hit bits (the 6
+// faces and the centre), so the key holds the whole mask; the sort reads
+// bits 19..0 only.
 __device__ __forceinline__ uint32_t group_key(uint32_t m) {
-  constexpr int kOrder[20] = {0, 2, 6, 8, 18, 20, 24, 26, 1, 3, 5, 7, 9, 11, 15, 17, 19, 21, 23, 25};
+  constexpr int kOrder[27] = {0, 2, 6, 8, 18, 20, 24, 26, 1, 3, 5, 7, 9, 11,
+                              15, 17, 19, 21, 23, 25, 4, 10, 12, 13, 14, 16, 22};
   uint32_t k = 0;
 #pragma unroll
   for (int i = 0; i < 20; ++i) k |= ((m >> kOrder[i]) & 1u) << (19 - i);
+#pragma unroll
+  for (int i = 20; i < 27; ++i) k |= ((m >> kOrder[i]) & 1u) << i;
   return k;
 }
 
-constexpr int kMapBlock = 256;
+// The hit mask back from a schedule key.
+__device__ __forceinline__ uint32_t key_hits(uint32_t k) {
+  constexpr int kOrder[27] = {0, 2, 6, 8, 18, 20, 24, 26, 1, 3, 5, 7, 9, 11,
+                              15, 17, 19, 21, 23, 25, 4, 10, 12, 13, 14, 16, 22};
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 20; ++i) m |= ((k >> (19 - i)) & 1u) << kOrder[i];
+#pragma unroll
+  for (int i = 20; i < 27; ++i) m |= ((k >> i) & 1u) << kOrder[i];
+  return m;
+}
 
 template <bool kWide>
 __global__ void __launch_bounds__(kMapBlock) k_neighbours(
     const int4* __restrict__ coords, int64_t n, int32_t Z, int32_t Y, int32_t X,
     const unsigned long long* __restrict__ table, int lg, int32_t* __restrict__ nbr,
-    uint32_t* __restrict__ gkey, uint32_t* __restrict__ hmask, int32_t* __restrict__ block_counts,
-    int nblocks) {
+    uint32_t* __restrict__ gkey, int32_t* __restrict__ block_counts, int nblocks,
+    int32_t* __restrict__ hist1, int radix_nblk) {
   __shared__ int32_t s_nbr[kMapBlock * kTaps];
   __shared__ int32_t s_cnt[kMapBlock / 32][kTaps];
   const uint64_t mask = (1ull << lg) - 1;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t base = static_cast<int64_t>(blockIdx.x) * kMapBlock;
   const int64_t v = base + tid;
-  uint32_t hits = 0;
+  uint32_t hits = 0, gk = 0;
   if (v < n) {
     const int4 c = coords[v];
     const uint64_t key = site_key(c, Z, Y, X);
@@ -193,8 +226,15 @@ __global__ void __launch_bounds__(kMapBlock) k_neighbours(
       }
     }
     }
-    gkey[v] = group_key(hits);
-    hmask[v] = hits;
+    gk = group_key(hits);
+    gkey[v] = gk;
+  }
+  if (hist1) {
+    // first radix digit: one atomic per distinct digit of the warp
+    const uint32_t digit = v < n ? (gk & (kRadixBins - 1)) : 0xFFFFFFFFu;
+    const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+    if (v < n && (__ffs(peers) - 1) == lane)
+      atomicAdd(&hist1[static_cast<int64_t>(digit) * radix_nblk + (base / kRadixChunk)], __popc(peers));
   }
 #pragma unroll
   for (int d = 0; d < kTaps; ++d) {
@@ -261,16 +301,31 @@ __global__ void __launch_bounds__(kMapBlock) k_pairs(const int32_t* __restrict__
     const uint32_t b = __ballot_sync(0xffffffffu, u >= 0);
     if (u >= 0) {
       const int64_t pos = s_off[d] + s_pre[warp][d] + __popc(b & lt);
-      in_idx[pos] = u;
-      out_idx[pos] = static_cast<int32_t>(v);
+      if (pos < kTaps * n) {  // always, unless the scan gave up on a wait (error bit set)
+        in_idx[pos] = u;
+        out_idx[pos] = static_cast<int32_t>(v);
+      }
     }
   }
 }
 
 // ------------------------------------------------------------------ scan
-constexpr int kScanThreads = 1024;
-constexpr int kScanItems = 4;
+constexpr int kScanThreads = 512;
+constexpr int kScanItems = 8;
 constexpr int kScanSeg = kScanThreads * kScanItems;
+constexpr unsigned long long kFlagAggregate = 1ull << 62;
+constexpr unsigned long long kFlagPrefix = 2ull << 62;
+constexpr unsigned long long kValueMask = (1ull << 62) - 1;
+
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_relaxed_gpu(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
 
 __device__ __forceinline__ int64_t block_exclusive_scan(int64_t x, int64_t* s_warp, int64_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -299,44 +354,82 @@ __device__ __forceinline__ int64_t block_exclusive_scan(int64_t x, int64_t* s_wa
   return before + incl - x;
 }
 
-__global__ void __launch_bounds__(kScanThreads) k_scan_reduce(const int32_t* __restrict__ in, int64_t L,
-                                                              int64_t* __restrict__ partials) {
+// Single-pass exclusive scan of int32 counts into int64 offsets (decoupled
+// look-back).  A block takes the next segment in start order (a ticket),
+// publishes the segment's total, then sums the totals of earlier segments,
+// reading a window of blockDim predecessors per step and stopping at the
+// nearest one that has published its inclusive prefix; last it publishes its
+// own inclusive prefix.  Statuses are one word each: flag (aggregate /
+// prefix) in bits 63..62, value below, so no fence orders them.  A block waits
+// only on segments with smaller tickets, which are resident and running, so
+// every wait ends; it is still bounded (kWaitLimitNs), after which the error
+// word gets kErrTimeout and the offsets are not to be trusted.
+//
+// When `info` is given, the offsets at positions d * stride (d < 27) -- the
+// starts of the per-offset pair lists -- and the grand total go to info[0..27].
+__global__ void __launch_bounds__(kScanThreads) k_scan_lookback(const int32_t* __restrict__ in, int64_t L,
+                                                                int64_t* __restrict__ out,
+                                                                unsigned long long* status, uint32_t* ticket,
+                                                                uint32_t* err, int64_t* __restrict__ info,
+                                                                int64_t stride) {
   __shared__ int64_t s_warp[32];
-  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * kScanSeg;
-  int64_t s = 0;
-#pragma unroll
-  for (int i = 0; i < kScanItems; ++i) {
-    const int64_t j = b0 + static_cast<int64_t>(i) * kScanThreads + threadIdx.x;
-    if (j < L) s += in[j];
+  __shared__ int64_t s_t;
+  __shared__ int s_first;
+  __shared__ int s_abort;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    s_t = atomicAdd(ticket, 1u);
+    s_first = kScanThreads;
+    s_abort = 0;
   }
-  int64_t tot;
-  block_exclusive_scan(s, s_warp, &tot);
-  if (threadIdx.x == 0) partials[blockIdx.x] = tot;
-}
-
-// Exclusive scan of one segment, offset by the sum of all earlier segments'
-// totals (summed by this block: segments are few).  When `info` is given, the
-// values at positions d * stride (d < 27) -- the starts of the per-offset pair
-// lists -- and the grand total go to info[0..27].
-__global__ void __launch_bounds__(kScanThreads) k_scan_apply(const int32_t* __restrict__ in, int64_t L,
-                                                             const int64_t* __restrict__ partials, int64_t nseg,
-                                                             int64_t* __restrict__ out, int64_t* __restrict__ info,
-                                                             int64_t stride) {
-  __shared__ int64_t s_warp[32];
-  int64_t pre = 0;
-  for (int64_t j = threadIdx.x; j < blockIdx.x; j += kScanThreads) pre += partials[j];
-  int64_t carry;
-  block_exclusive_scan(pre, s_warp, &carry);  // carry = sum of partials[0 .. blockIdx.x)
-  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * kScanSeg + threadIdx.x * kScanItems;
+  __syncthreads();
+  const int64_t t = s_t;
+  const int64_t nseg = (L + kScanSeg - 1) / kScanSeg;
+  const int64_t b0 = t * kScanSeg + static_cast<int64_t>(tid) * kScanItems;
   int32_t v[kScanItems];
-  int64_t s = 0;
+  int64_t sum = 0;
 #pragma unroll
   for (int i = 0; i < kScanItems; ++i) {
     v[i] = b0 + i < L ? in[b0 + i] : 0;
-    s += v[i];
+    sum += v[i];
   }
   int64_t tot;
-  int64_t run = carry + block_exclusive_scan(s, s_warp, &tot);
+  const int64_t mine = block_exclusive_scan(sum, s_warp, &tot);
+  if (tid == 0)
+    st_relaxed_gpu(&status[t], (t == 0 ? kFlagPrefix : kFlagAggregate) | static_cast<unsigned long long>(tot));
+  int64_t excl = 0;
+  if (t > 0) {
+    int64_t top = t - 1;  // nearest predecessor not summed yet
+    const uint64_t t_start = globaltimer_ns();
+    for (;;) {
+      const int64_t j = top - tid;
+      const unsigned long long w = j >= 0 ? ld_relaxed_gpu(&status[j]) : kFlagPrefix;
+      const unsigned long long flag = w & ~kValueMask;
+      if (flag == kFlagPrefix) atomicMin(&s_first, tid);
+      __syncthreads();
+      const int first = s_first;  // window index of the nearest inclusive prefix, or kScanThreads
+      if (!__syncthreads_and(tid > first || flag != 0)) {
+        // a predecessor up to that prefix has not published yet: read again
+        if (tid == 0) {
+          s_first = kScanThreads;
+          if (globaltimer_ns() - t_start > kWaitLimitNs) {
+            atomicOr(err, kErrTimeout);
+            s_abort = 1;
+          }
+        }
+        __syncthreads();
+        if (s_abort) break;
+        continue;
+      }
+      int64_t part;
+      block_exclusive_scan(tid <= first ? static_cast<int64_t>(w & kValueMask) : 0, s_warp, &part);
+      excl += part;
+      if (first < kScanThreads) break;
+      top -= kScanThreads;
+    }
+    if (tid == 0) st_relaxed_gpu(&status[t], kFlagPrefix | static_cast<unsigned long long>(excl + tot));
+  }
+  int64_t run = excl + mine;
 #pragma unroll
   for (int i = 0; i < kScanItems; ++i) {
     const int64_t j = b0 + i;
@@ -346,45 +439,29 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_apply(const int32_t* __re
     }
     run += v[i];
   }
-  if (info && blockIdx.x == nseg - 1 && threadIdx.x == 0) info[kTaps] = carry + tot;
+  if (info && t == nseg - 1 && tid == 0) info[kTaps] = excl + tot;
 }
 
 // ------------------------------------------------------------ radix sort
-constexpr int kRadixBits = 10;
-constexpr int kRadixBins = 1 << kRadixBits;
-constexpr int kRadixThreads = 256;
-constexpr int kRadixRounds = 8;
-constexpr int kRadixChunk = kRadixThreads * kRadixRounds;
-
-__global__ void __launch_bounds__(kRadixThreads) k_radix_hist(const uint32_t* __restrict__ keys, int64_t n,
-                                                              int shift, int32_t* __restrict__ hist,
-                                                              int nblk) {
-  __shared__ int32_t s_h[kRadixBins];
-  for (int i = threadIdx.x; i < kRadixBins; i += kRadixThreads) s_h[i] = 0;
-  __syncthreads();
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kRadixChunk;
-  for (int i = threadIdx.x; i < kRadixChunk; i += kRadixThreads) {
-    const int64_t j = c0 + i;
-    if (j < n) atomicAdd(&s_h[(keys[j] >> shift) & (kRadixBins - 1)], 1);
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < kRadixBins; i += kRadixThreads)
-    hist[static_cast<int64_t>(i) * nblk + blockIdx.x] = s_h[i];
-}
-
-// Stable scatter of one radix pass.  The chunk of a block is visited in
+// Stable scatter of one radix pass over a histogram already scanned into
+// `offsets` ([bins, nblk], digit-major).  The chunk of a block is visited in
 // rounds of 256 consecutive elements; inside a round, an element's rank is
 // (elements of its digit in earlier rounds) + (in earlier warps of this
 // round) + (in earlier lanes of its warp), so the input order is kept.
+// First pass (kLast false): writes keys and row indices and counts the next
+// digit per destination chunk into hist_next.  Last pass: writes the row
+// order and ORs each row's hit mask into the mask of its 128-row tile.
+template <bool kLast>
 __global__ void __launch_bounds__(kRadixThreads) k_radix_scatter(
     const uint32_t* __restrict__ keys_in, const int32_t* __restrict__ vals_in, int64_t n, int shift,
     const int64_t* __restrict__ offsets, int nblk, uint32_t* __restrict__ keys_out,
-    int32_t* __restrict__ vals_out) {
-  __shared__ unsigned long long s_base[kRadixBins];
+    int32_t* __restrict__ vals_out, int32_t* __restrict__ hist_next, uint32_t* __restrict__ tile_mask,
+    uint32_t* err) {
+  __shared__ uint32_t s_base[kRadixBins];  // positions < n < 2^31
   __shared__ int32_t s_wcnt[kRadixThreads / 32][kRadixBins];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int i = tid; i < kRadixBins; i += kRadixThreads)
-    s_base[i] = static_cast<unsigned long long>(offsets[static_cast<int64_t>(i) * nblk + blockIdx.x]);
+    s_base[i] = static_cast<uint32_t>(offsets[static_cast<int64_t>(i) * nblk + blockIdx.x]);
   for (int i = tid; i < (kRadixThreads / 32) * kRadixBins; i += kRadixThreads)
     (&s_wcnt[0][0])[i] = 0;
   __syncthreads();
@@ -409,78 +486,93 @@ __global__ void __launch_bounds__(kRadixThreads) k_radix_scatter(
     const bool leader = valid && (__ffs(peers) - 1) == lane;
     if (leader) s_wcnt[warp][digit] = __popc(peers);
     __syncthreads();
+    long long pos = -1;
     if (valid) {
-      long long pos = static_cast<long long>(s_base[digit]) + __popc(peers & lt);
-      for (int w = 0; w < warp; ++w) pos += s_wcnt[w][digit];
-      if (keys_out) keys_out[pos] = key;
+      int32_t r = __popc(peers & lt);
+      for (int w = 0; w < warp; ++w) r += s_wcnt[w][digit];
+      pos = static_cast<long long>(s_base[digit]) + r;
+      if (pos >= n) {  // only after a scan gave up on a wait
+        atomicOr(err, kErrTimeout);
+        pos = -1;
+      }
+    }
+    if (pos >= 0) {
+      if (!kLast) keys_out[pos] = key;
       vals_out[pos] = val;
+    }
+    if (!kLast) {
+      // next digit, counted per destination chunk: one atomic per distinct (digit, chunk) of the warp
+      const uint32_t tag = pos >= 0 ? ((((key >> (shift + kRadixBits)) & (kRadixBins - 1)) << 21) |
+                                       static_cast<uint32_t>(pos / kRadixChunk))
+                                    : 0xFFFFFFFFu;
+      const uint32_t grp = __match_any_sync(0xffffffffu, tag);
+      if (tag != 0xFFFFFFFFu && (__ffs(grp) - 1) == lane)
+        atomicAdd(&hist_next[static_cast<int64_t>(tag >> 21) * nblk + (tag & ((1u << 21) - 1))], __popc(grp));
+    } else {
+      // tile tap masks: a warp whose rows all land in one tile (dense data)
+      // ORs them first; otherwise every row ORs its own mask in
+      const uint32_t tile = pos >= 0 ? static_cast<uint32_t>(pos / kTileRows) : 0xFFFFFFFFu;
+      const uint32_t hm = pos >= 0 ? key_hits(key) : 0u;
+      const uint32_t t0 = __reduce_min_sync(0xffffffffu, tile);
+      if (__all_sync(0xffffffffu, tile == t0 || tile == 0xFFFFFFFFu)) {
+        const uint32_t r = __reduce_or_sync(0xffffffffu, hm);
+        if (lane == 0 && t0 != 0xFFFFFFFFu) atomicOr(&tile_mask[t0], r);
+      } else if (pos >= 0) {
+        atomicOr(&tile_mask[tile], hm);
+      }
     }
     __syncthreads();
     if (leader) {
-      atomicAdd(&s_base[digit], static_cast<unsigned long long>(__popc(peers)));
+      atomicAdd(&s_base[digit], static_cast<uint32_t>(__popc(peers)));
       s_wcnt[warp][digit] = 0;
     }
     __syncwarp();
   }
 }
 
-// Taps present in each 128-row tile of the schedule: OR of its rows' masks.
-// One warp per tile.
-__global__ void __launch_bounds__(256) k_tile_masks(const int32_t* __restrict__ perm,
-                                                    const uint32_t* __restrict__ hmask, int64_t n,
-                                                    uint32_t* __restrict__ tile_mask, int64_t ntiles) {
-  const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (t >= ntiles) return;
-  uint32_t m = 0;
-#pragma unroll
-  for (int i = 0; i < kTileRows / 32; ++i) {
-    const int64_t g = t * kTileRows + i * 32 + lane;
-    if (g < n) m |= hmask[perm[g]];
-  }
-  m = __reduce_or_sync(0xffffffffu, m);
-  if (lane == 0) tile_mask[t] = m;
-}
-
 // ------------------------------------------------------------ launchers
-static cudaError_t scan_i32(const int32_t* in, int64_t L, int64_t* out, int64_t* partials, int64_t* info,
-                            int64_t stride, cudaStream_t s) {
+static cudaError_t scan_i32(const int32_t* in, int64_t L, int64_t* out, unsigned long long* status,
+                            uint32_t* ticket, uint32_t* err, int64_t* info, int64_t stride, cudaStream_t s) {
   const int64_t nseg = (L + kScanSeg - 1) / kScanSeg;
   if (nseg == 0) return cudaSuccess;
-  k_scan_reduce<<<static_cast<unsigned>(nseg), kScanThreads, 0, s>>>(in, L, partials);
-  k_scan_apply<<<static_cast<unsigned>(nseg), kScanThreads, 0, s>>>(in, L, partials, nseg, out, info, stride);
-  count_launches(2);
+  k_scan_lookback<<<static_cast<unsigned>(nseg), kScanThreads, 0, s>>>(in, L, out, status, ticket, err, info,
+                                                                       stride);
+  count_launches(1);
   return cudaGetLastError();
 }
 
-int64_t scan_partials_len(int64_t L) { return (L + kScanSeg - 1) / kScanSeg + 1; }
+int64_t scan_status_len(int64_t L) { return (L + kScanSeg - 1) / kScanSeg; }
 int map_nblocks(int64_t n) { return static_cast<int>((n + kMapBlock - 1) / kMapBlock); }
 int radix_nblocks(int64_t n) { return static_cast<int>((n + kRadixChunk - 1) / kRadixChunk); }
 int radix_bins() { return kRadixBins; }
 
-cudaError_t launch_map_build(const MapBuildArgs& a, cudaStream_t s) {
+cudaError_t launch_map_lookups(const MapBuildArgs& a, cudaStream_t s) {
   const int64_t n = a.n;
   if (n == 0) return cudaSuccess;
   const int nb = map_nblocks(n);
+  const int rnb = radix_nblocks(n);
   const int grid_ins = static_cast<int>((n + 255) / 256);
   if (a.wide) {
-    k_insert<true><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.batch,
-                                            a.Z, a.Y, a.X, a.table, a.lg, a.err);
-    k_neighbours<true><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.Z,
-                                                a.Y, a.X, a.table, a.lg, a.nbr, a.gkey,
-                                                a.hmask, a.block_counts, nb);
+    k_insert<true><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.batch, a.Z, a.Y, a.X,
+                                            a.table, a.lg, a.err, a.zero, a.nzero);
+    k_neighbours<true><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.Z, a.Y, a.X,
+                                                a.table, a.lg, a.nbr, a.gkey, a.block_counts, nb, a.hist1, rnb);
   } else {
-    k_insert<false><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.batch,
-                                             a.Z, a.Y, a.X, a.table, a.lg, a.err);
-    k_neighbours<false><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.Z,
-                                                 a.Y, a.X, a.table, a.lg, a.nbr, a.gkey,
-                                                 a.hmask, a.block_counts, nb);
+    k_insert<false><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.batch, a.Z, a.Y, a.X,
+                                             a.table, a.lg, a.err, a.zero, a.nzero);
+    k_neighbours<false><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.Z, a.Y, a.X,
+                                                 a.table, a.lg, a.nbr, a.gkey, a.block_counts, nb, a.hist1, rnb);
   }
   count_launches(2);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pair_lists(const MapBuildArgs& a, cudaStream_t s) {
+  const int64_t n = a.n;
+  if (n == 0) return cudaSuccess;
+  const int nb = map_nblocks(n);
   const int64_t L = static_cast<int64_t>(kTaps) * nb;
-  e = scan_i32(a.block_counts, L, a.block_offsets, a.scan_partials, a.info, nb, s);
+  cudaError_t e = scan_i32(a.block_counts, L, a.block_offsets, a.scan_status, a.scan_ticket, a.err, a.info, nb, s);
   if (e != cudaSuccess) return e;
   k_pairs<<<nb, kMapBlock, 0, s>>>(a.nbr, n, a.block_offsets, nb, a.in_idx, a.out_idx);
   count_launches(1);
@@ -491,13 +583,14 @@ cudaError_t launch_map_build(const MapBuildArgs& a, cudaStream_t s) {
 // the entry point that writes the map into caller memory with fixed scratch.
 cudaError_t launch_neighbour_map_only(const int32_t* coords, int64_t n, int32_t batch, int32_t Z, int32_t Y,
                                       int32_t X, unsigned long long* table, int lg, uint32_t* err, int32_t* nbr,
-                                      uint32_t* gkey, uint32_t* hmask, int32_t* block_counts, cudaStream_t s) {
+                                      uint32_t* gkey, int32_t* block_counts, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
   const int nb = map_nblocks(n);
   const int grid_ins = static_cast<int>((n + 255) / 256);
-  k_insert<false><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(coords), n, batch, Z, Y, X, table, lg, err);
+  k_insert<false><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(coords), n, batch, Z, Y, X, table, lg,
+                                           err, nullptr, 0);
   k_neighbours<false><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(coords), n, Z, Y, X, table, lg, nbr,
-                                               gkey, hmask, block_counts, nb);
+                                               gkey, block_counts, nb, nullptr, 0);
   count_launches(2);
   return cudaGetLastError();
 }
@@ -507,21 +600,18 @@ cudaError_t launch_schedule(const ScheduleArgs& a, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
   const int nblk = radix_nblocks(n);
   const int64_t L = static_cast<int64_t>(kRadixBins) * nblk;
-  // pass 1: low 10 bits, rows in input order
-  k_radix_hist<<<nblk, kRadixThreads, 0, s>>>(a.gkey, n, 0, a.hist, nblk);
-  cudaError_t e = scan_i32(a.hist, L, a.hoff, a.scan_partials, nullptr, 1, s);
+  // pass 1: low 10 bits, rows in input order (histogram from the neighbour kernel)
+  cudaError_t e = scan_i32(a.hist1, L, a.hoff, a.status1, a.tickets, a.err, nullptr, 1, s);
   if (e != cudaSuccess) return e;
-  k_radix_scatter<<<nblk, kRadixThreads, 0, s>>>(a.gkey, nullptr, n, 0, a.hoff, nblk, a.key_tmp,
-                                                 a.val_tmp);
+  k_radix_scatter<false><<<nblk, kRadixThreads, 0, s>>>(a.gkey, nullptr, n, 0, a.hoff, nblk, a.key_tmp,
+                                                        a.val_tmp, a.hist2, nullptr, a.err);
+  count_launches(1);
   // pass 2: high 10 bits
-  k_radix_hist<<<nblk, kRadixThreads, 0, s>>>(a.key_tmp, n, kRadixBits, a.hist, nblk);
-  e = scan_i32(a.hist, L, a.hoff, a.scan_partials, nullptr, 1, s);
+  e = scan_i32(a.hist2, L, a.hoff, a.status2, a.tickets + 1, a.err, nullptr, 1, s);
   if (e != cudaSuccess) return e;
-  k_radix_scatter<<<nblk, kRadixThreads, 0, s>>>(a.key_tmp, a.val_tmp, n, kRadixBits, a.hoff, nblk,
-                                                 nullptr, a.perm);
-  const int64_t ntiles = (n + kTileRows - 1) / kTileRows;
-  k_tile_masks<<<static_cast<unsigned>((ntiles + 7) / 8), 256, 0, s>>>(a.perm, a.hmask, n, a.tile_mask, ntiles);
-  count_launches(5);
+  k_radix_scatter<true><<<nblk, kRadixThreads, 0, s>>>(a.key_tmp, a.val_tmp, n, kRadixBits, a.hoff, nblk,
+                                                       nullptr, a.perm, nullptr, a.tile_mask, a.err);
+  count_launches(1);
   return cudaGetLastError();
 }
 

@@ -70,6 +70,19 @@ def sample_rows(n, k, seed):
 
 
 # ------------------------------------------------------------------ map
+# The tile order of the tensor-core conv: rows stably sorted by a 20-bit key
+# whose bits, most significant first, say whether the 8 corner offsets and
+# then the 12 edge offsets have a neighbour.
+_KEY_TAPS = [0, 2, 6, 8, 18, 20, 24, 26, 1, 3, 5, 7, 9, 11, 15, 17, 19, 21, 23, 25]
+
+
+def expected_schedule(nbr):
+    key = np.zeros(nbr.shape[0], dtype=np.int64)
+    for i, d in enumerate(_KEY_TAPS):
+        key |= (nbr[:, d] >= 0).astype(np.int64) << (19 - i)
+    return np.argsort(key, kind="stable").astype(np.int32)
+
+
 MAP_CASES = ["tiny", "shell2", "shells6", "varlen4", "decoder0", "decoder3", "full128"]
 
 
@@ -87,7 +100,7 @@ def test_map_bit_exact(oracle_mod, name):
     np.testing.assert_array_equal(gi.cpu().numpy(), in_idx)
     np.testing.assert_array_equal(go.cpu().numpy(), out_idx)
     perm = m.schedule().cpu().numpy()
-    assert np.array_equal(np.sort(perm), np.arange(w.n))
+    np.testing.assert_array_equal(perm, expected_schedule(ref))
 
 
 def test_map_shuffled_rows(oracle_mod):
@@ -95,7 +108,9 @@ def test_map_shuffled_rows(oracle_mod):
     rng = np.random.default_rng(1)
     coords = w.coords[rng.permutation(w.n)]
     m = smc.build_map(torch.from_numpy(coords).cuda(), w.grid, batch=2)
-    np.testing.assert_array_equal(m.nbr().cpu().numpy(), oracle_mod.neighbour_map(coords, w.grid))
+    ref = oracle_mod.neighbour_map(coords, w.grid)
+    np.testing.assert_array_equal(m.nbr().cpu().numpy(), ref)
+    np.testing.assert_array_equal(m.schedule().cpu().numpy(), expected_schedule(ref))
 
 
 def test_map_wide_keys(oracle_mod):
@@ -108,7 +123,9 @@ def test_map_wide_keys(oracle_mod):
     coords = np.concatenate([np.zeros((len(zyx), 1), np.int32), zyx], axis=1)
     coords = np.concatenate([coords, coords + np.array([1, 0, 0, 0], np.int32)])
     m = smc.build_map(torch.from_numpy(coords).cuda(), grid, batch=2)
-    np.testing.assert_array_equal(m.nbr().cpu().numpy(), oracle_mod.neighbour_map(coords, grid))
+    ref = oracle_mod.neighbour_map(coords, grid)
+    np.testing.assert_array_equal(m.nbr().cpu().numpy(), ref)
+    np.testing.assert_array_equal(m.schedule().cpu().numpy(), expected_schedule(ref))
 
 
 def test_map_empty_and_single():
@@ -120,6 +137,7 @@ def test_map_empty_and_single():
     one = smc.build_map(torch.tensor([[0, 2, 2, 2]], dtype=torch.int32, device="cuda"), (5, 5, 5), batch=1)
     nbr = one.nbr().cpu().numpy()
     assert nbr[0, 13] == 0 and (np.delete(nbr[0], 13) == -1).all()
+    assert one.schedule().cpu().numpy().tolist() == [0]
 
 
 def test_map_errors():
