@@ -190,6 +190,12 @@ SMC_API const char* smc_strerror(int code);
  *   with the tile schedule; measured from the end of the lookups).
  * smc_kernel_launches: number of CUDA kernels this library has launched in
  *   the process so far (memsets and copies excluded).
+ * smc_set_conv_variant: tensor-core conv kernel for later convs: 0 = default
+ *   (currently the same as 1), 1 = one CTA per 128-row tile, 2 = CTA pairs (a
+ *   cluster of two CTAs sharing M = 256 tcgen05 MMAs, each loading half of
+ *   the weight block; slower on B200, where such clusters run one per TPC).
+ *   Results are identical; used to test and measure both kernels.
+ *   SMC_E_ARG for any other value.
  */
 /*
  * smc_neighbour_map_noalloc -- the int32 [n, 27] neighbour map of smc_build_map
@@ -225,6 +231,7 @@ SMC_API int smc_set_hash_capacity(int64_t slots);
 SMC_API int smc_set_profiling(int32_t on);
 SMC_API int smc_map_timing(const smc_map* map, float ms[3]);
 SMC_API int smc_kernel_launches(int64_t* count);
+SMC_API int smc_set_conv_variant(int32_t variant);
 
 #ifdef __cplusplus
 }

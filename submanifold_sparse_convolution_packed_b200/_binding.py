@@ -29,7 +29,7 @@ EXPORTS = [
     "smc_build_map", "smc_conv", "smc_map_info", "smc_map_nbr", "smc_map_pairs",
     "smc_map_schedule", "smc_free_map", "smc_status", "smc_strerror",
     "smc_set_hash_capacity", "smc_set_profiling", "smc_map_timing", "smc_kernel_launches",
-    "smc_build_map_async", "smc_map_wait", "smc_neighbour_map_noalloc",
+    "smc_build_map_async", "smc_map_wait", "smc_neighbour_map_noalloc", "smc_set_conv_variant",
 ]
 
 
@@ -71,6 +71,7 @@ def lib() -> ctypes.CDLL:
         L.smc_set_profiling.argtypes = [i32]
         L.smc_map_timing.argtypes = [P, P]
         L.smc_kernel_launches.argtypes = [P]
+        L.smc_set_conv_variant.argtypes = [i32]
         for name in EXPORTS:
             if name != "smc_strerror":
                 getattr(L, name).restype = ctypes.c_int
@@ -290,6 +291,11 @@ def conv(m: Map, feats: torch.Tensor, weight: torch.Tensor, bias: Optional[torch
 def status(stream=None) -> None:
     """Synchronise the stream and raise if a conv kernel reported a timeout."""
     _check(lib().smc_status(_stream(stream)), "smc_status")
+
+
+def set_conv_variant(variant: int) -> None:
+    """Tensor-core conv kernel: 0 by shape, 1 one CTA per tile, 2 CTA pairs."""
+    _check(lib().smc_set_conv_variant(int(variant)), "smc_set_conv_variant")
 
 
 def set_hash_capacity(slots: int) -> None:

@@ -443,6 +443,12 @@ int smc_set_hash_capacity(int64_t slots) {
   return SMC_OK;
 }
 
+int smc_set_conv_variant(int32_t variant) {
+  if (variant < 0 || variant > 2) return SMC_E_ARG;
+  smc::set_conv_variant(variant);
+  return SMC_OK;
+}
+
 int smc_set_profiling(int32_t on) {
   g_profiling.store(on ? 1 : 0);
   return SMC_OK;

@@ -24,6 +24,8 @@
 // Pipeline stages are (tap, channel block) pairs of KB = 32 or 64 channels in
 // swizzled shared memory (64-byte or 128-byte swizzle).  Every wait is
 // bounded; on timeout the error word gets a bit and the CTA winds down.
+#include <atomic>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -60,10 +62,16 @@ struct TcParams {
   uint16_t* out;
   uint32_t* err;
   int64_t n;
+  int64_t ntiles;
   int cin, cout, taps, orientation, bn, nsplit, stages, is_bf16, kb_elems;
   uint32_t tmem_cols;
 };
 
+// kPair: the CTA is one of a cluster pair sharing M = 256 MMAs (rows of two
+// consecutive schedule tiles, the union of their tap masks); it loads its own
+// 128 gathered rows and half of the weight block's N columns, and every load
+// and arrival counts on the even CTA's full barriers.
+template <bool kPair>
 __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant__ CUtensorMap fmap,
                                                         const __grid_constant__ CUtensorMap wmap,
                                                         const TcParams p) {
@@ -71,7 +79,8 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;  // swizzle atoms need aligned bases
   uint8_t* smem = smem_raw + (sbase - raw);
-  const TcSmemLayout L = tc_layout(p.stages, p.bn, p.kb_elems);
+  const int bn_cta = kPair ? p.bn / 2 : p.bn;  // weight rows (output channels) this CTA loads
+  const TcSmemLayout L = tc_layout(p.stages, bn_cta, p.kb_elems);
   const uint32_t bar_full = sbase + L.bar_off;
   const uint32_t bar_empty = bar_full + kMaxStages * 8;
   const uint32_t bar_acc = bar_empty + kMaxStages * 8;
@@ -79,16 +88,20 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool k3 = p.taps == kTaps;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
   const uint32_t row_bytes = static_cast<uint32_t>(p.kb_elems) * 2;
   const uint32_t a_bytes = kTileRows * row_bytes;
-  const uint32_t b_bytes = static_cast<uint32_t>(p.bn) * row_bytes;
+  const uint32_t b_bytes = static_cast<uint32_t>(bn_cta) * row_bytes;
   const int kblocks = (p.cin + p.kb_elems - 1) / p.kb_elems;
   const int last_ksteps = (p.cin - (kblocks - 1) * p.kb_elems + 15) / 16;
-  const int64_t tile = blockIdx.x / p.nsplit;
-  const int n0 = static_cast<int>(blockIdx.x % p.nsplit) * p.bn;
+  const int64_t unit = kPair ? blockIdx.x / 2 : blockIdx.x;
+  const int64_t tile0 = (unit / p.nsplit) * (kPair ? 2 : 1);  // first tile of the unit
+  const int64_t tile = tile0 + rank;
+  const int n0 = static_cast<int>(unit % p.nsplit) * p.bn;
   uint32_t mask = 1u;
   if (k3) {
-    mask = __ldg(p.tile_mask + tile);
+    mask = __ldg(p.tile_mask + tile0);
+    if (kPair && tile0 + 1 < p.ntiles) mask |= __ldg(p.tile_mask + tile0 + 1);
     if (p.orientation < 0) mask = mirror27(mask);
   }
 
@@ -96,7 +109,8 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
     prefetch_tmap(&fmap);
     prefetch_tmap(&wmap);
     for (int s = 0; s < p.stages; ++s) {
-      mbar_init(bar_full + 8 * s, k3 ? 5 : 1);  // weight loader (+ 4 gather warps)
+      // weight loader (+ 4 gather warps), of both CTAs for a pair
+      mbar_init(bar_full + 8 * s, (k3 ? 5 : 1) * (kPair ? 2 : 1));
       mbar_init(bar_empty + 8 * s, 1);
     }
     mbar_init(bar_acc, 1);
@@ -105,13 +119,21 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
     fence_proxy_async_smem();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(const_cast<uint32_t*>(&s_misc[0])), p.tmem_cols);
-    tmem_relinquish();
+    if (kPair) {
+      tmem_alloc_pair(smem_u32(const_cast<uint32_t*>(&s_misc[0])), p.tmem_cols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(const_cast<uint32_t*>(&s_misc[0])), p.tmem_cols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if (kPair) cluster_sync();  // both CTAs' barriers exist before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = s_misc[0];
+  // full barriers that loads and arrivals count on: the even CTA's for a pair
+  const uint32_t full_tgt = kPair ? mapa_shared(bar_full, 0) : bar_full;
 
   if (warp == 0) {
     // ---------------------------------------------------------- weight loader
@@ -127,18 +149,28 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
             ok = false;
             break;
           }
-          const uint32_t full = bar_full + 8 * stage;
-          mbar_arrive_expect_tx(full, b_bytes + (k3 ? 0u : a_bytes));
-          if (!k3) tma_load_2d(sbase + L.a_off + stage * a_bytes, &fmap, full, kb * p.kb_elems,
-                               static_cast<int32_t>(tile * kTileRows));
-          tma_load_3d(sbase + L.b_off + stage * b_bytes, &wmap, full, kb * p.kb_elems, k3 ? d : 0, n0);
+          const uint32_t full = full_tgt + 8 * stage;
+          const uint32_t a_dst = sbase + L.a_off + stage * a_bytes, b_dst = sbase + L.b_off + stage * b_bytes;
+          const int32_t a_row = static_cast<int32_t>(tile * kTileRows);
+          const int32_t b_row = n0 + static_cast<int32_t>(rank) * bn_cta;
+          if (kPair) {
+            mbar_arrive_expect_tx_cluster(full, b_bytes + (k3 ? 0u : a_bytes));
+            if (!k3) tma_load_2d_pair(a_dst, &fmap, full, kb * p.kb_elems, a_row);
+            tma_load_3d_pair(b_dst, &wmap, full, kb * p.kb_elems, k3 ? d : 0, b_row);
+          } else {
+            mbar_arrive_expect_tx(full, b_bytes + (k3 ? 0u : a_bytes));
+            if (!k3) tma_load_2d(a_dst, &fmap, full, kb * p.kb_elems, a_row);
+            tma_load_3d(b_dst, &wmap, full, kb * p.kb_elems, k3 ? d : 0, b_row);
+          }
         }
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_f16(static_cast<uint32_t>(p.is_bf16), static_cast<uint32_t>(p.bn));
+    // (for a pair only the even CTA issues; the odd one only holds TMEM)
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc =
+          idesc_f16(static_cast<uint32_t>(p.is_bf16), static_cast<uint32_t>(p.bn), kPair ? 256u : 128u);
       uint32_t it = 0;
       bool ok = true;
       for (uint32_t m = mask; m && ok; m &= m - 1) {
@@ -153,12 +185,16 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
           const uint64_t adesc = kmajor_desc(sbase + L.a_off + stage * a_bytes, row_bytes);
           const uint64_t bdesc = kmajor_desc(sbase + L.b_off + stage * b_bytes, row_bytes);
           const int ksteps = kb == kblocks - 1 ? last_ksteps : p.kb_elems / 16;
-          for (int k = 0; k < ksteps; ++k)
-            umma_f16(tmem_base, adesc + 2 * k, bdesc + 2 * k, idesc, (it > 0 || k > 0) ? 1u : 0u);
-          umma_commit(bar_empty + 8 * stage);
+          for (int k = 0; k < ksteps; ++k) {
+            if (kPair) umma_f16_pair(tmem_base, adesc + 2 * k, bdesc + 2 * k, idesc, (it > 0 || k > 0) ? 1u : 0u);
+            else umma_f16(tmem_base, adesc + 2 * k, bdesc + 2 * k, idesc, (it > 0 || k > 0) ? 1u : 0u);
+          }
+          if (kPair) umma_commit_pair(bar_empty + 8 * stage, 3);
+          else umma_commit(bar_empty + 8 * stage);
         }
       }
-      umma_commit(bar_acc);
+      if (kPair) umma_commit_pair(bar_acc, 3);
+      else umma_commit(bar_acc);
     }
   } else {
     // Gather / epilogue warps: this thread's tile row and its neighbour rows.
@@ -194,12 +230,17 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
             ok = false;
             break;
           }
-          const uint32_t full = bar_full + 8 * stage;
-          if (lane == 0) mbar_arrive_expect_tx(full, 32u * row_bytes);
+          const uint32_t full = full_tgt + 8 * stage;
+          if (lane == 0) {
+            if (kPair) mbar_arrive_expect_tx_cluster(full, 32u * row_bytes);
+            else mbar_arrive_expect_tx(full, 32u * row_bytes);
+          }
           __syncwarp();
-          if (lane < 8)
-            tma_gather4(sbase + L.a_off + stage * a_bytes + (q * 32 + 4 * lane) * row_bytes, &fmap, full,
-                        kb * p.kb_elems, r0, r1, r2, r3);
+          if (lane < 8) {
+            const uint32_t dst = sbase + L.a_off + stage * a_bytes + (q * 32 + 4 * lane) * row_bytes;
+            if (kPair) tma_gather4_pair(dst, &fmap, full, kb * p.kb_elems, r0, r1, r2, r3);
+            else tma_gather4(dst, &fmap, full, kb * p.kb_elems, r0, r1, r2, r3);
+          }
         }
       }
     }
@@ -248,9 +289,11 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
   }
   tc_fence_before();
   __syncthreads();
+  if (kPair) cluster_sync();  // every MMA of the pair is done and both CTAs have read their TMEM
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, p.tmem_cols);
+    if (kPair) tmem_dealloc_pair(tmem_base, p.tmem_cols);
+    else tmem_dealloc(tmem_base, p.tmem_cols);
   }
 }
 
@@ -283,44 +326,60 @@ static uint32_t next_pow2(uint32_t x) {
   return v;
 }
 
-// Launch shape of one conv: channel split, channel block and stage count.
+// Launch shape of one conv: channel split, channel block, CTA pairing and stage count.
 struct TcShape {
   int nsplit, bn, kb_elems, stages, ctas_per_sm;
+  bool pair;
   uint32_t tmem_cols, smem;
 };
 
-static TcShape choose_shape(int cin, int cout) {
+static std::atomic<int> g_conv_variant{0};
+
+static TcShape choose_shape(int cin, int cout, int64_t ntiles) {
   TcShape t;
-  // At most 256 output channels (one MMA N) per CTA; blocks of <= 128 let
-  // four CTAs share an SM's 512 TMEM columns.
+  // At most 256 output channels (one MMA N) per CTA or CTA pair.
   t.nsplit = (cout + 255) / 256;
   t.bn = ((cout + t.nsplit - 1) / t.nsplit + 15) / 16 * 16;
   t.tmem_cols = next_pow2(t.bn < 32 ? 32u : static_cast<uint32_t>(t.bn));
+  // CTA pairs halve the weight bytes each CTA pulls through its TMA path, but
+  // a cluster launch of a kernel that uses tcgen05 is limited to one cluster
+  // per TPC (74 on B200, from the occupancy API and ncu), i.e. one CTA per
+  // SM, and this kernel's row-gather rate grows with the CTAs per SM.  The
+  // pairs measured 1.5-1.7x slower on every workload, so one CTA per tile is
+  // the default and pairs are kept as a selectable, tested alternative.
+  (void)ntiles;
+  t.pair = g_conv_variant.load() == 2;
+  const int bn_cta = t.pair ? t.bn / 2 : t.bn;
   // 64-channel blocks (128-byte rows): one row request per gathered row and
   // K block.  Measured faster than 32-channel blocks with more CTAs per SM
   // (shells 128^3/128ch: 122 us vs 180 us), so the SM holds three CTAs of two
-  // stages each when BN <= 128.
+  // or more stages each when BN <= 128.
+  // (Pairs use the same per-CTA budget: sized for one CTA per SM, with
+  // eight stages, they measured slower still.)
   t.ctas_per_sm = t.tmem_cols <= 128 ? 3 : 2;
   t.kb_elems = 64;
   (void)cin;
   const uint32_t per_sm = 228u * 1024u;
   const uint32_t budget = per_sm / t.ctas_per_sm - 1024u;  // 1 KB per CTA is reserved by the system
-  const uint32_t stage_bytes = static_cast<uint32_t>(kTileRows + t.bn) * t.kb_elems * 2;
-  const uint32_t fixed = tc_layout(0, t.bn, t.kb_elems).total + 1024u;
+  const uint32_t stage_bytes = static_cast<uint32_t>(kTileRows + bn_cta) * t.kb_elems * 2;
+  const uint32_t fixed = tc_layout(0, bn_cta, t.kb_elems).total + 1024u;
   int stages = budget > fixed ? static_cast<int>((budget - fixed) / stage_bytes) : 0;
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) stages = 2;
   t.stages = stages;
-  t.smem = tc_layout(stages, t.bn, t.kb_elems).total + 1024u;
+  t.smem = tc_layout(stages, bn_cta, t.kb_elems).total + 1024u;
   return t;
 }
+
+void set_conv_variant(int v) { g_conv_variant.store(v); }
 
 cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s) {
   if (a.n == 0) return cudaSuccess;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   const CUtensorMapDataType dt = a.dtype == kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  const TcShape t = choose_shape(a.cin, a.cout);
+  const int64_t ntiles = (a.n + kTileRows - 1) / kTileRows;
+  const TcShape t = choose_shape(a.cin, a.cout, ntiles);
   const CUtensorMapSwizzle sw = t.kb_elems == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
 
   CUtensorMap fmap, wmap;
@@ -336,19 +395,18 @@ cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s) {
       return cudaErrorInvalidValue;
   }
   {
-    // weight [cout, taps, cin]
+    // weight [cout, taps, cin]; a CTA of a pair loads half of the block's rows
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(a.cin), static_cast<cuuint64_t>(a.taps),
                                 static_cast<cuuint64_t>(a.cout)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(a.cin) * 2,
                                    static_cast<cuuint64_t>(a.cin) * a.taps * 2};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(t.kb_elems), 1, static_cast<cuuint32_t>(t.bn)};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(t.kb_elems), 1,
+                               static_cast<cuuint32_t>(t.pair ? t.bn / 2 : t.bn)};
     const cuuint32_t estr[3] = {1, 1, 1};
     if (enc(&wmap, dt, 3, const_cast<void*>(a.weight), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  cudaError_t e = cudaFuncSetAttribute(k_conv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(t.smem));
-  if (e != cudaSuccess) return e;
   TcParams p;
   p.nbr = a.nbr;
   p.perm = a.perm;
@@ -357,6 +415,7 @@ cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s) {
   p.out = static_cast<uint16_t*>(a.out);
   p.err = a.err;
   p.n = a.n;
+  p.ntiles = ntiles;
   p.cin = a.cin;
   p.cout = a.cout;
   p.taps = a.taps;
@@ -367,10 +426,33 @@ cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s) {
   p.is_bf16 = a.dtype == kBF16 ? 1 : 0;
   p.kb_elems = t.kb_elems;
   p.tmem_cols = t.tmem_cols;
-  const int64_t units = (a.n + kTileRows - 1) / kTileRows * t.nsplit;
-  k_conv_tc<<<static_cast<unsigned>(units), kTcThreads, t.smem, s>>>(fmap, wmap, p);
+  cudaError_t e;
+  if (t.pair) {
+    e = cudaFuncSetAttribute(k_conv_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(t.smem));
+    if (e != cudaSuccess) return e;
+    const int64_t ctas = 2 * ((ntiles + 1) / 2) * t.nsplit;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
+    cfg.blockDim = dim3(kTcThreads, 1, 1);
+    cfg.dynamicSmemBytes = t.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k_conv_tc<true>, fmap, wmap, p);
+  } else {
+    e = cudaFuncSetAttribute(k_conv_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(t.smem));
+    if (e != cudaSuccess) return e;
+    const int64_t units = ntiles * t.nsplit;
+    k_conv_tc<false><<<static_cast<unsigned>(units), kTcThreads, t.smem, s>>>(fmap, wmap, p);
+    e = cudaGetLastError();
+  }
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace smc

@@ -92,6 +92,8 @@ cudaError_t launch_conv_simt(const ConvArgs& a, cudaStream_t s);
 // tcgen05 kernel: bf16/fp16, cin % 16 == 0 and cin >= 64, cout % 16 == 0, 16-byte aligned.
 bool conv_tc_supported(const ConvArgs& a);
 cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s);
+// Tensor-core kernel variant: 0 = by shape, 1 = one CTA per tile, 2 = CTA pairs.
+void set_conv_variant(int v);
 
 
 }  // namespace smc

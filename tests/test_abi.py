@@ -35,6 +35,9 @@ def test_strerror_without_gpu():
     assert lib.smc_strerror(-3) == b"duplicate coordinate"
     assert lib.smc_set_hash_capacity(-1) == -1
     assert lib.smc_set_hash_capacity(0) == 0
+    assert lib.smc_set_conv_variant(3) == -1
+    assert lib.smc_set_conv_variant(-1) == -1
+    assert lib.smc_set_conv_variant(0) == 0
 
 
 def test_argument_errors_without_gpu():

@@ -63,6 +63,15 @@ def check_close(got, ref, dtype, what=""):
     assert err <= TOL[dtype] * scale, f"{what}: max err {err:.3e} vs bound {TOL[dtype] * scale:.3e}"
 
 
+@pytest.fixture(params=[1, 2], ids=["one_cta", "cta_pair"])
+def conv_variant(request):
+    """Runs a test on both tensor-core kernels: one CTA per 128-row tile, and
+    CTA pairs sharing M = 256 MMAs."""
+    smc.set_conv_variant(request.param)
+    yield request.param
+    smc.set_conv_variant(0)
+
+
 def sample_rows(n, k, seed):
     if n <= k:
         return None
@@ -203,7 +212,7 @@ def test_conv_shell2_stacked(oracle_mod, dtype):
 
 
 @pytest.mark.parametrize("orientation", [1, -1])
-def test_conv_shells6_bf16(oracle_mod, orientation):
+def test_conv_shells6_bf16(oracle_mod, orientation, conv_variant):
     w = workload("shells6")
     m = build(w)
     f, wt, b = _layer(w, "bf16")
@@ -221,7 +230,7 @@ def test_conv_full128_bf16_sampled(oracle_mod):
     check_close(got, ref, "bf16", "full128")
 
 
-def test_conv_varlen4_f16_k3_then_k1(oracle_mod):
+def test_conv_varlen4_f16_k3_then_k1(oracle_mod, conv_variant):
     w = workload("varlen4")
     m = build(w, key="varlen4")
     f, wt, b = _layer(w, "f16", 0, 3)
@@ -260,7 +269,7 @@ def test_conv_decoder_stage(oracle_mod, stage):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("orientation", [1, -1])
-def test_conv_small_integers_bit_exact(oracle_mod, dtype, orientation):
+def test_conv_small_integers_bit_exact(oracle_mod, dtype, orientation, conv_variant):
     """Inputs in {-1, 0, 1}: every partial sum is a small integer, so the
     result is exact in any accumulation order and must match bit for bit."""
     w = workload("shell2")
@@ -277,7 +286,7 @@ def test_conv_small_integers_bit_exact(oracle_mod, dtype, orientation):
 
 
 @pytest.mark.parametrize("cin,cout", [(64, 16), (64, 512), (96, 48), (48, 64), (200, 24), (128, 272)])
-def test_conv_channel_shapes_bf16(oracle_mod, cin, cout):
+def test_conv_channel_shapes_bf16(oracle_mod, cin, cout, conv_variant):
     """Tensor-core path with ragged K blocks, narrow and split N tiles; shapes
     outside its limits run on the FMA kernel; all must meet the same bar."""
     w = workload("shell2")
@@ -289,9 +298,12 @@ def test_conv_channel_shapes_bf16(oracle_mod, cin, cout):
         check_close(got, ref, "bf16", f"cin={cin} cout={cout} s={s}")
 
 
-def test_conv_ragged_tail_and_no_bias(oracle_mod):
+@pytest.mark.parametrize("rows", [128 * 5 + 37, 128 * 6 + 5, 100])
+def test_conv_ragged_tail_and_no_bias(oracle_mod, rows, conv_variant):
+    """Ragged last tile; an odd tile count (the last CTA pair has no second
+    tile); a single partial tile."""
     w = workload("shell2")
-    coords = w.coords[: 128 * 5 + 37]
+    coords = w.coords[:rows]
     sub = S.Workload("ragged", coords, w.grid, 64, 64, ("bf16",))
     m = build(sub)
     f, wt, _ = _layer(sub, "bf16", 3)
@@ -299,6 +311,24 @@ def test_conv_ragged_tail_and_no_bias(oracle_mod):
         out = smc.conv(m, dev(f, dtype), dev(wt, dtype), None)
         ref = oracle_mod.conv(coords, w.grid, f, wt, None, 3, 1)
         check_close(host(out), ref, dtype, f"ragged {dtype}")
+    smc.status()
+
+
+@pytest.mark.parametrize("name,dtype", [("shells6", "bf16"), ("decoder3", "bf16"), ("varlen4", "f16")])
+def test_conv_variants_agree(name, dtype):
+    """Both tensor-core kernels give the same output bits: a pair issues the
+    union of its two tiles' taps, and a tap a row lacks adds exact zeros."""
+    w = workload(name)
+    m = build(w)
+    f, wt, b = _layer(w, dtype)
+    outs = []
+    for v in (1, 2):
+        smc.set_conv_variant(v)
+        try:
+            outs.append(smc.conv(m, dev(f, dtype), dev(wt, dtype), dev(b, dtype)).cpu())
+        finally:
+            smc.set_conv_variant(0)
+    assert torch.equal(outs[0], outs[1])
     smc.status()
 
 
