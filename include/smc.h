@@ -190,6 +190,13 @@ SMC_API const char* smc_strerror(int code);
  *   with the tile schedule; measured from the end of the lookups).
  * smc_kernel_launches: number of CUDA kernels this library has launched in
  *   the process so far (memsets and copies excluded).
+ * smc_set_map_lookup: lookup structure of later builds: 0 = by size
+ *   (default: a dense int32 index grid over the batch x Z x Y x X box when it
+ *   has at most 2^28 sites and at most 256 sites per voxel, else a hash
+ *   table), 1 = hash table, 2 = dense grid whenever the box has at most 2^28
+ *   sites.  Maps are identical either way.  A forced hash capacity
+ *   (smc_set_hash_capacity) always selects the hash table.  SMC_E_ARG for
+ *   any other value.
  * smc_set_conv_variant: tensor-core conv kernel for later convs: 0 = default
  *   (currently the same as 1), 1 = one CTA per 128-row tile, 2 = CTA pairs (a
  *   cluster of two CTAs sharing M = 256 tcgen05 MMAs, each loading half of
@@ -232,6 +239,7 @@ SMC_API int smc_set_profiling(int32_t on);
 SMC_API int smc_map_timing(const smc_map* map, float ms[3]);
 SMC_API int smc_kernel_launches(int64_t* count);
 SMC_API int smc_set_conv_variant(int32_t variant);
+SMC_API int smc_set_map_lookup(int32_t mode);
 
 #ifdef __cplusplus
 }

@@ -30,6 +30,7 @@ EXPORTS = [
     "smc_map_schedule", "smc_free_map", "smc_status", "smc_strerror",
     "smc_set_hash_capacity", "smc_set_profiling", "smc_map_timing", "smc_kernel_launches",
     "smc_build_map_async", "smc_map_wait", "smc_neighbour_map_noalloc", "smc_set_conv_variant",
+    "smc_set_map_lookup",
 ]
 
 
@@ -72,6 +73,7 @@ def lib() -> ctypes.CDLL:
         L.smc_map_timing.argtypes = [P, P]
         L.smc_kernel_launches.argtypes = [P]
         L.smc_set_conv_variant.argtypes = [i32]
+        L.smc_set_map_lookup.argtypes = [i32]
         for name in EXPORTS:
             if name != "smc_strerror":
                 getattr(L, name).restype = ctypes.c_int
@@ -296,6 +298,11 @@ def status(stream=None) -> None:
 def set_conv_variant(variant: int) -> None:
     """Tensor-core conv kernel: 0 by shape, 1 one CTA per tile, 2 CTA pairs."""
     _check(lib().smc_set_conv_variant(int(variant)), "smc_set_conv_variant")
+
+
+def set_map_lookup(mode: int) -> None:
+    """Lookup structure of later builds: 0 by size, 1 hash table, 2 dense grid."""
+    _check(lib().smc_set_map_lookup(int(mode)), "smc_set_map_lookup")
 
 
 def set_hash_capacity(slots: int) -> None:

@@ -36,6 +36,7 @@ struct smc_map {
   int32_t* perm;
   uint32_t* tile_mask;
   void* keep;           // one allocation holding nbr, pairs, schedule and tile masks
+  mutable void* tmp;    // the build's scratch, released at the first wait on the map
   cudaEvent_t done;     // recorded after the status block is copied back
   cudaEvent_t prof[4];  // optional timing events
   HostSlot* slot;       // pinned status block
@@ -53,6 +54,11 @@ namespace {
 std::atomic<int64_t> g_capacity_override{0};
 std::atomic<long long> g_launches{0};
 std::atomic<int32_t> g_profiling{0};
+std::atomic<int32_t> g_map_lookup{0};
+
+// Largest box (batch * Z * Y * X sites) that gets a dense index grid: 1 GB of
+// int32, cleared at every build.
+constexpr double kDenseMaxSites = 268435456.0;
 
 constexpr int kMaxDevices = 64;
 
@@ -114,17 +120,20 @@ cudaStream_t side_stream(int dev) {
 std::mutex g_ev_mu;
 std::vector<cudaEvent_t> g_events[kMaxDevices];
 
-cudaEvent_t take_event(int dev) {
+std::vector<cudaEvent_t> g_timing_events[kMaxDevices];  // the same, with timing (profiling)
+
+cudaEvent_t take_event(int dev, bool timing = false) {
   {
     std::lock_guard<std::mutex> lk(g_ev_mu);
-    if (!g_events[dev].empty()) {
-      cudaEvent_t e = g_events[dev].back();
-      g_events[dev].pop_back();
+    std::vector<cudaEvent_t>& pool = timing ? g_timing_events[dev] : g_events[dev];
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
       return e;
     }
   }
   cudaEvent_t e = nullptr;
-  if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+  if (cudaEventCreateWithFlags(&e, timing ? cudaEventDefault : cudaEventDisableTiming) != cudaSuccess) {
     cudaGetLastError();
     return nullptr;
   }
@@ -132,11 +141,12 @@ cudaEvent_t take_event(int dev) {
 }
 
 // An event may go back once every wait on it has been enqueued (a wait binds
-// to the record made before it) or, for a completion event, once it is done.
-void give_event(int dev, cudaEvent_t e) {
+// to the record made before it) or, for a completion or timing event, once
+// it is done.
+void give_event(int dev, cudaEvent_t e, bool timing = false) {
   if (!e) return;
   std::lock_guard<std::mutex> lk(g_ev_mu);
-  g_events[dev].push_back(e);
+  (timing ? g_timing_events[dev] : g_events[dev]).push_back(e);
 }
 
 // Pinned host status blocks, handed out from chunks of 256.
@@ -186,16 +196,32 @@ bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
   return a0 < b0 + nb && b0 < a0 + na;
 }
 
+// The build's scratch goes back to the pool on the build stream once the
+// build is known complete (its completion event has been waited on).  Freed
+// there, the next build on that stream reuses it; released on the side
+// stream, where its last user runs, it was never reused and the pool grew
+// by the scratch size at every build.
+void release_scratch(const smc_map* m) {
+  if (!m->tmp) return;
+  int cur = 0;
+  cudaGetDevice(&cur);
+  if (cur != m->device) cudaSetDevice(m->device);
+  cudaFreeAsync(m->tmp, m->stream);
+  m->tmp = nullptr;
+  if (cur != m->device) cudaSetDevice(cur);
+  cudaGetLastError();
+}
+
 void release_map(smc_map* m) {
   if (!m) return;
   int cur = 0;
   cudaGetDevice(&cur);
   if (cur != m->device) cudaSetDevice(m->device);
   if (m->done) cudaEventSynchronize(m->done);  // the status copy must land before the slot is reused
+  release_scratch(m);
   if (m->keep) cudaFreeAsync(m->keep, m->stream);
   give_event(m->device, m->done);
-  for (auto& e : m->prof)
-    if (e) cudaEventDestroy(e);
+  for (auto& e : m->prof) give_event(m->device, e, true);
   give_slot(m->slot);
   if (cur != m->device) cudaSetDevice(cur);
   cudaGetLastError();
@@ -211,6 +237,7 @@ int resolve(const smc_map* m) {
     cudaGetLastError();
     rc = SMC_E_CUDA;
   } else if (m->slot) {
+    release_scratch(m);
     const uint32_t err = m->slot->err;
     if (err & smc::kErrRange) rc = SMC_E_RANGE;
     else if (err & smc::kErrDuplicate) rc = SMC_E_DUPLICATE;
@@ -267,9 +294,16 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   }
 
   // ---- sizes
-  const bool wide = sites > 4294967294.0;  // packed slots need keys < 2^32 - 1
-  int lg = 4;
+  // Lookup structure.  A dense index grid turns each row's 27 lookups into 9
+  // runs of three consecutive sites, which neighbouring rows share; it is
+  // used when the box is at most 256 sites per voxel (clearing it then costs
+  // less than hash probing) and at most 2^28 sites.  Otherwise a hash table.
   const int64_t forced = g_capacity_override.load();
+  const int lookup = g_map_lookup.load();
+  const bool dense = forced == 0 && sites <= kDenseMaxSites &&
+                     (lookup == 2 || (lookup == 0 && sites <= 256.0 * static_cast<double>(n)));
+  const bool wide = !dense && sites > 4294967294.0;  // packed slots need keys < 2^32 - 1
+  int lg = 4;
   // Packed slots: load <= 1/4, so lookups (which read 2-slot groups) resolve
   // in one round almost always (measured: 256^3 shells+planes map 0.59 ms at
   // 1/4 vs 0.83 ms at 1/2).  Two-word slots: load <= 1/2.
@@ -289,7 +323,9 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   const size_t o_perm = keep.take<int32_t>(n);
   const size_t o_tmask = keep.take<uint32_t>((n + smc::kTileRows - 1) / smc::kTileRows);
   Carve tmp;
-  const size_t o_table = tmp.take<unsigned long long>(wide ? 2 * cap : cap);
+  const size_t table_bytes = dense ? static_cast<size_t>(sites) * sizeof(int32_t)
+                                   : (wide ? 2 : 1) * static_cast<size_t>(cap) * sizeof(unsigned long long);
+  const size_t o_table = tmp.take<uint8_t>(table_bytes);
   const size_t o_gkey = tmp.take<uint32_t>(n);
   const size_t o_bc = tmp.take<int32_t>(Lmap);
   const size_t o_bo = tmp.take<int64_t>(Lmap);
@@ -332,7 +368,7 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   m->tile_mask = reinterpret_cast<uint32_t*>(K + o_tmask);
 
   if (g_profiling.load() != 0)
-    for (auto& e : m->prof) cudaEventCreate(&e);
+    for (auto& e : m->prof) e = take_event(m->device, true);
 
   uint32_t* err = reinterpret_cast<uint32_t*>(T + o_err + offsetof(HostSlot, err));
   uint32_t* tickets = reinterpret_cast<uint32_t*>(T + o_tick);
@@ -343,7 +379,7 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   a.Z = grid[0];
   a.Y = grid[1];
   a.X = grid[2];
-  a.wide = wide;
+  a.kind = dense ? smc::kMapDense : (wide ? smc::kMapWide : smc::kMapPacked);
   a.table = reinterpret_cast<unsigned long long*>(T + o_table);
   a.lg = lg;
   a.err = err;
@@ -379,7 +415,7 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   // schedule is done too -- the status copy, the completion event and the
   // release of the scratch.  A conv enqueued on s behind the build waits for
   // the schedule only, and overlaps the pair lists.
-  cudaError_t ce = cudaMemsetAsync(T + o_table, 0xFF, (wide ? 2 : 1) * cap * sizeof(unsigned long long), s);
+  cudaError_t ce = cudaMemsetAsync(T + o_table, 0xFF, table_bytes, s);
   if (ce == cudaSuccess) ce = cudaMemsetAsync(T + o_err, 0, zero_bytes, s);
   if (ce == cudaSuccess && m->prof[0]) ce = cudaEventRecord(m->prof[0], s);
   if (ce == cudaSuccess) ce = smc::launch_map_lookups(a, s);
@@ -395,6 +431,7 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   // the only device->host traffic: error bits and pair offsets, into pinned memory
   if (ce == cudaSuccess) ce = cudaMemcpyAsync(m->slot, T + o_err, sizeof(HostSlot), cudaMemcpyDeviceToHost, side);
   if (ce == cudaSuccess) ce = cudaEventRecord(m->done, side);
+  m->tmp = tp;  // released after the first wait on the map (release_scratch)
   give_event(m->device, ev_fork);  // their waits are enqueued
   give_event(m->device, ev_sched);
   if (ce != cudaSuccess) {
@@ -402,11 +439,10 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
     cudaStreamSynchronize(s);
     cudaStreamSynchronize(side);
     cudaGetLastError();
-    cudaFreeAsync(tp, s);
+    m->tmp = tp;
     release_map(m);
     return SMC_E_CUDA;
   }
-  cudaFreeAsync(tp, side);
   *out = m;
   return SMC_OK;
 }
@@ -440,6 +476,12 @@ const char* smc_strerror(int code) {
 int smc_set_hash_capacity(int64_t slots) {
   if (slots < 0) return SMC_E_ARG;
   g_capacity_override.store(slots);
+  return SMC_OK;
+}
+
+int smc_set_map_lookup(int32_t mode) {
+  if (mode < 0 || mode > 2) return SMC_E_ARG;
+  g_map_lookup.store(mode);
   return SMC_OK;
 }
 

@@ -7,12 +7,15 @@
 
 namespace smc {
 
+// Lookup structure of a map build (see map_build.cu).
+enum MapKind : int { kMapPacked = 0, kMapWide = 1, kMapDense = 2 };
+
 struct MapBuildArgs {
   const int32_t* coords;  // [n, 4] (b, z, y, x)
   int64_t n;
   int32_t batch, Z, Y, X;
-  bool wide;                   // two-word hash slots (keys >= 2^32 - 1)
-  unsigned long long* table;   // 2^lg slots, pre-filled with ~0
+  int kind;                    // MapKind
+  unsigned long long* table;   // hash: 2^lg slots pre-filled with ~0; dense: int32 grid pre-filled with -1
   int lg;
   uint32_t* err;               // error bits (zeroed)
   uint32_t* zero;              // [nzero] words k_insert clears (the tile tap masks)

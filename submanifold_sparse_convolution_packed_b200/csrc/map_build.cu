@@ -20,6 +20,7 @@
 //                 scatter; the first scatter also counts the second digit,
 //                 the second one ORs the tile tap masks.
 #include <cstdint>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -47,9 +48,11 @@ __device__ __forceinline__ uint64_t site_key(int4 c, int32_t Z, int32_t Y, int32
   return ((static_cast<uint64_t>(c.x) * Z + c.y) * Y + c.z) * X + c.w;
 }
 
-// Packed layout: one word per slot, (key << 32) | row, for keys < 2^32 - 1.
-// Wide layout: two words per slot, key then row.
-template <bool kWide>
+// Lookup structures (MapKind): packed hash slots, one word (key << 32) | row,
+// for keys < 2^32 - 1; wide hash slots, two words, key then row; or a dense
+// index grid, one int32 row (-1 = empty) per site of the batch x Z x Y x X
+// box, for boxes small enough to clear at every build.
+template <int kKind>
 __global__ void __launch_bounds__(256) k_insert(const int4* __restrict__ coords, int64_t n, int32_t batch,
                                                 int32_t Z, int32_t Y, int32_t X,
                                                 unsigned long long* table, int lg, uint32_t* err,
@@ -67,10 +70,15 @@ __global__ void __launch_bounds__(256) k_insert(const int4* __restrict__ coords,
       continue;
     }
     const uint64_t key = site_key(c, Z, Y, X);
+    if (kKind == kMapDense) {
+      const int prev = atomicCAS(reinterpret_cast<int*>(table) + key, -1, static_cast<int>(v));
+      if (prev != -1) atomicOr(err, kErrDuplicate);
+      continue;
+    }
     uint64_t s = slot_of(key, lg);
     bool placed = false;
     for (uint64_t probe = 0; probe <= mask; ++probe) {
-      if (!kWide) {
+      if (kKind == kMapPacked) {
         const unsigned long long want = (key << 32) | static_cast<uint32_t>(v);
         const unsigned long long prev = atomicCAS(&table[s], kEmpty, want);
         if (prev == kEmpty) { placed = true; break; }
@@ -87,11 +95,11 @@ __global__ void __launch_bounds__(256) k_insert(const int4* __restrict__ coords,
 }
 
 // Linear probing from slot s; at most one pass over the table.
-template <bool kWide>
+template <int kKind>
 __device__ __noinline__ int32_t lookup_from(const unsigned long long* __restrict__ table, uint64_t mask,
                                             uint64_t s, uint64_t key) {
   for (uint64_t probe = 0; probe <= mask; ++probe) {
-    if (!kWide) {
+    if (kKind == kMapPacked) {
       const uint64_t e = __ldg(&table[s]);
       if (e == kEmpty) return -1;
       if ((e >> 32) == key) return static_cast<int32_t>(e & 0xFFFFFFFFull);
@@ -134,7 +142,7 @@ __device__ __forceinline__ uint32_t key_hits(uint32_t k) {
   return m;
 }
 
-template <bool kWide>
+template <int kKind>
 __global__ void __launch_bounds__(kMapBlock) k_neighbours(
     const int4* __restrict__ coords, int64_t n, int32_t Z, int32_t Y, int32_t X,
     const unsigned long long* __restrict__ table, int lg, int32_t* __restrict__ nbr,
@@ -151,7 +159,24 @@ __global__ void __launch_bounds__(kMapBlock) k_neighbours(
     const int4 c = coords[v];
     const uint64_t key = site_key(c, Z, Y, X);
     const int64_t sz = static_cast<int64_t>(Y) * X;
-    if (kWide) {
+    if (kKind == kMapDense) {
+      // dense grid: the 9 (dz, dy) lines, three consecutive x sites each
+      const int32_t* __restrict__ g = reinterpret_cast<const int32_t*>(table);
+#pragma unroll
+      for (int l = 0; l < 9; ++l) {
+        const int dz = l / 3 - 1, dy = l % 3 - 1;
+        const bool line = c.y + dz >= 0 && c.y + dz < Z && c.z + dy >= 0 && c.z + dy < Y;
+        const int64_t at = static_cast<int64_t>(key) + dz * sz + static_cast<int64_t>(dy) * X;
+        const int32_t r0 = line && c.w > 0 ? __ldg(g + at - 1) : -1;
+        const int32_t r1 = line ? __ldg(g + at) : -1;
+        const int32_t r2 = line && c.w + 1 < X ? __ldg(g + at + 1) : -1;
+        s_nbr[tid * kTaps + 3 * l + 0] = r0;
+        s_nbr[tid * kTaps + 3 * l + 1] = r1;
+        s_nbr[tid * kTaps + 3 * l + 2] = r2;
+        hits |= (static_cast<uint32_t>(r0 >= 0) | static_cast<uint32_t>(r1 >= 0) << 1 |
+                 static_cast<uint32_t>(r2 >= 0) << 2) << (3 * l);
+      }
+    } else if (kKind == kMapWide) {
       // two-word slots: plain linear probing per lookup
 #pragma unroll 1
       for (int d = 0; d < kTaps; ++d) {
@@ -159,7 +184,7 @@ __global__ void __launch_bounds__(kMapBlock) k_neighbours(
         int32_t r = -1;
         if (c.y + dz >= 0 && c.y + dz < Z && c.z + dy >= 0 && c.z + dy < Y && c.w + dx >= 0 && c.w + dx < X) {
           const uint64_t nk = key + static_cast<uint64_t>(dz * sz + static_cast<int64_t>(dy) * X + dx);
-          r = lookup_from<true>(table, mask, slot_of(nk, lg), nk);
+          r = lookup_from<kMapWide>(table, mask, slot_of(nk, lg), nk);
         }
         s_nbr[tid * kTaps + d] = r;
         hits |= static_cast<uint32_t>(r >= 0) << d;
@@ -552,17 +577,16 @@ cudaError_t launch_map_lookups(const MapBuildArgs& a, cudaStream_t s) {
   const int nb = map_nblocks(n);
   const int rnb = radix_nblocks(n);
   const int grid_ins = static_cast<int>((n + 255) / 256);
-  if (a.wide) {
-    k_insert<true><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.batch, a.Z, a.Y, a.X,
-                                            a.table, a.lg, a.err, a.zero, a.nzero);
-    k_neighbours<true><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.Z, a.Y, a.X,
-                                                a.table, a.lg, a.nbr, a.gkey, a.block_counts, nb, a.hist1, rnb);
-  } else {
-    k_insert<false><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.batch, a.Z, a.Y, a.X,
-                                             a.table, a.lg, a.err, a.zero, a.nzero);
-    k_neighbours<false><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.Z, a.Y, a.X,
-                                                 a.table, a.lg, a.nbr, a.gkey, a.block_counts, nb, a.hist1, rnb);
-  }
+  auto run = [&](auto kind) {
+    constexpr int K = decltype(kind)::value;
+    k_insert<K><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.batch, a.Z, a.Y, a.X,
+                                         a.table, a.lg, a.err, a.zero, a.nzero);
+    k_neighbours<K><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.Z, a.Y, a.X, a.table,
+                                             a.lg, a.nbr, a.gkey, a.block_counts, nb, a.hist1, rnb);
+  };
+  if (a.kind == kMapDense) run(std::integral_constant<int, kMapDense>());
+  else if (a.kind == kMapWide) run(std::integral_constant<int, kMapWide>());
+  else run(std::integral_constant<int, kMapPacked>());
   count_launches(2);
   return cudaGetLastError();
 }
@@ -587,9 +611,9 @@ cudaError_t launch_neighbour_map_only(const int32_t* coords, int64_t n, int32_t 
   if (n == 0) return cudaSuccess;
   const int nb = map_nblocks(n);
   const int grid_ins = static_cast<int>((n + 255) / 256);
-  k_insert<false><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(coords), n, batch, Z, Y, X, table, lg,
-                                           err, nullptr, 0);
-  k_neighbours<false><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(coords), n, Z, Y, X, table, lg, nbr,
+  k_insert<kMapPacked><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(coords), n, batch, Z, Y, X, table,
+                                                lg, err, nullptr, 0);
+  k_neighbours<kMapPacked><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(coords), n, Z, Y, X, table, lg, nbr,
                                                gkey, block_counts, nb, nullptr, 0);
   count_launches(2);
   return cudaGetLastError();

@@ -79,6 +79,14 @@ def sample_rows(n, k, seed):
 
 
 # ------------------------------------------------------------------ map
+@pytest.fixture(params=[1, 2], ids=["hash", "dense_grid"])
+def map_lookup(request):
+    """Runs a test with each lookup structure of the map build."""
+    smc.set_map_lookup(request.param)
+    yield request.param
+    smc.set_map_lookup(0)
+
+
 # The tile order of the tensor-core conv: rows stably sorted by a 20-bit key
 # whose bits, most significant first, say whether the 8 corner offsets and
 # then the 12 edge offsets have a neighbour.
@@ -96,7 +104,7 @@ MAP_CASES = ["tiny", "shell2", "shells6", "varlen4", "decoder0", "decoder3", "fu
 
 
 @pytest.mark.parametrize("name", MAP_CASES)
-def test_map_bit_exact(oracle_mod, name):
+def test_map_bit_exact(oracle_mod, name, map_lookup):
     w = workload(name)
     m = build(w)
     nbr = m.nbr().cpu().numpy()
@@ -112,7 +120,7 @@ def test_map_bit_exact(oracle_mod, name):
     np.testing.assert_array_equal(perm, expected_schedule(ref))
 
 
-def test_map_shuffled_rows(oracle_mod):
+def test_map_shuffled_rows(oracle_mod, map_lookup):
     w = workload("shell2")
     rng = np.random.default_rng(1)
     coords = w.coords[rng.permutation(w.n)]
@@ -137,7 +145,7 @@ def test_map_wide_keys(oracle_mod):
     np.testing.assert_array_equal(m.schedule().cpu().numpy(), expected_schedule(ref))
 
 
-def test_map_empty_and_single():
+def test_map_empty_and_single(map_lookup):
     m = smc.build_map(torch.zeros((0, 4), dtype=torch.int32, device="cuda"), (4, 4, 4), batch=1)
     assert m.n == 0 and m.counts == [0] * 27
     out = smc.conv(m, torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda"),
@@ -149,7 +157,7 @@ def test_map_empty_and_single():
     assert one.schedule().cpu().numpy().tolist() == [0]
 
 
-def test_map_errors():
+def test_map_errors(map_lookup):
     def err_of(coords, grid=(8, 8, 8), batch=1):
         with pytest.raises(smc.SmcError) as e:
             smc.build_map(torch.tensor(coords, dtype=torch.int32, device="cuda"), grid, batch=batch)
@@ -368,6 +376,37 @@ def test_async_build_matches_sync(oracle_mod):
     torch.testing.assert_close(out_a, out_s, rtol=0, atol=0)
     np.testing.assert_array_equal(ma.nbr().cpu().numpy(), ms.nbr().cpu().numpy())
     assert ma.counts == ms.counts
+
+
+def test_pipelined_builds_reuse_memory():
+    """Builds enqueued ahead of the host and retired later (the way a job runs
+    them) must reuse the library pool's memory: device memory in use stays
+    flat once the pipeline is full."""
+    w = workload("shells6")
+    coords = torch.from_numpy(w.coords).cuda()
+    f, wt, b = (dev(x, "bf16") for x in _layer(w, "bf16"))
+    out = torch.empty((w.n, w.cout), dtype=torch.bfloat16, device="cuda")
+
+    def run(steps):
+        pending = []
+        for _ in range(steps):
+            m = smc.build_map(coords, w.grid, batch=1, sync=False)
+            smc.conv(m, f, wt, b, out=out)
+            pending.append(m)
+            if len(pending) > 4:
+                old = pending.pop(0)
+                old.wait()
+                old.free()
+        for m in pending:
+            m.wait()
+            m.free()
+        torch.cuda.synchronize()
+        return torch.cuda.mem_get_info()[0]
+
+    free0 = run(12)
+    free1 = run(60)
+    assert free0 - free1 < 64 << 20, f"device memory grew by {(free0 - free1) >> 20} MiB over 60 builds"
+    smc.status()
 
 
 def test_async_build_reports_errors_late():
