@@ -215,22 +215,24 @@ def run_gpu(args):
             self.times, self.conv_times, self.map_times = [], [], []
 
         def submit(self):
-            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            e0, e1, ec, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
             e0.record(stream)
             m = smc.build_map(coords_d, w.grid, batch=batch, stream=stream, sync=False)
             e1.record(stream)
             smc.conv(m, feats_d, w_d, b_d, ksize=3, orientation=1, out=out_d, stream=stream)
+            ec.record(stream)
+            m.stream_wait(stream)  # the step ends when the whole build (pair lists too) is done
             e2.record(stream)
-            self.pending.append((e0, e1, e2, m))
+            self.pending.append((e0, e1, ec, e2, m))
             if len(self.pending) > self.DEPTH:
                 self.retire()
 
         def retire(self):
-            e0, e1, e2, m = self.pending.pop(0)
+            e0, e1, ec, e2, m = self.pending.pop(0)
             e2.synchronize()
             m.wait()  # raises if the build failed on the device
             self.times.append(e0.elapsed_time(e2))
-            self.conv_times.append(e1.elapsed_time(e2))
+            self.conv_times.append(e1.elapsed_time(ec))
             if self.profile:
                 self.map_times.append(m.timing())
             m.free()

@@ -113,6 +113,11 @@ SMC_API int smc_build_map_async(const int32_t* coords, int64_t n, int32_t batch,
 /* Block until the map's build has finished; return its outcome. */
 SMC_API int smc_map_wait(const smc_map* map);
 
+/* Make `stream` wait (on the device, without blocking the host) until the
+ * whole build has finished, pair lists included: work enqueued on `stream`
+ * afterwards may read every part of the map. */
+SMC_API int smc_map_stream_wait(const smc_map* map, void* stream);
+
 /*
  * smc_conv -- one submanifold convolution over a built map.
  *

@@ -30,7 +30,7 @@ EXPORTS = [
     "smc_map_schedule", "smc_free_map", "smc_status", "smc_strerror",
     "smc_set_hash_capacity", "smc_set_profiling", "smc_map_timing", "smc_kernel_launches",
     "smc_build_map_async", "smc_map_wait", "smc_neighbour_map_noalloc", "smc_set_conv_variant",
-    "smc_set_map_lookup",
+    "smc_set_map_lookup", "smc_map_stream_wait",
 ]
 
 
@@ -58,6 +58,7 @@ def lib() -> ctypes.CDLL:
         L.smc_build_map.argtypes = [P, i64, i32, P, P, ctypes.POINTER(P)]
         L.smc_build_map_async.argtypes = [P, i64, i32, P, P, ctypes.POINTER(P)]
         L.smc_map_wait.argtypes = [P]
+        L.smc_map_stream_wait.argtypes = [P, P]
         L.smc_neighbour_map_noalloc.argtypes = [P, i64, i32, P, P, P]
         L.smc_conv.argtypes = [P, P, i64, P, P, P, i64, i32, i32, i32, P]
         L.smc_map_info.argtypes = [P, P, P]
@@ -122,6 +123,12 @@ class Map:
     def wait(self) -> "Map":
         """Block until the build has finished; raise SmcError if it failed."""
         _check(lib().smc_map_wait(self.handle), "smc_build_map")
+        return self
+
+    def stream_wait(self, stream=None) -> "Map":
+        """Make `stream` wait on the device for the whole build, pair lists
+        included (no host synchronisation)."""
+        _check(lib().smc_map_stream_wait(self.handle, _stream(stream)), "smc_map_stream_wait")
         return self
 
     @property

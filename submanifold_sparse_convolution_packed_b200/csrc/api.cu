@@ -506,6 +506,16 @@ int smc_map_wait(const smc_map* map) {
   return resolve(map);
 }
 
+int smc_map_stream_wait(const smc_map* map, void* stream) {
+  if (!map) return SMC_E_ARG;
+  if (!map->done) return SMC_OK;  // empty map: nothing was enqueued
+  if (cudaStreamWaitEvent(static_cast<cudaStream_t>(stream), map->done, 0) != cudaSuccess) {
+    cudaGetLastError();
+    return SMC_E_CUDA;
+  }
+  return SMC_OK;
+}
+
 int smc_build_map(const int32_t* coords, int64_t n, int32_t batch, const int32_t grid[3], void* stream,
                   smc_map** out) {
   smc_map* m = nullptr;

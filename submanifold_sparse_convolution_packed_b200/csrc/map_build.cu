@@ -469,10 +469,13 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_lookback(const int32_t* _
 
 // ------------------------------------------------------------ radix sort
 // Stable scatter of one radix pass over a histogram already scanned into
-// `offsets` ([bins, nblk], digit-major).  The chunk of a block is visited in
-// rounds of 256 consecutive elements; inside a round, an element's rank is
-// (elements of its digit in earlier rounds) + (in earlier warps of this
-// round) + (in earlier lanes of its warp), so the input order is kept.
+// `offsets` ([bins, nblk], digit-major).  Warp w of a block ranks elements
+// 256w .. 256w + 255 of the block's chunk in 8 rounds of 32, keeping a
+// warp-private count per digit in shared memory (no block barrier between
+// rounds); the 8 warps' counts are then scanned per digit on top of the
+// block's base offset.  An element's position is base[digit] + (its digit in
+// earlier warps) + (in earlier rounds of its warp) + (in earlier lanes of its
+// round), so the input order is kept.
 // First pass (kLast false): writes keys and row indices and counts the next
 // digit per destination chunk into hist_next.  Last pass: writes the row
 // order and ORs each row's hit mask into the mask of its 128-row tile.
@@ -482,48 +485,60 @@ __global__ void __launch_bounds__(kRadixThreads) k_radix_scatter(
     const int64_t* __restrict__ offsets, int nblk, uint32_t* __restrict__ keys_out,
     int32_t* __restrict__ vals_out, int32_t* __restrict__ hist_next, uint32_t* __restrict__ tile_mask,
     uint32_t* err) {
-  __shared__ uint32_t s_base[kRadixBins];  // positions < n < 2^31
-  __shared__ int32_t s_wcnt[kRadixThreads / 32][kRadixBins];
+  constexpr int kWarps = kRadixThreads / 32;
+  __shared__ int32_t s_cnt[kWarps][kRadixBins];  // counts, then positions (< n < 2^31)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int i = tid; i < kRadixBins; i += kRadixThreads)
-    s_base[i] = static_cast<uint32_t>(offsets[static_cast<int64_t>(i) * nblk + blockIdx.x]);
-  for (int i = tid; i < (kRadixThreads / 32) * kRadixBins; i += kRadixThreads)
-    (&s_wcnt[0][0])[i] = 0;
-  __syncthreads();
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kRadixChunk;
+  for (int i = tid; i < kWarps * kRadixBins; i += kRadixThreads) (&s_cnt[0][0])[i] = 0;
+  const int64_t w0 = static_cast<int64_t>(blockIdx.x) * kRadixChunk + warp * (kRadixRounds * 32);
   const uint32_t lt = (1u << lane) - 1u;
   uint32_t keys[kRadixRounds];
-  int32_t vals[kRadixRounds];
+  int32_t vals[kRadixRounds], rank[kRadixRounds];
 #pragma unroll
   for (int round = 0; round < kRadixRounds; ++round) {
-    const int64_t j = c0 + static_cast<int64_t>(round) * kRadixThreads + tid;
+    const int64_t j = w0 + round * 32 + lane;
     keys[round] = j < n ? keys_in[j] : 0u;
     vals[round] = j < n ? (vals_in ? vals_in[j] : static_cast<int32_t>(j)) : 0;
   }
+  __syncthreads();
+  int32_t* my = s_cnt[warp];
 #pragma unroll
   for (int round = 0; round < kRadixRounds; ++round) {
-    const int64_t j = c0 + static_cast<int64_t>(round) * kRadixThreads + tid;
-    const bool valid = j < n;
-    const uint32_t key = keys[round];
-    const int32_t val = vals[round];
-    const uint32_t digit = (key >> shift) & (kRadixBins - 1);
+    const bool valid = w0 + round * 32 + lane < n;
+    const uint32_t digit = (keys[round] >> shift) & (kRadixBins - 1);
     const uint32_t peers = __match_any_sync(0xffffffffu, valid ? digit : 0xFFFFFFFFu);
-    const bool leader = valid && (__ffs(peers) - 1) == lane;
-    if (leader) s_wcnt[warp][digit] = __popc(peers);
-    __syncthreads();
+    const int32_t before = valid ? my[digit] : 0;
+    rank[round] = before + __popc(peers & lt);
+    __syncwarp();
+    if (valid && (__ffs(peers) - 1) == lane) my[digit] = before + __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  for (int d = tid; d < kRadixBins; d += kRadixThreads) {
+    int64_t run = offsets[static_cast<int64_t>(d) * nblk + blockIdx.x];
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const int32_t c = s_cnt[w][d];
+      s_cnt[w][d] = static_cast<int32_t>(run);
+      run += c;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int round = 0; round < kRadixRounds; ++round) {
+    const bool valid = w0 + round * 32 + lane < n;
+    const uint32_t key = keys[round];
+    const uint32_t digit = (key >> shift) & (kRadixBins - 1);
     long long pos = -1;
     if (valid) {
-      int32_t r = __popc(peers & lt);
-      for (int w = 0; w < warp; ++w) r += s_wcnt[w][digit];
-      pos = static_cast<long long>(s_base[digit]) + r;
-      if (pos >= n) {  // only after a scan gave up on a wait
+      pos = static_cast<long long>(my[digit]) + rank[round];
+      if (pos < 0 || pos >= n) {  // only after a scan gave up on a wait
         atomicOr(err, kErrTimeout);
         pos = -1;
       }
     }
     if (pos >= 0) {
       if (!kLast) keys_out[pos] = key;
-      vals_out[pos] = val;
+      vals_out[pos] = vals[round];
     }
     if (!kLast) {
       // next digit, counted per destination chunk: one atomic per distinct (digit, chunk) of the warp
@@ -546,12 +561,6 @@ __global__ void __launch_bounds__(kRadixThreads) k_radix_scatter(
         atomicOr(&tile_mask[tile], hm);
       }
     }
-    __syncthreads();
-    if (leader) {
-      atomicAdd(&s_base[digit], static_cast<uint32_t>(__popc(peers)));
-      s_wcnt[warp][digit] = 0;
-    }
-    __syncwarp();
   }
 }
 
