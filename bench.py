@@ -175,6 +175,34 @@ def pair_flops(p: int, cin: int, cout: int) -> float:
 
 
 # ------------------------------------------------------------- GPU arm
+def conv_variant_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, w_d, b_d, out_d, reps=5):
+    """Median device time (ms) of one conv with each tensor-core variant on
+    the bench's map, L2 flushed before each: the fused 27-tap kernel (the
+    step's), and the per-offset gather-GEMM-scatter over the pair lists, the
+    comparator the pages measure against.  Untimed for the bench value."""
+    m = smc.build_map(coords_d, w.grid, batch=batch, stream=stream)
+    res = {}
+    try:
+        for name, v in (("fused", 1), ("per_offset", 3)):
+            smc.set_conv_variant(v)
+            ts = []
+            for _ in range(reps + 1):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                smc.conv(m, feats_d, w_d, b_d, ksize=3, orientation=1, out=out_d, stream=stream)
+                e1.record(stream)
+                e1.synchronize()
+                ts.append(e0.elapsed_time(e1))
+            res[name] = round(float(np.median(ts[1:])), 4)
+    finally:
+        smc.set_conv_variant(0)
+        m.free()
+    smc.status(stream)
+    res["fused_speedup"] = round(res["per_offset"] / res["fused"], 2)
+    return res
+
+
 def run_gpu(args):
     import torch
 
@@ -282,6 +310,7 @@ def run_gpu(args):
     prof.drain()
     smc.set_profiling(False)
     map_times = prof.map_times
+    variants = conv_variant_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, w_d, b_d, out_d)
 
     total_ms = reduce_max(sum(times), world, dev)
     conv_ms = reduce_max(sum(conv_times) / len(conv_times), world, dev)
@@ -333,6 +362,7 @@ def run_gpu(args):
                                   for q, v in (("p50", 0.5), ("p90", 0.9), ("p99", 0.99), ("max", 1.0))},
             "conv_mvoxels_per_s": round(w.n / (conv_ms * 1e-3) / 1e6, 2),
             "conv_tap_efficiency": round(eff, 4),
+            "conv_variants_ms": variants,
             "roofline": {"kernel": "k_conv_tc", "bound": "tensor", "achieved": round(conv_tflops, 2),
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": round(conv_tflops / peaks["bf16_tflops"], 4), "traffic": traffic,

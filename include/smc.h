@@ -202,11 +202,15 @@ SMC_API const char* smc_strerror(int code);
  *   sites.  Maps are identical either way.  A forced hash capacity
  *   (smc_set_hash_capacity) always selects the hash table.  SMC_E_ARG for
  *   any other value.
- * smc_set_conv_variant: tensor-core conv kernel for later convs: 0 = default
- *   (currently the same as 1), 1 = one CTA per 128-row tile, 2 = CTA pairs (a
- *   cluster of two CTAs sharing M = 256 tcgen05 MMAs, each loading half of
- *   the weight block; slower on B200, where such clusters run one per TPC).
- *   Results are identical; used to test and measure both kernels.
+ * smc_set_conv_variant: tensor-core conv kernel for later convs (bf16/fp16
+ *   shapes the tensor cores take; others always use the FMA kernel): 0 =
+ *   default (currently the same as 1), 1 = fused 27-tap gather-GEMM, one CTA
+ *   per 128-row tile, 2 = the same with CTA pairs (a cluster of two CTAs
+ *   sharing M = 256 tcgen05 MMAs, each loading half of the weight block;
+ *   slower on B200, where such clusters run one per TPC), 3 = per-offset
+ *   gather-GEMM-scatter over the pair lists with fp32 atomic accumulation
+ *   (k = 3 only; waits for the whole build; results equal to rounding).
+ *   1 and 2 give identical bits.  Used to test and measure the variants.
  *   SMC_E_ARG for any other value.
  */
 /*

@@ -303,7 +303,8 @@ def status(stream=None) -> None:
 
 
 def set_conv_variant(variant: int) -> None:
-    """Tensor-core conv kernel: 0 by shape, 1 one CTA per tile, 2 CTA pairs."""
+    """Tensor-core conv: 0 default, 1 fused (one CTA per tile), 2 fused with CTA
+    pairs, 3 per-offset gather-GEMM-scatter."""
     _check(lib().smc_set_conv_variant(int(variant)), "smc_set_conv_variant")
 
 

@@ -35,6 +35,7 @@ struct smc_map {
   int32_t* out_idx;
   int32_t* perm;
   uint32_t* tile_mask;
+  int64_t* pair_offsets;  // device copy of the 28 pair-list offsets
   void* keep;           // one allocation holding nbr, pairs, schedule and tile masks
   mutable void* tmp;    // the build's scratch, released at the first wait on the map
   cudaEvent_t done;     // recorded after the status block is copied back
@@ -322,6 +323,7 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   const size_t o_out = keep.take<int32_t>(pair_cap);
   const size_t o_perm = keep.take<int32_t>(n);
   const size_t o_tmask = keep.take<uint32_t>((n + smc::kTileRows - 1) / smc::kTileRows);
+  const size_t o_poff = keep.take<int64_t>(28);
   Carve tmp;
   const size_t table_bytes = dense ? static_cast<size_t>(sites) * sizeof(int32_t)
                                    : (wide ? 2 : 1) * static_cast<size_t>(cap) * sizeof(unsigned long long);
@@ -366,6 +368,7 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   m->out_idx = reinterpret_cast<int32_t*>(K + o_out);
   m->perm = reinterpret_cast<int32_t*>(K + o_perm);
   m->tile_mask = reinterpret_cast<uint32_t*>(K + o_tmask);
+  m->pair_offsets = reinterpret_cast<int64_t*>(K + o_poff);
 
   if (g_profiling.load() != 0)
     for (auto& e : m->prof) e = take_event(m->device, true);
@@ -423,6 +426,8 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   if (ce == cudaSuccess) ce = cudaEventRecord(ev_fork, s);
   if (ce == cudaSuccess) ce = cudaStreamWaitEvent(side, ev_fork, 0);
   if (ce == cudaSuccess) ce = smc::launch_pair_lists(a, side);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpyAsync(m->pair_offsets, a.info, 28 * sizeof(int64_t), cudaMemcpyDeviceToDevice, side);
   if (ce == cudaSuccess && m->prof[3]) ce = cudaEventRecord(m->prof[3], side);
   if (ce == cudaSuccess) ce = smc::launch_schedule(b, s);
   if (ce == cudaSuccess && m->prof[2]) ce = cudaEventRecord(m->prof[2], s);
@@ -486,7 +491,7 @@ int smc_set_map_lookup(int32_t mode) {
 }
 
 int smc_set_conv_variant(int32_t variant) {
-  if (variant < 0 || variant > 2) return SMC_E_ARG;
+  if (variant < 0 || variant > 3) return SMC_E_ARG;
   smc::set_conv_variant(variant);
   return SMC_OK;
 }
@@ -572,11 +577,30 @@ int smc_conv(const smc_map* map, const void* feats, int64_t cin, const void* wei
   a.err = st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dev != map->device) return SMC_E_ARG;
-  if (s != map->stream && map->done && cudaStreamWaitEvent(s, map->done, 0) != cudaSuccess) {
+  a.in_idx = map->in_idx;
+  a.out_idx = map->out_idx;
+  a.pair_offsets = map->pair_offsets;
+  const bool tc = smc::conv_tc_supported(a);
+  const bool per_offset = tc && taps == 27 && smc::conv_variant() == 3;
+  // The per-offset kernel reads the pair lists, which are built on the side
+  // stream: it waits for the whole build even on the build stream.
+  if ((s != map->stream || per_offset) && map->done && cudaStreamWaitEvent(s, map->done, 0) != cudaSuccess) {
     cudaGetLastError();
     return SMC_E_CUDA;
   }
-  const cudaError_t e = smc::conv_tc_supported(a) ? smc::launch_conv_tc(a, s) : smc::launch_conv_simt(a, s);
+  cudaError_t e;
+  if (per_offset) {
+    void* acc = nullptr;
+    cudaMemPool_t pool = device_pool(dev);
+    if (!pool || cudaMallocFromPoolAsync(&acc, static_cast<size_t>(n) * cout * sizeof(float), pool, s) != cudaSuccess) {
+      cudaGetLastError();
+      return SMC_E_OOM;
+    }
+    e = smc::launch_conv_offsets(a, static_cast<float*>(acc), s);
+    cudaFreeAsync(acc, s);
+  } else {
+    e = tc ? smc::launch_conv_tc(a, s) : smc::launch_conv_simt(a, s);
+  }
   if (e != cudaSuccess) {
     cudaGetLastError();
     return SMC_E_CUDA;

@@ -372,6 +372,7 @@ static TcShape choose_shape(int cin, int cout, int64_t ntiles) {
 }
 
 void set_conv_variant(int v) { g_conv_variant.store(v); }
+int conv_variant() { return g_conv_variant.load(); }
 
 cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s) {
   if (a.n == 0) return cudaSuccess;

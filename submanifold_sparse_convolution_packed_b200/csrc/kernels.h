@@ -78,6 +78,9 @@ struct ConvArgs {
   const int32_t* nbr;   // [n, 27] (taps == 27)
   const int32_t* perm;  // [n] tile order (tensor-core kernel, taps == 27) or null
   const uint32_t* tile_mask;  // [ceil(n/128)] taps present in each tile (taps == 27)
+  const int32_t* in_idx;      // pair lists (per-offset kernel)
+  const int32_t* out_idx;
+  const int64_t* pair_offsets;  // [28] device copy of the list offsets
   int64_t n;
   int cin, cout, taps, orientation, dtype;
   uint32_t* err;
@@ -95,8 +98,13 @@ cudaError_t launch_conv_simt(const ConvArgs& a, cudaStream_t s);
 // tcgen05 kernel: bf16/fp16, cin % 16 == 0 and cin >= 64, cout % 16 == 0, 16-byte aligned.
 bool conv_tc_supported(const ConvArgs& a);
 cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s);
-// Tensor-core kernel variant: 0 = by shape, 1 = one CTA per tile, 2 = CTA pairs.
+// Conv kernel variant: 0 = default, 1 = one CTA per tile, 2 = CTA pairs,
+// 3 = per-offset gather-GEMM-scatter.
 void set_conv_variant(int v);
+int conv_variant();
+// Per-offset gather-GEMM-scatter over the map's pair lists (bf16/fp16 on the
+// tensor-core shapes, k = 3); acc is [n, cout] fp32 scratch.
+cudaError_t launch_conv_offsets(const ConvArgs& a, float* acc, cudaStream_t s);
 
 
 }  // namespace smc

@@ -144,7 +144,7 @@ __device__ __forceinline__ uint32_t key_hits(uint32_t k) {
 
 template <int kKind>
 __global__ void __launch_bounds__(kMapBlock) k_neighbours(
-    const int4* __restrict__ coords, int64_t n, int32_t Z, int32_t Y, int32_t X,
+    const int4* __restrict__ coords, int64_t n, int32_t batch, int32_t Z, int32_t Y, int32_t X,
     const unsigned long long* __restrict__ table, int lg, int32_t* __restrict__ nbr,
     uint32_t* __restrict__ gkey, int32_t* __restrict__ block_counts, int nblocks,
     int32_t* __restrict__ hist1, int radix_nblk) {
@@ -155,8 +155,15 @@ __global__ void __launch_bounds__(kMapBlock) k_neighbours(
   const int64_t base = static_cast<int64_t>(blockIdx.x) * kMapBlock;
   const int64_t v = base + tid;
   uint32_t hits = 0, gk = 0;
-  if (v < n) {
-    const int4 c = coords[v];
+  const int4 c = v < n ? coords[v] : make_int4(-1, 0, 0, 0);
+  if (v < n && !site_ok(c, batch, Z, Y, X)) {
+    // a row outside the box (the build reports SMC_E_RANGE) has no
+    // neighbours, so every map entry stays -1 or a valid row
+#pragma unroll
+    for (int d = 0; d < kTaps; ++d) s_nbr[tid * kTaps + d] = -1;
+    gk = group_key(0u);
+    gkey[v] = gk;
+  } else if (v < n) {
     const uint64_t key = site_key(c, Z, Y, X);
     const int64_t sz = static_cast<int64_t>(Y) * X;
     if (kKind == kMapDense) {
@@ -590,8 +597,8 @@ cudaError_t launch_map_lookups(const MapBuildArgs& a, cudaStream_t s) {
     constexpr int K = decltype(kind)::value;
     k_insert<K><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.batch, a.Z, a.Y, a.X,
                                          a.table, a.lg, a.err, a.zero, a.nzero);
-    k_neighbours<K><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.Z, a.Y, a.X, a.table,
-                                             a.lg, a.nbr, a.gkey, a.block_counts, nb, a.hist1, rnb);
+    k_neighbours<K><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.batch, a.Z, a.Y, a.X,
+                                             a.table, a.lg, a.nbr, a.gkey, a.block_counts, nb, a.hist1, rnb);
   };
   if (a.kind == kMapDense) run(std::integral_constant<int, kMapDense>());
   else if (a.kind == kMapWide) run(std::integral_constant<int, kMapWide>());
@@ -622,7 +629,7 @@ cudaError_t launch_neighbour_map_only(const int32_t* coords, int64_t n, int32_t 
   const int grid_ins = static_cast<int>((n + 255) / 256);
   k_insert<kMapPacked><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(coords), n, batch, Z, Y, X, table,
                                                 lg, err, nullptr, 0);
-  k_neighbours<kMapPacked><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(coords), n, Z, Y, X, table, lg, nbr,
+  k_neighbours<kMapPacked><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(coords), n, batch, Z, Y, X, table, lg, nbr,
                                                gkey, block_counts, nb, nullptr, 0);
   count_launches(2);
   return cudaGetLastError();

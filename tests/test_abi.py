@@ -35,7 +35,7 @@ def test_strerror_without_gpu():
     assert lib.smc_strerror(-3) == b"duplicate coordinate"
     assert lib.smc_set_hash_capacity(-1) == -1
     assert lib.smc_set_hash_capacity(0) == 0
-    assert lib.smc_set_conv_variant(3) == -1
+    assert lib.smc_set_conv_variant(4) == -1
     assert lib.smc_set_conv_variant(-1) == -1
     assert lib.smc_set_conv_variant(0) == 0
     assert lib.smc_set_map_lookup(3) == -1

@@ -63,10 +63,11 @@ def check_close(got, ref, dtype, what=""):
     assert err <= TOL[dtype] * scale, f"{what}: max err {err:.3e} vs bound {TOL[dtype] * scale:.3e}"
 
 
-@pytest.fixture(params=[1, 2], ids=["one_cta", "cta_pair"])
+@pytest.fixture(params=[1, 2, 3], ids=["one_cta", "cta_pair", "per_offset"])
 def conv_variant(request):
-    """Runs a test on both tensor-core kernels: one CTA per 128-row tile, and
-    CTA pairs sharing M = 256 MMAs."""
+    """Runs a test on each tensor-core conv: the fused 27-tap kernel with one
+    CTA per 128-row tile, the same with CTA pairs sharing M = 256 MMAs, and the
+    per-offset gather-GEMM-scatter over the pair lists."""
     smc.set_conv_variant(request.param)
     yield request.param
     smc.set_conv_variant(0)
@@ -406,6 +407,28 @@ def test_pipelined_builds_reuse_memory():
     free0 = run(12)
     free1 = run(60)
     assert free0 - free1 < 64 << 20, f"device memory grew by {(free0 - free1) >> 20} MiB over 60 builds"
+    smc.status()
+
+
+def test_failed_build_map_is_memory_safe(map_lookup):
+    """Rows outside the box (SMC_E_RANGE) or repeated (SMC_E_DUPLICATE) still
+    leave a map whose every entry is -1 or a valid row, and a schedule that is
+    a permutation: a conv enqueued before the error is known stays in bounds."""
+    rng = np.random.default_rng(7)
+    good = np.unique(rng.integers(0, 8, size=(300, 3)), axis=0)
+    coords = np.concatenate([np.zeros((len(good), 1), np.int64), good], axis=1).astype(np.int32)
+    bad = np.array([[1, 0, 0, 0], [0, 8, 0, 0], [0, 0, -1, 3], [0, 3, 3, 9], [-1, 2, 2, 2]], np.int32)
+    for extra, name in ((bad, "SMC_E_RANGE"), (coords[:3], "SMC_E_DUPLICATE")):
+        allc = np.concatenate([coords, extra])
+        m = smc.build_map(torch.from_numpy(allc).cuda(), (8, 8, 8), batch=1, sync=False)
+        nbr = m.nbr().cpu().numpy()
+        perm = m.schedule().cpu().numpy()
+        with pytest.raises(smc.SmcError) as e:
+            m.wait()
+        assert e.value.name == name
+        assert ((nbr >= -1) & (nbr < len(allc))).all()
+        assert np.array_equal(np.sort(perm), np.arange(len(allc)))
+        m.free()
     smc.status()
 
 
