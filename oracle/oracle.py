@@ -10,6 +10,7 @@ Functions
 neighbour_map(coords, grid, k=3)          -> int32 [N, k^3]
 pair_lists(nbr)                           -> (counts int64[T], offsets int64[T+1], in_idx, out_idx)
 conv(coords, grid, feats, weight, bias, k=3, orientation=+1, rows=None, threads=1) -> fp64 [rows, Cout]
+subdivide(coords, keep=None)              -> int32 [M, 4] children, (parent row, octant) order
 
 The definition each follows is cited in smc_oracle.cpp.
 """
@@ -131,3 +132,23 @@ def conv(coords, grid, feats, weight, bias=None, k: int = 3, orientation: int = 
     if rc:
         raise OracleError(rc)
     return out
+
+
+def subdivide(coords, keep=None) -> np.ndarray:
+    """Children of every voxel, the decoders' x2 upsampling: voxel (b, z, y, x)
+    splits into (b, 2z+a, 2y+c, 2x+e) for a, c, e in {0, 1}, octant
+    o = 4a + 2c + e in C order (LATO.2 MLX port README, "The scope, once
+    measured" table; shared sparse-core commit log).  `keep` [N, 8] (nonzero =
+    keep) prunes children; the result lists the kept children parent by
+    parent, octants ascending.  Plain definition, one loop per octant."""
+    c = _coords(coords).astype(np.int64)
+    n = c.shape[0]
+    kept = np.ones((n, 8), dtype=bool) if keep is None else (np.asarray(keep).reshape(n, 8) != 0)
+    children = np.empty((n, 8, 4), dtype=np.int64)
+    for o in range(8):
+        a, cc, e = o >> 2, (o >> 1) & 1, o & 1
+        children[:, o, 0] = c[:, 0]
+        children[:, o, 1] = 2 * c[:, 1] + a
+        children[:, o, 2] = 2 * c[:, 2] + cc
+        children[:, o, 3] = 2 * c[:, 3] + e
+    return children[kept].astype(np.int32)

@@ -15,7 +15,9 @@ one of them:
 * closed forms: identity centre tap, single-tap translation, k=1 linear layer,
   full-box hit counts (Z-|dz|)(Y-|dy|)(X-|dx|);
 * invariants: centre tap is the identity map, neighbour symmetry, batch
-  isolation, linearity, brute-force all-pairs neighbour search.
+  isolation, linearity, brute-force all-pairs neighbour search;
+* subdivision: a hand-listed voxel, a full box that must become the full
+  doubled box, and parent/octant recovery from each child.
 
 Grids are deliberately non-cubic and channel counts unequal so that an axis
 swap or an operand transposition cannot cancel out.
@@ -309,3 +311,36 @@ def test_empty_input(oracle_mod):
     assert counts.sum() == 0 and in_idx.size == 0
     out = oracle_mod.conv(coords, (3, 3, 3), np.zeros((0, 2)), np.zeros((3, 3, 3, 3, 2)), None)
     assert out.shape == (0, 3)
+
+
+# ------------------------------------------------------------------ subdivision
+def test_golden_subdivide_one_voxel(oracle_mod):
+    g = _golden("subdivide_one_voxel.json")
+    coords = np.array(g["coords"], np.int32)
+    assert oracle_mod.subdivide(coords).tolist() == g["expected_children"]
+    assert oracle_mod.subdivide(coords, np.array(g["keep"], np.uint8)).tolist() == g["expected_kept"]
+
+
+def test_subdivide_full_box_is_full_doubled_box(oracle_mod):
+    """Subdividing every site of a 2 x (2, 3, 4) box gives every site of the
+    2 x (4, 6, 8) box exactly once."""
+    box = np.array([(b, z, y, x) for b in range(2) for z in range(2) for y in range(3) for x in range(4)], np.int32)
+    kids = oracle_mod.subdivide(box)
+    full = {(b, z, y, x) for b in range(2) for z in range(4) for y in range(6) for x in range(8)}
+    assert len(kids) == 8 * len(box) == len(full)
+    assert {tuple(r) for r in kids.tolist()} == full
+
+
+def test_subdivide_parent_and_octant_recovery(oracle_mod):
+    """Each child halves back to its parent; its low bits are its octant, in
+    C order, and a keep mask drops exactly the masked children."""
+    rng = np.random.default_rng(3)
+    coords = np.unique(rng.integers(0, 9, size=(60, 4)), axis=0).astype(np.int32)
+    keep = (rng.random((len(coords), 8)) < 0.6).astype(np.uint8)
+    kids = oracle_mod.subdivide(coords, keep)
+    parents = np.repeat(np.arange(len(coords)), 8).reshape(-1, 8)[keep != 0]
+    octs = np.tile(np.arange(8), (len(coords), 1))[keep != 0]
+    assert len(kids) == int(keep.sum())
+    np.testing.assert_array_equal(kids[:, 0], coords[parents, 0])
+    np.testing.assert_array_equal(kids[:, 1:] // 2, coords[parents, 1:])
+    np.testing.assert_array_equal(4 * (kids[:, 1] % 2) + 2 * (kids[:, 2] % 2) + kids[:, 3] % 2, octs)
