@@ -203,6 +203,42 @@ def conv_variant_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, w
     return res
 
 
+def subdivide_times(smc, torch, stream, flush, reps=5):
+    """Median device time (ms) of one decoder step's map, stage 2 -> 3 of the
+    decoder chain (children inside the next shell kept): built from the parent
+    map by smc_subdivide (including its host read of the child count), and
+    built from scratch from the same child coordinates.  The maps are equal
+    (tested); untimed for the bench value."""
+    w2, w3 = S.workload("decoder2"), S.workload("decoder3")
+    keep = torch.from_numpy(S.subdivision_keep_mask(w2.coords, w3.coords, w3.grid)).cuda()
+    pc = torch.from_numpy(w2.coords).cuda()
+    parent = smc.build_map(pc, w2.grid, batch=1, stream=stream)
+    inc, full = [], []
+    for _ in range(reps + 1):
+        flush.zero_()
+        e0, e1, e2, e3 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
+        e0.record(stream)
+        kids, child = smc.subdivide(parent, pc, keep, stream=stream)
+        child.stream_wait(stream)
+        e1.record(stream)
+        flush.zero_()
+        e2.record(stream)
+        again = smc.build_map(kids, child.grid, batch=1, stream=stream, sync=False)
+        again.stream_wait(stream)
+        e3.record(stream)
+        e3.synchronize()
+        child.wait()
+        again.wait()
+        inc.append(e0.elapsed_time(e1))
+        full.append(e2.elapsed_time(e3))
+        child.free()
+        again.free()
+    parent.free()
+    smc.status(stream)
+    return {"workload": f"decoder stage 2 -> 3: {w2.n} voxels on {w2.grid[0]}^3 -> {int(keep.sum())} on {w3.grid[0]}^3",
+            "incremental": round(float(np.median(inc[1:])), 4), "full_build": round(float(np.median(full[1:])), 4)}
+
+
 def run_gpu(args):
     import torch
 
@@ -311,6 +347,7 @@ def run_gpu(args):
     smc.set_profiling(False)
     map_times = prof.map_times
     variants = conv_variant_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, w_d, b_d, out_d)
+    subdiv = subdivide_times(smc, torch, stream, flush)
 
     total_ms = reduce_max(sum(times), world, dev)
     conv_ms = reduce_max(sum(conv_times) / len(conv_times), world, dev)
@@ -363,6 +400,7 @@ def run_gpu(args):
             "conv_mvoxels_per_s": round(w.n / (conv_ms * 1e-3) / 1e6, 2),
             "conv_tap_efficiency": round(eff, 4),
             "conv_variants_ms": variants,
+            "subdivide_map_ms": subdiv,
             "roofline": {"kernel": "k_conv_tc", "bound": "tensor", "achieved": round(conv_tflops, 2),
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": round(conv_tflops / peaks["bf16_tflops"], 4), "traffic": traffic,

@@ -113,6 +113,33 @@ SMC_API int smc_build_map_async(const int32_t* coords, int64_t n, int32_t batch,
 /* Block until the map's build has finished; return its outcome. */
 SMC_API int smc_map_wait(const smc_map* map);
 
+/*
+ * smc_subdivide -- the map of a parent map's children, built from the parent
+ * map without any lookup structure (the decoders' x2 upsampling step: every
+ * voxel splits into its 8 children in C order; LATO.2 MLX port README, "The
+ * scope, once measured" table, and the shared sparse-core commit log).
+ *
+ * parent        : a built map; the call waits for its build and returns its
+ *                 error if it failed.
+ * parent_coords : device int32 [n, 4], the coordinates the parent was built
+ *                 from (same rows), 16-byte aligned.
+ * keep          : device uint8 [n * 8] or NULL (keep all): keep[8v + o] != 0
+ *                 keeps child o = 4a + 2c + e of parent v, the site
+ *                 (b, 2z + a, 2y + c, 2x + e).
+ * child_coords  : device int32 [8n, 4] capacity, 16-byte aligned; receives
+ *                 the m kept children in (parent row, octant) order.
+ * m             : host, receives m.
+ * child         : receives the children's map on the grid (2Z, 2Y, 2X), the
+ *                 same batch; as a smc_build_map_async result (pair lists on
+ *                 the side stream, errors at smc_map_wait).
+ * One host synchronisation of `stream` (to read m).  A child's neighbour at
+ * offset D is the kept child, in octant (o + D) mod 2, of the parent's
+ * neighbour at offset floor((o + D) / 2).  Errors: SMC_E_ARG, SMC_E_ALIGN,
+ * SMC_E_OOM, SMC_E_CUDA, SMC_E_TIMEOUT, or the parent's build error.
+ */
+SMC_API int smc_subdivide(const smc_map* parent, const int32_t* parent_coords, const uint8_t* keep,
+                  int32_t* child_coords, int64_t* m, void* stream, smc_map** child);
+
 /* Make `stream` wait (on the device, without blocking the host) until the
  * whole build has finished, pair lists included: work enqueued on `stream`
  * afterwards may read every part of the map. */

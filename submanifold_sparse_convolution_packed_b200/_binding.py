@@ -30,7 +30,7 @@ EXPORTS = [
     "smc_map_schedule", "smc_free_map", "smc_status", "smc_strerror",
     "smc_set_hash_capacity", "smc_set_profiling", "smc_map_timing", "smc_kernel_launches",
     "smc_build_map_async", "smc_map_wait", "smc_neighbour_map_noalloc", "smc_set_conv_variant",
-    "smc_set_map_lookup", "smc_map_stream_wait",
+    "smc_set_map_lookup", "smc_map_stream_wait", "smc_subdivide",
 ]
 
 
@@ -59,6 +59,7 @@ def lib() -> ctypes.CDLL:
         L.smc_build_map_async.argtypes = [P, i64, i32, P, P, ctypes.POINTER(P)]
         L.smc_map_wait.argtypes = [P]
         L.smc_map_stream_wait.argtypes = [P, P]
+        L.smc_subdivide.argtypes = [P, P, P, P, P, P, P]
         L.smc_neighbour_map_noalloc.argtypes = [P, i64, i32, P, P, P]
         L.smc_conv.argtypes = [P, P, i64, P, P, P, i64, i32, i32, i32, P]
         L.smc_map_info.argtypes = [P, P, P]
@@ -232,6 +233,29 @@ def build_map(coords: torch.Tensor, grid: Sequence[int], batch: Optional[int] = 
     if key is not None:
         _cache[key] = m
     return m
+
+
+def subdivide(parent: "Map", parent_coords: torch.Tensor, keep: Optional[torch.Tensor] = None, stream=None):
+    """Children of every voxel of `parent` (x2 per axis, 8 per voxel in C
+    order), optionally pruned by a uint8 [N, 8] `keep` mask; returns
+    (child_coords int32 [M, 4], child Map on the doubled grid).  The child map
+    is built from the parent map (smc_subdivide in include/smc.h)."""
+    n = parent.n
+    if parent_coords.dtype != torch.int32 or parent_coords.shape != (n, 4) or not parent_coords.is_cuda:
+        raise ValueError("parent_coords must be the parent's int32 [N, 4] CUDA tensor")
+    parent_coords = parent_coords.contiguous()
+    if keep is not None:
+        if keep.dtype not in (torch.uint8, torch.bool) or keep.numel() != 8 * n or not keep.is_cuda:
+            raise ValueError("keep must be a uint8/bool CUDA tensor of N * 8 entries")
+        keep = keep.contiguous().view(torch.uint8)
+    out = torch.empty((max(8 * n, 1), 4), dtype=torch.int32, device=parent_coords.device)
+    m = ctypes.c_int64()
+    h = ctypes.c_void_p()
+    with torch.cuda.device(parent_coords.device):
+        _check(lib().smc_subdivide(parent.handle, _ptr(parent_coords), _ptr(keep) if keep is not None else None,
+                                   _ptr(out), ctypes.byref(m), _stream(stream), ctypes.byref(h)), "smc_subdivide")
+    grid = tuple(2 * int(g) for g in parent.grid)
+    return out[: m.value], Map(h, int(m.value), parent.batch, grid, parent_coords.device)
 
 
 NOALLOC_MAX_N = 1 << 18

@@ -257,15 +257,23 @@ int resolve(const smc_map* m) {
   return rc;
 }
 
+// Children of a parent map whose rows are read off the parent map
+// (smc_subdivide): replaces the lookup structure and the lookup kernels.
+struct SubdivSource {
+  const int32_t* parent_nbr;
+  const int32_t* child_src;  // [n] 8 * parent row + octant
+  const int32_t* remap;      // [8 * parent n] child row or -1
+};
+
 // Enqueue a whole map build on `s`; no synchronisation.
 int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t grid[3], cudaStream_t s,
-                smc_map** out) {
+                smc_map** out, const SubdivSource* sub = nullptr) {
   if (!out) return SMC_E_ARG;
   *out = nullptr;
-  if (!grid || n < 0 || batch < 1 || (n > 0 && !coords)) return SMC_E_ARG;
+  if (!grid || n < 0 || batch < 1 || (n > 0 && !coords && !sub)) return SMC_E_ARG;
   if (grid[0] < 1 || grid[1] < 1 || grid[2] < 1) return SMC_E_ARG;
   if (n >= (1ll << 31) - 1) return SMC_E_ARG;  // rows are int32
-  if (n > 0 && (reinterpret_cast<uintptr_t>(coords) & 15u)) return SMC_E_ALIGN;
+  if (n > 0 && !sub && (reinterpret_cast<uintptr_t>(coords) & 15u)) return SMC_E_ALIGN;
   const double sites = static_cast<double>(batch) * grid[0] * grid[1] * grid[2];
   if (sites >= 4.6e18) return SMC_E_ARG;
   if (pending_cuda_error() != SMC_OK) return SMC_E_CUDA;
@@ -301,7 +309,7 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   // less than hash probing) and at most 2^28 sites.  Otherwise a hash table.
   const int64_t forced = g_capacity_override.load();
   const int lookup = g_map_lookup.load();
-  const bool dense = forced == 0 && sites <= kDenseMaxSites &&
+  const bool dense = !sub && forced == 0 && sites <= kDenseMaxSites &&
                      (lookup == 2 || (lookup == 0 && sites <= 256.0 * static_cast<double>(n)));
   const bool wide = !dense && sites > 4294967294.0;  // packed slots need keys < 2^32 - 1
   int lg = 4;
@@ -325,8 +333,9 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   const size_t o_tmask = keep.take<uint32_t>((n + smc::kTileRows - 1) / smc::kTileRows);
   const size_t o_poff = keep.take<int64_t>(28);
   Carve tmp;
-  const size_t table_bytes = dense ? static_cast<size_t>(sites) * sizeof(int32_t)
-                                   : (wide ? 2 : 1) * static_cast<size_t>(cap) * sizeof(unsigned long long);
+  const size_t table_bytes = sub     ? 16
+                             : dense ? static_cast<size_t>(sites) * sizeof(int32_t)
+                                     : (wide ? 2 : 1) * static_cast<size_t>(cap) * sizeof(unsigned long long);
   const size_t o_table = tmp.take<uint8_t>(table_bytes);
   const size_t o_gkey = tmp.take<uint32_t>(n);
   const size_t o_bc = tmp.take<int32_t>(Lmap);
@@ -421,7 +430,12 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   cudaError_t ce = cudaMemsetAsync(T + o_table, 0xFF, table_bytes, s);
   if (ce == cudaSuccess) ce = cudaMemsetAsync(T + o_err, 0, zero_bytes, s);
   if (ce == cudaSuccess && m->prof[0]) ce = cudaEventRecord(m->prof[0], s);
-  if (ce == cudaSuccess) ce = smc::launch_map_lookups(a, s);
+  if (ce == cudaSuccess && sub) {
+    ce = cudaMemsetAsync(m->tile_mask, 0, a.nzero * sizeof(uint32_t), s);  // k_insert clears them otherwise
+    if (ce == cudaSuccess) ce = smc::launch_subdiv_lookups(a, sub->parent_nbr, sub->child_src, sub->remap, s);
+  } else if (ce == cudaSuccess) {
+    ce = smc::launch_map_lookups(a, s);
+  }
   if (ce == cudaSuccess && m->prof[1]) ce = cudaEventRecord(m->prof[1], s);
   if (ce == cudaSuccess) ce = cudaEventRecord(ev_fork, s);
   if (ce == cudaSuccess) ce = cudaStreamWaitEvent(side, ev_fork, 0);
@@ -509,6 +523,99 @@ int smc_build_map_async(const int32_t* coords, int64_t n, int32_t batch, const i
 int smc_map_wait(const smc_map* map) {
   if (!map) return SMC_E_ARG;
   return resolve(map);
+}
+
+int smc_subdivide(const smc_map* parent, const int32_t* parent_coords, const uint8_t* keep, int32_t* child_coords,
+                  int64_t* m_out, void* stream, smc_map** child) {
+  if (!child || !m_out) return SMC_E_ARG;
+  *child = nullptr;
+  *m_out = 0;
+  if (!parent) return SMC_E_ARG;
+  const int64_t n = parent->n;
+  if (n > 0 && (!parent_coords || !child_coords)) return SMC_E_ARG;
+  if (n > 0 && ((reinterpret_cast<uintptr_t>(parent_coords) & 15u) || (reinterpret_cast<uintptr_t>(child_coords) & 15u)))
+    return SMC_E_ALIGN;
+  int32_t grid2[3];
+  for (int i = 0; i < 3; ++i) {
+    if (parent->grid[i] > (1 << 30) - 1) return SMC_E_ARG;
+    grid2[i] = 2 * parent->grid[i];
+  }
+  if (8 * n >= (1ll << 31) - 1) return SMC_E_ARG;  // child rows and parent slots are int32
+  const int rc = resolve(parent);  // the parent map must be complete (and sound)
+  if (rc != SMC_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != parent->device) return SMC_E_ARG;
+  if (n == 0) return build_async(nullptr, 0, parent->batch, grid2, s, child);
+  if (pending_cuda_error() != SMC_OK) return SMC_E_CUDA;
+  cudaMemPool_t pool = device_pool(dev);
+  HostSlot* slot = take_slot();
+  if (!pool || !slot) {
+    give_slot(slot);
+    return SMC_E_OOM;
+  }
+  // scratch: error word + ticket, scan statuses, list info, per-parent bits,
+  // counts and first child, the parent-slot -> child-row remap, child sources
+  Carve c;
+  const size_t o_hdr = c.take<HostSlot>(1);
+  const size_t o_tick = c.take<uint32_t>(1);
+  const size_t o_st = c.take<unsigned long long>(smc::scan_status_len(n));
+  const size_t zero_bytes = c.off - o_hdr;
+  const size_t o_bits = c.take<uint8_t>(n);
+  const size_t o_cnt = c.take<int32_t>(n);
+  const size_t o_first = c.take<int64_t>(n);
+  const size_t o_remap = c.take<int32_t>(8 * n);
+  const size_t o_src = c.take<int32_t>(8 * n);
+  void* sp = nullptr;
+  if (cudaMallocFromPoolAsync(&sp, c.off, pool, s) != cudaSuccess) {
+    cudaGetLastError();
+    give_slot(slot);
+    return SMC_E_OOM;
+  }
+  char* S = static_cast<char*>(sp);
+  uint32_t* err = reinterpret_cast<uint32_t*>(S + o_hdr + offsetof(HostSlot, err));
+  int64_t* info = reinterpret_cast<int64_t*>(S + o_hdr + offsetof(HostSlot, info));
+  uint8_t* bits = reinterpret_cast<uint8_t*>(S + o_bits);
+  int32_t* cnt = reinterpret_cast<int32_t*>(S + o_cnt);
+  int64_t* first = reinterpret_cast<int64_t*>(S + o_first);
+  int32_t* remap = reinterpret_cast<int32_t*>(S + o_remap);
+  int32_t* src = reinterpret_cast<int32_t*>(S + o_src);
+  // children per parent, then their first row; the total comes back to size the child map
+  cudaError_t ce = cudaMemsetAsync(S + o_hdr, 0, zero_bytes, s);
+  if (ce == cudaSuccess) ce = smc::launch_subdiv_count(keep, n, bits, cnt, s);
+  if (ce == cudaSuccess)
+    ce = smc::launch_scan_counts(cnt, n, first, reinterpret_cast<unsigned long long*>(S + o_st),
+                                 reinterpret_cast<uint32_t*>(S + o_tick), err, info, n, s);
+  if (ce == cudaSuccess) ce = cudaMemcpyAsync(slot, S + o_hdr, sizeof(HostSlot), cudaMemcpyDeviceToHost, s);
+  if (ce == cudaSuccess) ce = cudaStreamSynchronize(s);
+  const uint32_t scan_err = slot->err;
+  const int64_t m = slot->info[27];
+  give_slot(slot);
+  int out = SMC_OK;
+  if (ce != cudaSuccess) {
+    cudaGetLastError();
+    out = SMC_E_CUDA;
+  } else if (scan_err & smc::kErrTimeout) {
+    out = SMC_E_TIMEOUT;
+  } else if (m < 0 || m > 8 * n) {
+    out = SMC_E_CUDA;
+  }
+  if (out == SMC_OK) {
+    ce = smc::launch_subdiv_emit(parent_coords, n, bits, first, child_coords, src, remap, s);
+    if (ce != cudaSuccess) {
+      cudaGetLastError();
+      out = SMC_E_CUDA;
+    }
+  }
+  if (out == SMC_OK) {
+    const SubdivSource sub{parent->nbr, src, remap};
+    out = build_async(child_coords, m, parent->batch, grid2, s, child, &sub);
+  }
+  cudaFreeAsync(sp, s);  // after the child lookups, which read remap and src, in stream order
+  cudaGetLastError();
+  if (out == SMC_OK) *m_out = m;
+  return out;
 }
 
 int smc_map_stream_wait(const smc_map* map, void* stream) {

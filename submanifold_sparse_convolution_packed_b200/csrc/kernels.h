@@ -66,6 +66,18 @@ cudaError_t launch_neighbour_map_only(const int32_t* coords, int64_t n, int32_t 
                                       int32_t X, unsigned long long* table, int lg, uint32_t* err, int32_t* nbr,
                                       uint32_t* gkey, int32_t* block_counts, cudaStream_t s);
 cudaError_t launch_schedule(const ScheduleArgs& a, cudaStream_t s);
+// Single-pass exclusive scan of int32 counts (k_scan_lookback); status and
+// ticket zeroed, status of scan_status_len(L) words.
+cudaError_t launch_scan_counts(const int32_t* in, int64_t L, int64_t* out, unsigned long long* status,
+                               uint32_t* ticket, uint32_t* err, int64_t* info, int64_t stride, cudaStream_t s);
+// Subdivision: children per parent (bit mask and count), the children's
+// coordinates with their (parent, octant) and the parent-slot -> child-row
+// remap, then the children's map rows from the parent map.
+cudaError_t launch_subdiv_count(const uint8_t* keep, int64_t n, uint8_t* bits, int32_t* cnt, cudaStream_t s);
+cudaError_t launch_subdiv_emit(const int32_t* coords, int64_t n, const uint8_t* bits, const int64_t* first,
+                               int32_t* child_coords, int32_t* child_src, int32_t* remap, cudaStream_t s);
+cudaError_t launch_subdiv_lookups(const MapBuildArgs& a, const int32_t* parent_nbr, const int32_t* child_src,
+                                  const int32_t* remap, cudaStream_t s);
 
 // dtype codes as in smc.h
 enum DType : int { kF32 = 0, kBF16 = 1, kF16 = 2 };

@@ -142,6 +142,43 @@ __device__ __forceinline__ uint32_t key_hits(uint32_t k) {
   return m;
 }
 
+// The end of a 256-row block of a map-building kernel, once each thread's row
+// is in s_nbr and its hit mask and schedule key are known: the first radix
+// digit's histogram (one atomic per distinct digit of a warp), the per-offset
+// hit counts of the block, and the block's map rows stored in 16-byte vectors.
+__device__ __forceinline__ void emit_map_block(const int32_t* s_nbr, int32_t (*s_cnt)[kTaps], uint32_t hits,
+                                               uint32_t gk, int64_t base, int64_t n, int32_t* __restrict__ nbr,
+                                               int32_t* __restrict__ block_counts, int nblocks,
+                                               int32_t* __restrict__ hist1, int radix_nblk) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t v = base + tid;
+  if (hist1) {
+    const uint32_t digit = v < n ? (gk & (kRadixBins - 1)) : 0xFFFFFFFFu;
+    const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+    if (v < n && (__ffs(peers) - 1) == lane)
+      atomicAdd(&hist1[static_cast<int64_t>(digit) * radix_nblk + (base / kRadixChunk)], __popc(peers));
+  }
+#pragma unroll
+  for (int d = 0; d < kTaps; ++d) {
+    const uint32_t b = __ballot_sync(0xffffffffu, (hits >> d) & 1u);
+    if (lane == 0) s_cnt[warp][d] = __popc(b);
+  }
+  __syncthreads();
+  const int64_t rows = n - base < kMapBlock ? n - base : kMapBlock;
+  const int total = static_cast<int>(rows) * kTaps;
+  int32_t* dst = nbr + base * kTaps;  // base*27*4 bytes is a multiple of 16
+  const int vec = total >> 2;
+  for (int i = tid; i < vec; i += kMapBlock)
+    reinterpret_cast<int4*>(dst)[i] = reinterpret_cast<const int4*>(s_nbr)[i];
+  for (int i = (vec << 2) + tid; i < total; i += kMapBlock) dst[i] = s_nbr[i];
+  if (tid < kTaps) {
+    int32_t c = 0;
+#pragma unroll
+    for (int w = 0; w < kMapBlock / 32; ++w) c += s_cnt[w][tid];
+    block_counts[static_cast<int64_t>(tid) * nblocks + blockIdx.x] = c;
+  }
+}
+
 template <int kKind>
 __global__ void __launch_bounds__(kMapBlock) k_neighbours(
     const int4* __restrict__ coords, int64_t n, int32_t batch, int32_t Z, int32_t Y, int32_t X,
@@ -261,32 +298,82 @@ __global__ void __launch_bounds__(kMapBlock) k_neighbours(
     gk = group_key(hits);
     gkey[v] = gk;
   }
-  if (hist1) {
-    // first radix digit: one atomic per distinct digit of the warp
-    const uint32_t digit = v < n ? (gk & (kRadixBins - 1)) : 0xFFFFFFFFu;
-    const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-    if (v < n && (__ffs(peers) - 1) == lane)
-      atomicAdd(&hist1[static_cast<int64_t>(digit) * radix_nblk + (base / kRadixChunk)], __popc(peers));
-  }
+  emit_map_block(s_nbr, s_cnt, hits, gk, base, n, nbr, block_counts, nblocks, hist1, radix_nblk);
+}
+
+// ------------------------------------------------------------ subdivision
+// The children of parent row v are the sites (b, 2z+a, 2y+c, 2x+e) of octant
+// o = 4a + 2c + e (C order), kept where keep[8v+o] is nonzero (all when keep
+// is null) and numbered in (parent row, octant) order.
+__global__ void k_subdiv_count(const uint8_t* __restrict__ keep, int64_t n, uint8_t* __restrict__ bits,
+                               int32_t* __restrict__ cnt) {
+  for (int64_t v = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; v < n;
+       v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    uint32_t b = 0xFFu;
+    if (keep) {
+      b = 0;
 #pragma unroll
-  for (int d = 0; d < kTaps; ++d) {
-    const uint32_t b = __ballot_sync(0xffffffffu, (hits >> d) & 1u);
-    if (lane == 0) s_cnt[warp][d] = __popc(b);
+      for (int o = 0; o < 8; ++o) b |= static_cast<uint32_t>(keep[8 * v + o] != 0) << o;
+    }
+    bits[v] = static_cast<uint8_t>(b);
+    cnt[v] = __popc(b);
   }
-  __syncthreads();
-  const int64_t rows = n - base < kMapBlock ? n - base : kMapBlock;
-  const int total = static_cast<int>(rows) * kTaps;
-  int32_t* dst = nbr + base * kTaps;  // base*27*4 bytes is a multiple of 16
-  const int vec = total >> 2;
-  for (int i = tid; i < vec; i += kMapBlock)
-    reinterpret_cast<int4*>(dst)[i] = reinterpret_cast<const int4*>(s_nbr)[i];
-  for (int i = (vec << 2) + tid; i < total; i += kMapBlock) dst[i] = s_nbr[i];
-  if (tid < kTaps) {
-    int32_t s = 0;
+}
+
+__global__ void k_subdiv_emit(const int4* __restrict__ coords, int64_t n, const uint8_t* __restrict__ bits,
+                              const int64_t* __restrict__ first, int4* __restrict__ child_coords,
+                              int32_t* __restrict__ child_src, int32_t* __restrict__ remap) {
+  for (int64_t v = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; v < n;
+       v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int4 c = coords[v];
+    const uint32_t b = bits[v];
+    int64_t r = first[v];
 #pragma unroll
-    for (int w = 0; w < kMapBlock / 32; ++w) s += s_cnt[w][tid];
-    block_counts[static_cast<int64_t>(tid) * nblocks + blockIdx.x] = s;
+    for (int o = 0; o < 8; ++o) {
+      if ((b >> o) & 1u) {
+        child_coords[r] = make_int4(c.x, 2 * c.y + (o >> 2), 2 * c.z + ((o >> 1) & 1), 2 * c.w + (o & 1));
+        child_src[r] = static_cast<int32_t>(8 * v + o);
+        remap[8 * v + o] = static_cast<int32_t>(r);
+        ++r;
+      } else {
+        remap[8 * v + o] = -1;
+      }
+    }
   }
+}
+
+// Map rows of the children, read off the parent map with no lookup
+// structure: child 2p+o and offset D reach the site 2p+o+D, whose parent is
+// p's neighbour at offset floor((o+D)/2) and whose octant is (o+D) mod 2;
+// that child's row is remap[8*parent + octant] (-1 if it was not kept).
+__global__ void __launch_bounds__(kMapBlock) k_subdiv_neighbours(
+    const int32_t* __restrict__ parent_nbr, const int32_t* __restrict__ child_src,
+    const int32_t* __restrict__ remap, int64_t m, int32_t* __restrict__ nbr, uint32_t* __restrict__ gkey,
+    int32_t* __restrict__ block_counts, int nblocks, int32_t* __restrict__ hist1, int radix_nblk) {
+  __shared__ int32_t s_nbr[kMapBlock * kTaps];
+  __shared__ int32_t s_cnt[kMapBlock / 32][kTaps];
+  const int tid = threadIdx.x;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kMapBlock;
+  const int64_t v = base + tid;
+  uint32_t hits = 0, gk = 0;
+  if (v < m) {
+    const int32_t src = child_src[v];
+    const int64_t p = src >> 3;
+    const int oz = (src >> 2) & 1, oy = (src >> 1) & 1, ox = src & 1;
+    const int32_t* prow = parent_nbr + p * kTaps;
+#pragma unroll
+    for (int d = 0; d < kTaps; ++d) {
+      const int tz = oz + d / 9 - 1, ty = oy + (d / 3) % 3 - 1, tx = ox + d % 3 - 1;  // in -1 .. 2
+      const int pd = 9 * ((tz >> 1) + 1) + 3 * ((ty >> 1) + 1) + ((tx >> 1) + 1);
+      const int32_t q = __ldg(prow + pd);
+      const int32_t r = q < 0 ? -1 : __ldg(remap + 8 * static_cast<int64_t>(q) + 4 * (tz & 1) + 2 * (ty & 1) + (tx & 1));
+      s_nbr[tid * kTaps + d] = r;
+      hits |= static_cast<uint32_t>(r >= 0) << d;
+    }
+    gk = group_key(hits);
+    gkey[v] = gk;
+  }
+  emit_map_block(s_nbr, s_cnt, hits, gk, base, m, nbr, block_counts, nblocks, hist1, radix_nblk);
 }
 
 __global__ void __launch_bounds__(kMapBlock) k_pairs(const int32_t* __restrict__ nbr, int64_t n,
@@ -615,6 +702,41 @@ cudaError_t launch_pair_lists(const MapBuildArgs& a, cudaStream_t s) {
   cudaError_t e = scan_i32(a.block_counts, L, a.block_offsets, a.scan_status, a.scan_ticket, a.err, a.info, nb, s);
   if (e != cudaSuccess) return e;
   k_pairs<<<nb, kMapBlock, 0, s>>>(a.nbr, n, a.block_offsets, nb, a.in_idx, a.out_idx);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scan_counts(const int32_t* in, int64_t L, int64_t* out, unsigned long long* status,
+                               uint32_t* ticket, uint32_t* err, int64_t* info, int64_t stride, cudaStream_t s) {
+  return scan_i32(in, L, out, status, ticket, err, info, stride, s);
+}
+
+cudaError_t launch_subdiv_count(const uint8_t* keep, int64_t n, uint8_t* bits, int32_t* cnt, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  const int64_t blocks = (n + 255) / 256;
+  k_subdiv_count<<<static_cast<unsigned>(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, s>>>(keep, n, bits, cnt);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_subdiv_emit(const int32_t* coords, int64_t n, const uint8_t* bits, const int64_t* first,
+                               int32_t* child_coords, int32_t* child_src, int32_t* remap, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  const int64_t blocks = (n + 255) / 256;
+  k_subdiv_emit<<<static_cast<unsigned>(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, s>>>(
+      reinterpret_cast<const int4*>(coords), n, bits, first, reinterpret_cast<int4*>(child_coords), child_src,
+      remap);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_subdiv_lookups(const MapBuildArgs& a, const int32_t* parent_nbr, const int32_t* child_src,
+                                  const int32_t* remap, cudaStream_t s) {
+  const int64_t n = a.n;
+  if (n == 0) return cudaSuccess;
+  const int nb = map_nblocks(n);
+  k_subdiv_neighbours<<<nb, kMapBlock, 0, s>>>(parent_nbr, child_src, remap, n, a.nbr, a.gkey, a.block_counts, nb,
+                                               a.hist1, radix_nblocks(n));
   count_launches(1);
   return cudaGetLastError();
 }

@@ -30,7 +30,7 @@ import numpy as np
 __all__ = [
     "rng_for", "round_to", "to_bf16_bits", "bf16_bits_to_f32",
     "random_occupancy", "shell_points", "plane_points", "union_of_shells",
-    "full_grid", "varlen_item", "subdivide_shell", "Workload", "workload",
+    "full_grid", "varlen_item", "subdivide_shell", "subdivision_keep_mask", "Workload", "workload",
     "features", "weights", "bias", "WORKLOADS", "small_integer_values",
 ]
 
@@ -163,6 +163,24 @@ def subdivide_shell(zyx: np.ndarray, c: np.ndarray, r: float) -> Tuple[np.ndarra
     kids = kids[np.abs(d - r2) < 1.0]
     order = np.lexsort((kids[:, 2], kids[:, 1], kids[:, 0]))
     return kids[order].astype(np.int32), c2, r2
+
+
+def subdivision_keep_mask(parent_coords: np.ndarray, child_coords: np.ndarray,
+                          child_grid: Tuple[int, int, int]) -> np.ndarray:
+    """uint8 [N, 8]: which of each parent's 8 children (octant o = 4a + 2b + c,
+    the child 2p + (a, b, c)) appear in `child_coords` -- the pruning decision
+    of a decoder step, as input data for a subdivision."""
+    off = np.argwhere(np.ones((2, 2, 2), dtype=bool)).astype(np.int64)  # C order
+    p = parent_coords.astype(np.int64)
+    kids = 2 * p[:, None, 1:] + off[None, :, :]
+    G = np.asarray(child_grid, dtype=np.int64)
+
+    def key(b, zyx):
+        return ((b * G[0] + zyx[..., 0]) * G[1] + zyx[..., 1]) * G[2] + zyx[..., 2]
+
+    c = child_coords.astype(np.int64)
+    have = np.isin(key(p[:, None, 0], kids), key(c[:, 0], c[:, 1:]))
+    return have.astype(np.uint8)
 
 
 # ----------------------------------------------------------------------------

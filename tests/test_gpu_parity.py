@@ -179,6 +179,85 @@ def test_map_errors(map_lookup):
     smc.status()
 
 
+# ------------------------------------------------------------------ subdivision
+def _site_keys(coords, grid):
+    c = coords.astype(np.int64)
+    return ((c[:, 0] * grid[0] + c[:, 1]) * grid[1] + c[:, 2]) * grid[2] + c[:, 3]
+
+
+def _check_child_map(oracle_mod, parent_coords, grid, keep, got_coords, child):
+    ref_coords = oracle_mod.subdivide(parent_coords, keep)
+    np.testing.assert_array_equal(got_coords.cpu().numpy(), ref_coords)
+    grid2 = tuple(2 * g for g in grid)
+    assert child.n == len(ref_coords) and child.grid == grid2
+    ref = oracle_mod.neighbour_map(ref_coords, grid2)  # built from scratch, not from the parent map
+    np.testing.assert_array_equal(child.nbr().cpu().numpy(), ref)
+    counts, offsets, in_idx, out_idx = oracle_mod.pair_lists(ref)
+    assert child.counts == counts.tolist()
+    gi, go, _ = child.pairs()
+    np.testing.assert_array_equal(gi.cpu().numpy(), in_idx)
+    np.testing.assert_array_equal(go.cpu().numpy(), out_idx)
+    np.testing.assert_array_equal(child.schedule().cpu().numpy(), expected_schedule(ref))
+    return ref_coords
+
+
+@pytest.mark.parametrize("mode", ["all", "random", "none_kept"])
+def test_subdivide_matches_oracle(oracle_mod, mode):
+    """Children of the two-item shell workload, all kept, half kept at random,
+    or none: coordinates, map, pair lists and schedule bit-exact against the
+    oracle's subdivision and a map the oracle builds from scratch."""
+    w = workload("shell2")
+    parent = build(w)
+    pc = torch.from_numpy(w.coords).cuda()
+    keep = None
+    if mode == "random":
+        keep = (np.random.default_rng(5).random((w.n, 8)) < 0.5).astype(np.uint8)
+    elif mode == "none_kept":
+        keep = np.zeros((w.n, 8), np.uint8)
+    kids, child = smc.subdivide(parent, pc, None if keep is None else torch.from_numpy(keep).cuda())
+    if mode == "none_kept":
+        assert child.n == 0 and kids.shape == (0, 4)
+        return
+    _check_child_map(oracle_mod, w.coords, w.grid, keep, kids, child)
+    smc.status()
+
+
+def test_subdivide_decoder_chain(oracle_mod):
+    """One decoder step: stage-1 voxels split and the children inside the
+    stage-2 shell are kept; the child set is stage 2, its map is exact, and a
+    conv over it meets the bf16 bar against the oracle."""
+    w1, w2 = workload("decoder1"), workload("decoder2")
+    kids_all = oracle_mod.subdivide(w1.coords)
+    keep = np.isin(_site_keys(kids_all, w2.grid), _site_keys(w2.coords, w2.grid)).reshape(w1.n, 8).astype(np.uint8)
+    parent = build(w1)
+    kids, child = smc.subdivide(parent, torch.from_numpy(w1.coords).cuda(), torch.from_numpy(keep).cuda())
+    ref_coords = _check_child_map(oracle_mod, w1.coords, w1.grid, keep, kids, child)
+    assert set(_site_keys(ref_coords, w2.grid).tolist()) == set(_site_keys(w2.coords, w2.grid).tolist())
+    sub = S.Workload("decoder2_from_subdivide", ref_coords, w2.grid, w2.cin, w2.cout, ("bf16",))
+    f, wt, b = _layer(sub, "bf16")
+    rows = sample_rows(sub.n, 2048, 9)
+    out = smc.conv(child, dev(f, "bf16"), dev(wt, "bf16"), dev(b, "bf16"))
+    ref = oracle_mod.conv(ref_coords, w2.grid, f, wt, b, 3, 1, rows=rows, threads=THREADS)
+    check_close(host(out)[rows], ref, "bf16", "conv on the subdivided map")
+    smc.status()
+
+
+def test_subdivide_errors():
+    w = workload("tiny")
+    parent = build(w)
+    pc = torch.from_numpy(w.coords).cuda()
+    with pytest.raises(ValueError):
+        smc.subdivide(parent, pc[:-1])
+    empty = smc.build_map(torch.zeros((0, 4), dtype=torch.int32, device="cuda"), (4, 4, 4), batch=1)
+    kids, child = smc.subdivide(empty, torch.zeros((0, 4), dtype=torch.int32, device="cuda"))
+    assert child.n == 0 and child.grid == (8, 8, 8)
+    bad = smc.build_map(torch.tensor([[0, 1, 1, 1], [0, 1, 1, 1]], dtype=torch.int32, device="cuda"), (4, 4, 4),
+                        batch=1, sync=False)
+    with pytest.raises(smc.SmcError) as e:
+        smc.subdivide(bad, torch.tensor([[0, 1, 1, 1], [0, 1, 1, 1]], dtype=torch.int32, device="cuda"))
+    assert e.value.name == "SMC_E_DUPLICATE"
+
+
 # ------------------------------------------------------------------ conv
 def _layer(w, dtype, layer=0, ksize=3, cin=None, cout=None):
     return S.layer_tensors(w, dtype, layer, ksize, cin, cout)
