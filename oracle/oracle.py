@@ -11,6 +11,9 @@ neighbour_map(coords, grid, k=3)          -> int32 [N, k^3]
 pair_lists(nbr)                           -> (counts int64[T], offsets int64[T+1], in_idx, out_idx)
 conv(coords, grid, feats, weight, bias, k=3, orientation=+1, rows=None, threads=1) -> fp64 [rows, Cout]
 subdivide(coords, keep=None)              -> int32 [M, 4] children, (parent row, octant) order
+activation(y, act)                        -> fp64, act 0 none / 1 ReLU / 2 SiLU
+group_stats(x, coords, batch, groups)     -> fp64 [batch, groups, 3] (sum, sum of squares, count)
+group_norm(x, coords, batch, groups, gamma, beta, eps, act) -> fp64 [N, C]
 
 The definition each follows is cited in smc_oracle.cpp.
 """
@@ -152,3 +155,60 @@ def subdivide(coords, keep=None) -> np.ndarray:
         children[:, o, 2] = 2 * c[:, 2] + cc
         children[:, o, 3] = 2 * c[:, 3] + e
     return children[kept].astype(np.int32)
+
+
+ACT_NONE, ACT_RELU, ACT_SILU = 0, 1, 2
+
+
+def activation(y, act: int) -> np.ndarray:
+    """The activations around the decoders' convs (Pixal3D MLX README
+    "Status": norms, activations, ResBlock; LATO.2 MLX port README "Status":
+    remaining sparse ops SparseGroupNorm32, activations): ReLU max(y, 0) and
+    SiLU y * sigmoid(y) = y / (1 + exp(-y)), in fp64."""
+    y = np.asarray(y, dtype=np.float64)
+    if act == ACT_NONE:
+        return y.copy()
+    if act == ACT_RELU:
+        return np.maximum(y, 0.0)
+    if act == ACT_SILU:
+        return y / (1.0 + np.exp(-y))
+    raise ValueError("act must be 0, 1 or 2")
+
+
+def group_stats(x, coords, batch: int, groups: int) -> np.ndarray:
+    """Per batch item b and channel group g (channels g*C/groups .. (g+1)*C/groups - 1):
+    the sum, the sum of squares and the number of values of x over the item's
+    rows, in fp64 -- what GroupNorm over a sparse tensor normalises with."""
+    x = np.asarray(x, dtype=np.float64)
+    n, c = x.shape
+    assert c % groups == 0
+    b = _coords(coords)[:, 0].astype(np.int64)
+    xg = x.reshape(n, groups, c // groups)
+    out = np.zeros((batch, groups, 3))
+    for item in range(batch):
+        rows = xg[b == item]
+        out[item, :, 0] = rows.sum(axis=(0, 2))
+        out[item, :, 1] = (rows * rows).sum(axis=(0, 2))
+        out[item, :, 2] = rows.shape[0] * (c // groups)
+    return out
+
+
+def group_norm(x, coords, batch: int, groups: int, gamma=None, beta=None, eps: float = 1e-5, act: int = 0):
+    """GroupNorm over a sparse tensor followed by an activation: for every
+    batch item and channel group, (x - mean) / sqrt(var + eps) with the
+    item's rows and the group's channels as the population (biased
+    variance), then gamma * . + beta per channel, then `act`."""
+    x = np.asarray(x, dtype=np.float64)
+    n, c = x.shape
+    st = group_stats(x, coords, batch, groups)
+    b = _coords(coords)[:, 0].astype(np.int64)
+    cnt = np.maximum(st[:, :, 2], 1.0)
+    mean = st[:, :, 0] / cnt
+    var = st[:, :, 1] / cnt - mean * mean
+    g_of_c = np.arange(c) // (c // groups)
+    y = (x - mean[b][:, g_of_c]) / np.sqrt(var[b][:, g_of_c] + eps)
+    if gamma is not None:
+        y = y * np.asarray(gamma, dtype=np.float64)[None, :]
+    if beta is not None:
+        y = y + np.asarray(beta, dtype=np.float64)[None, :]
+    return activation(y, act)

@@ -344,3 +344,39 @@ def test_subdivide_parent_and_octant_recovery(oracle_mod):
     np.testing.assert_array_equal(kids[:, 0], coords[parents, 0])
     np.testing.assert_array_equal(kids[:, 1:] // 2, coords[parents, 1:])
     np.testing.assert_array_equal(4 * (kids[:, 1] % 2) + 2 * (kids[:, 2] % 2) + kids[:, 3] % 2, octs)
+
+
+# ------------------------------------------------------------------ norm / activation
+def test_activation_matches_torch(oracle_mod):
+    x = np.random.default_rng(11).standard_normal((50, 7)) * 4
+    t = torch.from_numpy(x)
+    np.testing.assert_allclose(oracle_mod.activation(x, 2), torch.nn.functional.silu(t).numpy(), rtol=1e-12, atol=1e-15)
+    np.testing.assert_array_equal(oracle_mod.activation(x, 1), torch.relu(t).numpy())
+    np.testing.assert_array_equal(oracle_mod.activation(x, 0), x)
+
+
+def test_group_norm_matches_torch_per_item(oracle_mod):
+    """GroupNorm over a sparse tensor is torch's GroupNorm applied to each
+    batch item's rows laid out as [1, C, rows]; two items of unequal size
+    must not mix."""
+    rng = np.random.default_rng(12)
+    coords = np.array([[b, z, 0, 0] for b, cnt in ((0, 37), (1, 21)) for z in range(cnt)], np.int32)
+    x = rng.standard_normal((len(coords), 12)) * 3 + 1
+    gamma, beta = rng.standard_normal(12), rng.standard_normal(12)
+    got = oracle_mod.group_norm(x, coords, 2, 4, gamma, beta, 1e-5, act=2)
+    for item in range(2):
+        rows = coords[:, 0] == item
+        t = torch.from_numpy(x[rows].T.copy())[None]
+        ref = torch.nn.functional.group_norm(t, 4, torch.from_numpy(gamma), torch.from_numpy(beta), 1e-5)
+        ref = torch.nn.functional.silu(ref)[0].T.numpy()
+        np.testing.assert_allclose(got[rows], ref, rtol=1e-10, atol=1e-12)
+
+
+def test_group_stats_hand_example(oracle_mod):
+    coords = np.array([[0, 0, 0, 0], [1, 0, 0, 0], [0, 1, 0, 0]], np.int32)
+    x = np.array([[1.0, 2.0, 3.0, 4.0], [5.0, 6.0, 7.0, 8.0], [-1.0, 0.5, 2.0, -2.0]])
+    st = oracle_mod.group_stats(x, coords, 2, 2)
+    np.testing.assert_array_equal(st[0, 0], [1 + 2 - 1 + 0.5, 1 + 4 + 1 + 0.25, 4])
+    np.testing.assert_array_equal(st[0, 1], [3 + 4 + 2 - 2, 9 + 16 + 4 + 4, 4])
+    np.testing.assert_array_equal(st[1, 0], [11, 61, 2])
+    np.testing.assert_array_equal(st[1, 1], [15, 113, 2])
