@@ -203,6 +203,42 @@ def conv_variant_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, w
     return res
 
 
+def epilogue_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, w_d, b_d, out_d, reps=5):
+    """Median device time (ms) of one conv on the bench's map: plain; with
+    SiLU and a residual fused into the epilogue; the same plus the GroupNorm-32
+    statistics of its output (smc_conv_ex, a statistics pass behind the conv);
+    and plain followed by the statistics pass.  Untimed for the bench value."""
+    m = smc.build_map(coords_d, w.grid, batch=batch, stream=stream)
+    residual = torch.randn(out_d.shape, device=out_d.device).to(out_d.dtype)
+    stats = torch.zeros((batch, 32, 3), dtype=torch.float64, device=out_d.device)
+    runs = {
+        "plain": lambda: smc.conv(m, feats_d, w_d, b_d, out=out_d, stream=stream),
+        "silu_residual_fused": lambda: smc.conv(m, feats_d, w_d, b_d, out=out_d, stream=stream,
+                                                residual=residual, act="silu"),
+        "silu_residual_fused_with_stats": lambda: smc.conv(m, feats_d, w_d, b_d, out=out_d, stream=stream,
+                                                           residual=residual, act="silu", coords=coords_d,
+                                                           stats=stats, groups=32),
+        "plain_then_stats_pass": lambda: (smc.conv(m, feats_d, w_d, b_d, out=out_d, stream=stream),
+                                          smc.group_stats(out_d, coords_d, batch, 32, stats, stream=stream)),
+    }
+    res = {}
+    for name, fn in runs.items():
+        ts = []
+        for _ in range(reps + 1):
+            flush.zero_()
+            stats.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        res[name] = round(float(np.median(ts[1:])), 4)
+    m.free()
+    smc.status(stream)
+    return res
+
+
 def subdivide_times(smc, torch, stream, flush, reps=5):
     """Median device time (ms) of one decoder step's map, stage 2 -> 3 of the
     decoder chain (children inside the next shell kept): built from the parent
@@ -348,6 +384,7 @@ def run_gpu(args):
     map_times = prof.map_times
     variants = conv_variant_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, w_d, b_d, out_d)
     subdiv = subdivide_times(smc, torch, stream, flush)
+    epilogue = epilogue_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, w_d, b_d, out_d)
 
     total_ms = reduce_max(sum(times), world, dev)
     conv_ms = reduce_max(sum(conv_times) / len(conv_times), world, dev)
@@ -401,6 +438,7 @@ def run_gpu(args):
             "conv_tap_efficiency": round(eff, 4),
             "conv_variants_ms": variants,
             "subdivide_map_ms": subdiv,
+            "conv_epilogue_ms": epilogue,
             "roofline": {"kernel": "k_conv_tc", "bound": "tensor", "achieved": round(conv_tflops, 2),
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": round(conv_tflops / peaks["bf16_tflops"], 4), "traffic": traffic,

@@ -51,6 +51,9 @@ typedef struct smc_map smc_map;
 /* Storage type of feats, weight, bias and out in smc_conv. */
 typedef enum { SMC_F32 = 0, SMC_BF16 = 1, SMC_F16 = 2 } smc_dtype;
 
+/* Activations of the fused epilogue and of smc_group_norm. */
+typedef enum { SMC_ACT_NONE = 0, SMC_ACT_RELU = 1, SMC_ACT_SILU = 2 } smc_act;
+
 enum {
   SMC_OK = 0,
   SMC_E_ARG = -1,       /* null pointer, negative size, bad ksize/orientation/dtype value */
@@ -173,6 +176,59 @@ SMC_API int smc_map_stream_wait(const smc_map* map, void* stream);
 SMC_API int smc_conv(const smc_map* map, const void* feats, int64_t cin, const void* weight,
              const void* bias, void* out, int64_t cout, int32_t ksize, int32_t orientation,
              int32_t dtype, void* stream);
+
+/*
+ * smc_conv_ex -- smc_conv with a fused epilogue for the layers around the
+ * decoders' convs (norms, activations and ResBlocks: Pixal3D MLX README
+ * "Status"; SparseGroupNorm32 and activations: LATO.2 MLX port README
+ * "Status"):
+ *
+ *   out = round(act(bias + conv(feats)) + residual)
+ *
+ * residual : device [n, cout] in the output type, or NULL; it may be `out`
+ *            itself (y = conv + out) but must not otherwise overlap it.
+ * act      : SMC_ACT_NONE, SMC_ACT_RELU (max(y, 0)) or SMC_ACT_SILU
+ *            (y / (1 + exp(-y))), applied before the residual.
+ * stats    : device fp64 [batch, groups, 3] or NULL: for every batch item b
+ *            and channel group g (cout / groups channels each), the sum, the
+ *            sum of squares and the number of the stored output values of
+ *            the item's rows are ADDED (the caller zeroes it) -- what a
+ *            following smc_group_norm normalises with.  Computed by the
+ *            smc_group_stats pass over `out`, enqueued right behind the conv.
+ * coords   : device int32 [n, 4], the map's coordinates (the batch index of
+ *            each row); needed with stats.
+ * groups   : >= 1 and dividing cout; used with stats.
+ * Other arguments and errors as smc_conv.  smc_conv(...) is
+ * smc_conv_ex(..., residual NULL, act NONE, coords NULL, stats NULL, 1, ...).
+ */
+SMC_API int smc_conv_ex(const smc_map* map, const void* feats, int64_t cin, const void* weight,
+                const void* bias, const void* residual, void* out, int64_t cout, int32_t ksize,
+                int32_t orientation, int32_t dtype, int32_t act, const int32_t* coords, double* stats,
+                int32_t groups, void* stream);
+
+/*
+ * smc_group_stats -- add to stats (device fp64 [batch, groups, 3], zeroed by
+ * the caller) the sum, sum of squares and count of x (device [n, c], dtype)
+ * over each batch item's rows and each group of c / groups channels; the
+ * batch index of row v is coords[4v] (rows outside [0, batch) are skipped).
+ * batch * groups <= 1024.  Asynchronous on `stream`.
+ * Errors: SMC_E_ARG, SMC_E_DTYPE, SMC_E_SHAPE, SMC_E_CUDA.
+ */
+SMC_API int smc_group_stats(const void* x, int64_t n, int64_t c, const int32_t* coords, int32_t batch,
+                    int32_t groups, double* stats, int32_t dtype, void* stream);
+
+/*
+ * smc_group_norm -- GroupNorm over a sparse tensor and an activation:
+ *   out = round(act(gamma * (x - mean) / sqrt(var + eps) + beta))
+ * with mean and biased variance of the row's (batch item, channel group) from
+ * stats (as filled by smc_group_stats or smc_conv_ex).  gamma, beta: device
+ * [c] in dtype, or NULL (1 and 0).  out may equal x.  batch * groups <= 1024.
+ * Asynchronous on `stream`.  Errors: SMC_E_ARG, SMC_E_DTYPE, SMC_E_SHAPE,
+ * SMC_E_CUDA.
+ */
+SMC_API int smc_group_norm(const void* x, int64_t n, int64_t c, const int32_t* coords, int32_t batch,
+                   int32_t groups, const double* stats, const void* gamma, const void* beta, float eps,
+                   int32_t act, void* out, int32_t dtype, void* stream);
 
 /* n and the per-offset pair counts counts[27] (host) of a map. */
 SMC_API int smc_map_info(const smc_map* map, int64_t* n, int64_t counts[27]);

@@ -30,7 +30,8 @@ EXPORTS = [
     "smc_map_schedule", "smc_free_map", "smc_status", "smc_strerror",
     "smc_set_hash_capacity", "smc_set_profiling", "smc_map_timing", "smc_kernel_launches",
     "smc_build_map_async", "smc_map_wait", "smc_neighbour_map_noalloc", "smc_set_conv_variant",
-    "smc_set_map_lookup", "smc_map_stream_wait", "smc_subdivide",
+    "smc_set_map_lookup", "smc_map_stream_wait", "smc_subdivide", "smc_conv_ex", "smc_group_stats",
+    "smc_group_norm",
 ]
 
 
@@ -60,6 +61,9 @@ def lib() -> ctypes.CDLL:
         L.smc_map_wait.argtypes = [P]
         L.smc_map_stream_wait.argtypes = [P, P]
         L.smc_subdivide.argtypes = [P, P, P, P, P, P, P]
+        L.smc_conv_ex.argtypes = [P, P, i64, P, P, P, P, i64, i32, i32, i32, i32, P, P, i32, P]
+        L.smc_group_stats.argtypes = [P, i64, i64, P, i32, i32, P, i32, P]
+        L.smc_group_norm.argtypes = [P, i64, i64, P, i32, i32, P, P, P, ctypes.c_float, i32, P, i32, P]
         L.smc_neighbour_map_noalloc.argtypes = [P, i64, i32, P, P, P]
         L.smc_conv.argtypes = [P, P, i64, P, P, P, i64, i32, i32, i32, P]
         L.smc_map_info.argtypes = [P, P, P]
@@ -292,16 +296,27 @@ def clear_cache() -> None:
     _cache.clear()
 
 
+ACTS = {None: 0, "none": 0, "relu": 1, "silu": 2}
+
+
 def conv(m: Map, feats: torch.Tensor, weight: torch.Tensor, bias: Optional[torch.Tensor] = None,
          ksize: int = 3, orientation: int = 1, out: Optional[torch.Tensor] = None,
-         stream=None) -> torch.Tensor:
-    """Submanifold conv over map `m`: feats [N, Cin], KRSC weight [Cout, k, k, k, Cin]."""
+         stream=None, residual: Optional[torch.Tensor] = None, act: Optional[str] = None,
+         coords: Optional[torch.Tensor] = None, stats: Optional[torch.Tensor] = None,
+         groups: int = 1) -> torch.Tensor:
+    """Submanifold conv over map `m`: feats [N, Cin], KRSC weight [Cout, k, k, k, Cin].
+    Fused epilogue (smc_conv_ex): out = act(conv + bias) + residual, act in
+    {None, "relu", "silu"}; with `stats` (fp64 [batch, groups, 3], zeroed by
+    the caller) and `coords` (the map's int32 [N, 4]) the GroupNorm
+    statistics of the output are added into `stats`."""
     if feats.dtype not in _DTYPES:
         raise TypeError(f"unsupported dtype {feats.dtype}")
     if weight.dtype != feats.dtype or (bias is not None and bias.dtype != feats.dtype):
         raise TypeError("feats, weight and bias must share one dtype")
     if feats.dim() != 2 or feats.shape[0] != m.n:
         raise ValueError(f"feats must be [N={m.n}, Cin]")
+    if act not in ACTS:
+        raise ValueError(f"act must be one of {list(ACTS)}")
     cin = feats.shape[1]
     cout = weight.shape[0]
     if tuple(weight.shape) != (cout, ksize, ksize, ksize, cin):
@@ -315,9 +330,66 @@ def conv(m: Map, feats: torch.Tensor, weight: torch.Tensor, bias: Optional[torch
         out = torch.empty((m.n, cout), dtype=feats.dtype, device=feats.device)
     elif out.shape != (m.n, cout) or out.dtype != feats.dtype or not out.is_contiguous():
         raise ValueError("out must be a contiguous [N, Cout] tensor of the feats dtype")
+    if residual is not None and (residual.shape != (m.n, cout) or residual.dtype != feats.dtype
+                                 or not residual.is_contiguous()):
+        raise ValueError("residual must be a contiguous [N, Cout] tensor of the feats dtype")
+    if stats is not None:
+        if coords is None or coords.dtype != torch.int32 or coords.shape != (m.n, 4):
+            raise ValueError("stats need the map's int32 [N, 4] coords")
+        if stats.dtype != torch.float64 or stats.shape != (m.batch, groups, 3) or not stats.is_contiguous():
+            raise ValueError(f"stats must be a contiguous float64 [{m.batch}, {groups}, 3] tensor")
+        coords = coords.contiguous()
     with torch.cuda.device(feats.device):
-        _check(lib().smc_conv(m.handle, _ptr(feats), cin, _ptr(weight), _ptr(bias), _ptr(out), cout,
-                              ksize, orientation, _DTYPES[feats.dtype], _stream(stream)), "smc_conv")
+        if residual is None and act is None and stats is None:
+            _check(lib().smc_conv(m.handle, _ptr(feats), cin, _ptr(weight), _ptr(bias), _ptr(out), cout,
+                                  ksize, orientation, _DTYPES[feats.dtype], _stream(stream)), "smc_conv")
+        else:
+            _check(lib().smc_conv_ex(m.handle, _ptr(feats), cin, _ptr(weight), _ptr(bias), _ptr(residual),
+                                     _ptr(out), cout, ksize, orientation, _DTYPES[feats.dtype], ACTS[act],
+                                     _ptr(coords) if stats is not None else None, _ptr(stats), int(groups),
+                                     _stream(stream)), "smc_conv_ex")
+    return out
+
+
+def group_stats(x: torch.Tensor, coords: torch.Tensor, batch: int, groups: int,
+                stats: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """fp64 [batch, groups, 3]: (sum, sum of squares, count) of x [N, C] per
+    batch item (coords[:, 0]) and group of C / groups channels, added into
+    `stats` if given (smc_group_stats)."""
+    if x.dtype not in _DTYPES or x.dim() != 2:
+        raise TypeError("x must be a 2-D float32 / bfloat16 / float16 tensor")
+    n, c = x.shape
+    if coords.dtype != torch.int32 or coords.shape != (n, 4):
+        raise ValueError("coords must be int32 [N, 4]")
+    if stats is None:
+        stats = torch.zeros((batch, groups, 3), dtype=torch.float64, device=x.device)
+    x, coords = x.contiguous(), coords.contiguous()
+    with torch.cuda.device(x.device):
+        _check(lib().smc_group_stats(_ptr(x), n, c, _ptr(coords), int(batch), int(groups), _ptr(stats),
+                                     _DTYPES[x.dtype], _stream(stream)), "smc_group_stats")
+    return stats
+
+
+def group_norm(x: torch.Tensor, coords: torch.Tensor, batch: int, groups: int, stats: torch.Tensor,
+               gamma: Optional[torch.Tensor] = None, beta: Optional[torch.Tensor] = None, eps: float = 1e-5,
+               act: Optional[str] = None, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """GroupNorm over a sparse tensor then `act` (smc_group_norm), with the
+    statistics of `stats` (from group_stats or conv(..., stats=...))."""
+    if x.dtype not in _DTYPES or x.dim() != 2:
+        raise TypeError("x must be a 2-D float32 / bfloat16 / float16 tensor")
+    if act not in ACTS:
+        raise ValueError(f"act must be one of {list(ACTS)}")
+    n, c = x.shape
+    x, coords = x.contiguous(), coords.contiguous()
+    if out is None:
+        out = torch.empty_like(x)
+    for t in (gamma, beta):
+        if t is not None and (t.dtype != x.dtype or t.shape != (c,)):
+            raise ValueError("gamma and beta must be [C] of the x dtype")
+    with torch.cuda.device(x.device):
+        _check(lib().smc_group_norm(_ptr(x), n, c, _ptr(coords), int(batch), int(groups), _ptr(stats.contiguous()),
+                                    _ptr(gamma), _ptr(beta), float(eps), ACTS[act], _ptr(out), _DTYPES[x.dtype],
+                                    _stream(stream)), "smc_group_norm")
     return out
 
 

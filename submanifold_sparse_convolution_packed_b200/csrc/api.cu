@@ -466,6 +466,41 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   return SMC_OK;
 }
 
+// GroupNorm statistics are accumulated into kStatStripes copies (each block
+// adds into copy blockIdx % kStatStripes, spreading concurrent fp64 atomics
+// on one (item, group) over that many addresses) and folded into the
+// caller's array at the end: one pool allocation, memset and fold per call.
+constexpr int kStatStripes = 64;
+
+int stats_begin(int dev, cudaStream_t s, int batch, int groups, double** copies) {
+  *copies = nullptr;
+  const size_t bytes = static_cast<size_t>(kStatStripes) * batch * groups * 3 * sizeof(double);
+  cudaMemPool_t pool = device_pool(dev);
+  void* p = nullptr;
+  if (!pool || cudaMallocFromPoolAsync(&p, bytes, pool, s) != cudaSuccess) {
+    cudaGetLastError();
+    return SMC_E_OOM;
+  }
+  if (cudaMemsetAsync(p, 0, bytes, s) != cudaSuccess) {
+    cudaGetLastError();
+    cudaFreeAsync(p, s);
+    return SMC_E_CUDA;
+  }
+  *copies = static_cast<double*>(p);
+  return SMC_OK;
+}
+
+int stats_end(double* copies, int batch, int groups, double* stats, cudaStream_t s, bool ok) {
+  cudaError_t e = cudaSuccess;
+  if (ok) e = smc::launch_stats_fold(copies, kStatStripes, static_cast<int64_t>(batch) * groups * 3, stats, s);
+  cudaFreeAsync(copies, s);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return SMC_E_CUDA;
+  }
+  return SMC_OK;
+}
+
 }  // namespace
 
 namespace smc {
@@ -618,6 +653,48 @@ int smc_subdivide(const smc_map* parent, const int32_t* parent_coords, const uin
   return out;
 }
 
+int smc_group_stats(const void* x, int64_t n, int64_t c, const int32_t* coords, int32_t batch, int32_t groups,
+                    double* stats, int32_t dtype, void* stream) {
+  if (n < 0 || c < 1 || batch < 1 || groups < 1 || c % groups != 0) return SMC_E_ARG;
+  if (dtype != SMC_F32 && dtype != SMC_BF16 && dtype != SMC_F16) return SMC_E_DTYPE;
+  if (n == 0) return SMC_OK;
+  if (!x || !coords || !stats) return SMC_E_ARG;
+  if (static_cast<int64_t>(batch) * groups > 1024 || c > (1 << 24)) return SMC_E_SHAPE;
+  if (pending_cuda_error() != SMC_OK) return SMC_E_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int dev = 0;
+  cudaGetDevice(&dev);
+  smc::Epilogue ep;
+  ep.batch = batch;
+  ep.groups = groups;
+  ep.stripes = kStatStripes;
+  const int rc = stats_begin(dev, s, batch, groups, &ep.stats);
+  if (rc != SMC_OK) return rc;
+  const cudaError_t e = smc::launch_group_stats(x, n, static_cast<int>(c), coords, ep, dtype, s);
+  if (e != cudaSuccess) cudaGetLastError();
+  const int rc2 = stats_end(ep.stats, batch, groups, stats, s, e == cudaSuccess);
+  if (e != cudaSuccess) return SMC_E_CUDA;
+  return rc2;
+}
+
+int smc_group_norm(const void* x, int64_t n, int64_t c, const int32_t* coords, int32_t batch, int32_t groups,
+                   const double* stats, const void* gamma, const void* beta, float eps, int32_t act, void* out,
+                   int32_t dtype, void* stream) {
+  if (n < 0 || c < 1 || batch < 1 || groups < 1 || c % groups != 0 || !(eps >= 0.f)) return SMC_E_ARG;
+  if (act != SMC_ACT_NONE && act != SMC_ACT_RELU && act != SMC_ACT_SILU) return SMC_E_ARG;
+  if (dtype != SMC_F32 && dtype != SMC_BF16 && dtype != SMC_F16) return SMC_E_DTYPE;
+  if (n == 0) return SMC_OK;
+  if (!x || !coords || !stats || !out) return SMC_E_ARG;
+  if (static_cast<int64_t>(batch) * groups > 1024 || c > (1 << 24)) return SMC_E_SHAPE;
+  if (pending_cuda_error() != SMC_OK) return SMC_E_CUDA;
+  if (smc::launch_group_norm(x, n, static_cast<int>(c), coords, batch, groups, stats, gamma, beta, eps, act, out,
+                             dtype, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return SMC_E_CUDA;
+  }
+  return SMC_OK;
+}
+
 int smc_map_stream_wait(const smc_map* map, void* stream) {
   if (!map) return SMC_E_ARG;
   if (!map->done) return SMC_OK;  // empty map: nothing was enqueued
@@ -644,7 +721,16 @@ int smc_build_map(const int32_t* coords, int64_t n, int32_t batch, const int32_t
 
 int smc_conv(const smc_map* map, const void* feats, int64_t cin, const void* weight, const void* bias,
              void* out, int64_t cout, int32_t ksize, int32_t orientation, int32_t dtype, void* stream) {
+  return smc_conv_ex(map, feats, cin, weight, bias, nullptr, out, cout, ksize, orientation, dtype, SMC_ACT_NONE,
+                     nullptr, nullptr, 1, stream);
+}
+
+int smc_conv_ex(const smc_map* map, const void* feats, int64_t cin, const void* weight, const void* bias,
+                const void* residual, void* out, int64_t cout, int32_t ksize, int32_t orientation, int32_t dtype,
+                int32_t act, const int32_t* coords, double* stats, int32_t groups, void* stream) {
   if (!map) return SMC_E_ARG;
+  if (act != SMC_ACT_NONE && act != SMC_ACT_RELU && act != SMC_ACT_SILU) return SMC_E_ARG;
+  if (stats && (!coords || groups < 1 || cout % groups != 0)) return SMC_E_ARG;
   if (ksize != 1 && ksize != 3) return SMC_E_ARG;
   if (orientation != 1 && orientation != -1) return SMC_E_ARG;
   if (dtype != SMC_F32 && dtype != SMC_BF16 && dtype != SMC_F16) return SMC_E_DTYPE;
@@ -658,6 +744,9 @@ int smc_conv(const smc_map* map, const void* feats, int64_t cin, const void* wei
   }
   const size_t esz = dtype == SMC_F32 ? 4 : 2;
   const int taps = ksize == 3 ? 27 : 1;
+  // the residual may be the output itself (y = conv + out), not a part of it
+  if (residual && residual != out && ranges_overlap(out, n * cout * esz, residual, n * cout * esz))
+    return SMC_E_ALIAS;
   if (ranges_overlap(out, n * cout * esz, feats, n * cin * esz) ||
       ranges_overlap(out, n * cout * esz, weight, static_cast<size_t>(cout) * taps * cin * esz) ||
       ranges_overlap(out, n * cout * esz, bias, static_cast<size_t>(cout) * esz))
@@ -682,6 +771,9 @@ int smc_conv(const smc_map* map, const void* feats, int64_t cin, const void* wei
   a.orientation = orientation;
   a.dtype = dtype;
   a.err = st;
+  a.ep.residual = residual;
+  a.ep.act = act;
+  if (stats && static_cast<int64_t>(map->batch) * groups > 1024) return SMC_E_SHAPE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dev != map->device) return SMC_E_ARG;
   a.in_idx = map->in_idx;
@@ -712,6 +804,10 @@ int smc_conv(const smc_map* map, const void* feats, int64_t cin, const void* wei
     cudaGetLastError();
     return SMC_E_CUDA;
   }
+  // Group statistics of the stored output: a pass right behind the conv on
+  // the same stream (measured faster than folding them into the conv's
+  // epilogue, see conv_tc.cu).
+  if (stats) return smc_group_stats(out, n, cout, coords, map->batch, groups, stats, dtype, stream);
   return SMC_OK;
 }
 

@@ -21,6 +21,7 @@
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "epilogue.cuh"
 #include "kernels.h"
 
 namespace smc {
@@ -194,9 +195,11 @@ __global__ void __launch_bounds__(kOffThreads, 3) k_conv_offsets(const __grid_co
   }
 }
 
-// out = round(acc + bias), four values per thread.
+// out = round(act(acc + bias) + residual), four values per thread.
 __global__ void k_offsets_finalize(const float4* __restrict__ acc, const uint16_t* __restrict__ bias,
-                                   uint16_t* __restrict__ out, int64_t n4, int cout, int is_bf16) {
+                                   uint16_t* __restrict__ out, int64_t n4, int cout, int is_bf16, const Epilogue ep) {
+  const bool bf = is_bf16 != 0;
+  const uint16_t* res = static_cast<const uint16_t*>(ep.residual);
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const float4 a = acc[i];
@@ -205,11 +208,10 @@ __global__ void k_offsets_finalize(const float4* __restrict__ acc, const uint16_
     uint16_t h[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      if (bias) {
-        const uint16_t b = __ldg(bias + c + e);
-        x[e] += is_bf16 ? __bfloat162float(__ushort_as_bfloat16(b)) : __half2float(__ushort_as_half(b));
-      }
-      h[e] = is_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(x[e])) : __half_as_ushort(__float2half_rn(x[e]));
+      if (bias) x[e] += half_bits_to_float(__ldg(bias + c + e), bf);
+      x[e] = apply_act(x[e], ep.act);
+      if (res) x[e] += half_bits_to_float(res[i * 4 + e], bf);
+      h[e] = float_to_half_bits(x[e], bf);
     }
     reinterpret_cast<uint2*>(out)[i] =
         make_uint2(static_cast<uint32_t>(h[0]) | (static_cast<uint32_t>(h[1]) << 16),
@@ -288,7 +290,7 @@ cudaError_t launch_conv_offsets(const ConvArgs& a, float* acc, cudaStream_t s) {
   const int64_t n4 = a.n * a.cout / 4;
   k_offsets_finalize<<<static_cast<unsigned>((n4 + 255) / 256 < 148 * 16 ? (n4 + 255) / 256 : 148 * 16), 256, 0,
                        s>>>(reinterpret_cast<const float4*>(acc), static_cast<const uint16_t*>(a.bias),
-                            static_cast<uint16_t*>(a.out), n4, a.cout, p.is_bf16);
+                            static_cast<uint16_t*>(a.out), n4, a.cout, p.is_bf16, a.ep);
   count_launches(2);
   return cudaGetLastError();
 }

@@ -13,6 +13,7 @@
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "epilogue.cuh"
 #include "kernels.h"
 
 namespace smc {
@@ -33,7 +34,7 @@ template <typename T>
 __global__ void __launch_bounds__(kSimtThreads) k_conv_simt(
     const T* __restrict__ feats, const T* __restrict__ weight, const T* __restrict__ bias,
     T* __restrict__ out, const int32_t* __restrict__ nbr, int64_t n, int cin, int cout, int taps,
-    int orientation) {
+    int orientation, const Epilogue ep) {
   __shared__ float As[kBK][kBM + 4];
   __shared__ float Ws[kBK][kBN + 4];
   __shared__ int32_t s_idx[kBM];
@@ -89,6 +90,8 @@ __global__ void __launch_bounds__(kSimtThreads) k_conv_simt(
       __syncthreads();
     }
   }
+  // epilogue: y = act(acc + bias) + residual, rounded
+  const T* res = static_cast<const T*>(ep.residual);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int64_t m = row0 + ty * 4 + i;
@@ -96,7 +99,10 @@ __global__ void __launch_bounds__(kSimtThreads) k_conv_simt(
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int o = col0 + tx * 4 + j;
-      if (o < cout) out[m * cout + o] = from_f<T>(acc[i][j] + (bias ? to_f<T>(bias[o]) : 0.f));
+      if (o >= cout) break;
+      float y = apply_act(acc[i][j] + (bias ? to_f<T>(bias[o]) : 0.f), ep.act);
+      if (res) y += to_f<T>(res[m * cout + o]);
+      out[m * cout + o] = from_f<T>(y);
     }
   }
 }
@@ -109,19 +115,19 @@ cudaError_t launch_conv_simt(const ConvArgs& a, cudaStream_t s) {
       k_conv_simt<float><<<grid, kSimtThreads, 0, s>>>(
           static_cast<const float*>(a.feats), static_cast<const float*>(a.weight),
           static_cast<const float*>(a.bias), static_cast<float*>(a.out), a.nbr, a.n, a.cin, a.cout,
-          a.taps, a.orientation);
+          a.taps, a.orientation, a.ep);
       break;
     case kBF16:
       k_conv_simt<__nv_bfloat16><<<grid, kSimtThreads, 0, s>>>(
           static_cast<const __nv_bfloat16*>(a.feats), static_cast<const __nv_bfloat16*>(a.weight),
           static_cast<const __nv_bfloat16*>(a.bias), static_cast<__nv_bfloat16*>(a.out), a.nbr, a.n,
-          a.cin, a.cout, a.taps, a.orientation);
+          a.cin, a.cout, a.taps, a.orientation, a.ep);
       break;
     case kF16:
       k_conv_simt<__half><<<grid, kSimtThreads, 0, s>>>(
           static_cast<const __half*>(a.feats), static_cast<const __half*>(a.weight),
           static_cast<const __half*>(a.bias), static_cast<__half*>(a.out), a.nbr, a.n, a.cin, a.cout,
-          a.taps, a.orientation);
+          a.taps, a.orientation, a.ep);
       break;
     default:
       return cudaErrorInvalidValue;

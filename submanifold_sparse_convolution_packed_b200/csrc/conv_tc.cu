@@ -31,6 +31,7 @@
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "epilogue.cuh"
 #include "kernels.h"
 
 namespace smc {
@@ -65,13 +66,19 @@ struct TcParams {
   int64_t ntiles;
   int cin, cout, taps, orientation, bn, nsplit, stages, is_bf16, kb_elems;
   uint32_t tmem_cols;
+  Epilogue ep;  // activation and residual
 };
 
 // kPair: the CTA is one of a cluster pair sharing M = 256 MMAs (rows of two
 // consecutive schedule tiles, the union of their tap masks); it loads its own
 // 128 gathered rows and half of the weight block's N columns, and every load
 // and arrival counts on the even CTA's full barriers.
-template <bool kPair>
+// kEpi: 0 = bias only; 1 = activation and residual.  Separate instances keep
+// the plain conv free of the extra epilogue code, which measured 5-19% slower
+// even when unused.  (Group statistics of the output are a separate pass,
+// k_group_stats: folded into this epilogue they measured slower than the
+// pass, by the registers and the reduction work they add to every CTA.)
+template <bool kPair, int kEpi>
 __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant__ CUtensorMap fmap,
                                                         const __grid_constant__ CUtensorMap wmap,
                                                         const TcParams p) {
@@ -203,6 +210,15 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
     const int64_t g = tile * kTileRows + r;
     int32_t v = g < p.n ? (k3 ? __ldg(p.perm + g) : static_cast<int32_t>(g)) : -1;
     if (v >= p.n) v = -1;  // a schedule left incomplete by a failed build is skipped, never followed
+    if constexpr (kEpi >= 1) {
+      // the epilogue reads this row's residual: bring it into L2 now, while
+      // the tile's taps are gathered and multiplied
+      if (p.ep.residual && v >= 0) {
+        const char* rrow = static_cast<const char*>(p.ep.residual) + (static_cast<int64_t>(v) * p.cout + n0) * 2;
+        const int bytes = (p.cout - n0 < p.bn ? p.cout - n0 : p.bn) * 2;
+        for (int off = 0; off < bytes; off += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(rrow + off));
+      }
+    }
     // ---------------------------------------------------------- A gather (k=3)
     if (k3) {
       int32_t nb[kTaps];
@@ -245,44 +261,49 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
       }
     }
     // ---------------------------------------------------------- epilogue
+    // y = act(acc + bias) + residual, rounded and stored as 16-byte vectors.
     const bool ready = mbar_wait_bounded(bar_acc, 0, p.err) && !s_misc[1];
     tc_fence_after();
     if (ready) {
+      const bool bf = p.is_bf16 != 0;
+      constexpr bool extra = kEpi >= 1;  // activation and residual
+      const uint16_t* res = static_cast<const uint16_t*>(p.ep.residual);
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
       for (int c0 = 0; c0 < p.bn; c0 += 32) {
         float acc[32];
         tmem_ld_32cols(t_row + c0, acc);
-        if (v < 0) continue;
+        int ncols = p.bn - c0 < 32 ? p.bn - c0 : 32;
+        if (p.cout - (n0 + c0) < ncols) ncols = p.cout - (n0 + c0);
+        if (v >= 0) {
 #pragma unroll
-        for (int j = 0; j < 32; j += 8) {
-          const int col = n0 + c0 + j;
-          if (c0 + j >= p.bn || col >= p.cout) break;
-          uint32_t packed[4];
+          for (int j = 0; j < 32; j += 8) {
+            if (j >= ncols) break;
+            const int col = n0 + c0 + j;
+            const int64_t at = static_cast<int64_t>(v) * p.cout + col;
+            uint4 rv = make_uint4(0, 0, 0, 0);
+            if (extra && res) rv = *reinterpret_cast<const uint4*>(res + at);
+            const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
+            uint32_t packed[4];
 #pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            float x0 = acc[j + e], x1 = acc[j + e + 1];
-            if (p.bias) {
-              const uint16_t b0 = __ldg(p.bias + col + e), b1 = __ldg(p.bias + col + e + 1);
-              if (p.is_bf16) {
-                x0 += __bfloat162float(__ushort_as_bfloat16(b0));
-                x1 += __bfloat162float(__ushort_as_bfloat16(b1));
-              } else {
-                x0 += __half2float(__ushort_as_half(b0));
-                x1 += __half2float(__ushort_as_half(b1));
+            for (int e = 0; e < 8; e += 2) {
+              float x0 = acc[j + e], x1 = acc[j + e + 1];
+              if (p.bias) {
+                x0 += half_bits_to_float(__ldg(p.bias + col + e), bf);
+                x1 += half_bits_to_float(__ldg(p.bias + col + e + 1), bf);
               }
+              if constexpr (extra) {
+                x0 = apply_act(x0, p.ep.act);
+                x1 = apply_act(x1, p.ep.act);
+              }
+              if (extra && res) {
+                x0 += half_bits_to_float(static_cast<uint16_t>(rw[e / 2] & 0xFFFFu), bf);
+                x1 += half_bits_to_float(static_cast<uint16_t>(rw[e / 2] >> 16), bf);
+              }
+              const uint16_t h0 = float_to_half_bits(x0, bf), h1 = float_to_half_bits(x1, bf);
+              packed[e / 2] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
             }
-            uint16_t h0, h1;
-            if (p.is_bf16) {
-              h0 = __bfloat16_as_ushort(__float2bfloat16_rn(x0));
-              h1 = __bfloat16_as_ushort(__float2bfloat16_rn(x1));
-            } else {
-              h0 = __half_as_ushort(__float2half_rn(x0));
-              h1 = __half_as_ushort(__float2half_rn(x1));
-            }
-            packed[e / 2] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+            *reinterpret_cast<uint4*>(p.out + at) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
           }
-          *reinterpret_cast<uint4*>(p.out + static_cast<int64_t>(v) * p.cout + col) =
-              make_uint4(packed[0], packed[1], packed[2], packed[3]);
         }
       }
     }
@@ -316,6 +337,7 @@ static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr
 bool conv_tc_supported(const ConvArgs& a) {
   return (a.dtype == kBF16 || a.dtype == kF16) && a.cin >= 64 && a.cin % 16 == 0 && a.cout >= 16 &&
          a.cout % 16 == 0 && aligned16(a.feats) && aligned16(a.weight) && aligned16(a.out) &&
+         aligned16(a.ep.residual) &&
          a.n < (1ll << 31) && (a.taps == 1 || (a.taps == kTaps && a.perm && a.tile_mask)) &&
          encode_fn() != nullptr;
 }
@@ -354,9 +376,13 @@ static TcShape choose_shape(int cin, int cout, int64_t ntiles) {
   // K block.  Measured faster than 32-channel blocks with more CTAs per SM
   // (shells 128^3/128ch: 122 us vs 180 us), so the SM holds three CTAs of two
   // or more stages each when BN <= 128.
-  // (Pairs use the same per-CTA budget: sized for one CTA per SM, with
-  // eight stages, they measured slower still.)
-  t.ctas_per_sm = t.tmem_cols <= 128 ? 3 : 2;
+  // More CTAs per SM pull gathered rows faster than deeper pipelines: at
+  // BN = 128, 3 CTAs x 2 stages beat 2 x 3 and 1 x 6 (shells 128^3/128ch:
+  // 111 / 135 / 221 us); at BN <= 64, 4 x 2 beat 3 x 3 (256^3 varlen, 64ch:
+  // 776 vs 817 us) and 5 x 3 with 32-channel blocks (944 us).  (Pairs use the
+  // same per-CTA budget: sized for one CTA per SM, with eight stages, they
+  // measured slower still.)
+  t.ctas_per_sm = t.tmem_cols <= 64 ? 4 : (t.tmem_cols <= 128 ? 3 : 2);
   t.kb_elems = 64;
   (void)cin;
   const uint32_t per_sm = 228u * 1024u;
@@ -427,9 +453,12 @@ cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s) {
   p.is_bf16 = a.dtype == kBF16 ? 1 : 0;
   p.kb_elems = t.kb_elems;
   p.tmem_cols = t.tmem_cols;
+  p.ep = a.ep;
   cudaError_t e;
+  const int epi = a.ep.act != kActNone || a.ep.residual ? 1 : 0;
   if (t.pair) {
-    e = cudaFuncSetAttribute(k_conv_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(t.smem));
+    auto kern = epi == 1 ? k_conv_tc<true, 1> : k_conv_tc<true, 0>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(t.smem));
     if (e != cudaSuccess) return e;
     const int64_t ctas = 2 * ((ntiles + 1) / 2) * t.nsplit;
     cudaLaunchConfig_t cfg = {};
@@ -444,12 +473,13 @@ cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, k_conv_tc<true>, fmap, wmap, p);
+    e = cudaLaunchKernelEx(&cfg, kern, fmap, wmap, p);
   } else {
-    e = cudaFuncSetAttribute(k_conv_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(t.smem));
+    auto kern = epi == 1 ? k_conv_tc<false, 1> : k_conv_tc<false, 0>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(t.smem));
     if (e != cudaSuccess) return e;
     const int64_t units = ntiles * t.nsplit;
-    k_conv_tc<false><<<static_cast<unsigned>(units), kTcThreads, t.smem, s>>>(fmap, wmap, p);
+    kern<<<static_cast<unsigned>(units), kTcThreads, t.smem, s>>>(fmap, wmap, p);
     e = cudaGetLastError();
   }
   count_launches(1);

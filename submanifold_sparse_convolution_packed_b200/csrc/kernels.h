@@ -5,6 +5,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "epilogue.cuh"
+
 namespace smc {
 
 // Lookup structure of a map build (see map_build.cu).
@@ -79,6 +81,17 @@ cudaError_t launch_subdiv_emit(const int32_t* coords, int64_t n, const uint8_t* 
 cudaError_t launch_subdiv_lookups(const MapBuildArgs& a, const int32_t* parent_nbr, const int32_t* child_src,
                                   const int32_t* remap, cudaStream_t s);
 
+// GroupNorm over a sparse tensor (norm.cu): statistics of x per (batch item,
+// channel group) added into stats [batch, groups, 3], and the normalisation
+// y = act(gamma * (x - mean) / sqrt(var + eps) + beta) from such statistics.
+cudaError_t launch_group_stats(const void* x, int64_t n, int c, const int32_t* coords, const Epilogue& ep, int dtype,
+                               cudaStream_t s);
+// stats[i] += sum over s < stripes of copies[s * len + i]
+cudaError_t launch_stats_fold(const double* copies, int stripes, int64_t len, double* stats, cudaStream_t s);
+cudaError_t launch_group_norm(const void* x, int64_t n, int c, const int32_t* coords, int batch, int groups,
+                              const double* stats, const void* gamma, const void* beta, float eps, int act,
+                              void* out, int dtype, cudaStream_t s);
+
 // dtype codes as in smc.h
 enum DType : int { kF32 = 0, kBF16 = 1, kF16 = 2 };
 
@@ -96,6 +109,7 @@ struct ConvArgs {
   int64_t n;
   int cin, cout, taps, orientation, dtype;
   uint32_t* err;
+  Epilogue ep;                // activation, residual, group statistics
 };
 
 // cuTensorMapEncodeTiled, fetched from the driver through the runtime.
@@ -107,7 +121,8 @@ EncodeTiledFn encode_fn();
 
 // FMA kernel: every dtype, every shape.
 cudaError_t launch_conv_simt(const ConvArgs& a, cudaStream_t s);
-// tcgen05 kernel: bf16/fp16, cin % 16 == 0 and cin >= 64, cout % 16 == 0, 16-byte aligned.
+// tcgen05 kernel: bf16/fp16, cin % 16 == 0 and cin >= 64, cout % 16 == 0, 16-byte aligned
+// (feats, weight, out and residual).
 bool conv_tc_supported(const ConvArgs& a);
 cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s);
 // Conv kernel variant: 0 = default, 1 = one CTA per tile, 2 = CTA pairs,

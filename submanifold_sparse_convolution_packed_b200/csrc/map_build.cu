@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(kMapBlock) k_neighbours(
   __shared__ int32_t s_nbr[kMapBlock * kTaps];
   __shared__ int32_t s_cnt[kMapBlock / 32][kTaps];
   const uint64_t mask = (1ull << lg) - 1;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int64_t base = static_cast<int64_t>(blockIdx.x) * kMapBlock;
   const int64_t v = base + tid;
   uint32_t hits = 0, gk = 0;

@@ -420,6 +420,103 @@ def test_conv_variants_agree(name, dtype):
     smc.status()
 
 
+# ------------------------------------------------------------------ fused epilogue / GroupNorm
+def _np_stats(x, coords, batch, groups):
+    """fp64 (sum, sum of squares, count) per (item, group), summed directly."""
+    n, c = x.shape
+    xg = x.reshape(n, groups, c // groups)
+    st = np.zeros((batch, groups, 3))
+    for b in range(batch):
+        r = xg[coords[:, 0] == b]
+        st[b, :, 0], st[b, :, 1], st[b, :, 2] = r.sum(axis=(0, 2)), (r * r).sum(axis=(0, 2)), r.shape[0] * (c // groups)
+    return st
+
+
+@pytest.mark.parametrize("dtype,variant", [("bf16", 1), ("bf16", 2), ("bf16", 3), ("f32", 1), ("f16", 1)])
+@pytest.mark.parametrize("act", [None, "relu", "silu"])
+def test_conv_ex_epilogue(oracle_mod, dtype, variant, act):
+    """out = act(conv + bias) + residual, and the GroupNorm statistics of the
+    stored output: the output against the oracle, the statistics against
+    fp64 sums of that very output (the two-item shell workload, 64 -> 64
+    channels, 32 groups; bf16 on the three tensor-core variants, fp32 and
+    fp16 on their kernels)."""
+    w = workload("shell2")
+    m = build(w)
+    f, wt, b = _layer(w, dtype, 2)
+    rng = np.random.default_rng(31)
+    res = S.round_to(rng.standard_normal((w.n, w.cout)).astype(np.float32), dtype)
+    coords = torch.from_numpy(w.coords).cuda()
+    stats = torch.zeros((2, 32, 3), dtype=torch.float64, device="cuda")
+    smc.set_conv_variant(variant)
+    try:
+        out = smc.conv(m, dev(f, dtype), dev(wt, dtype), dev(b, dtype), residual=dev(res, dtype), act=act,
+                       coords=coords, stats=stats, groups=32)
+    finally:
+        smc.set_conv_variant(0)
+    smc.status()
+    got = host(out)
+    ref = oracle_mod.activation(oracle_mod.conv(w.coords, w.grid, f, wt, b, 3, 1, threads=THREADS),
+                                {None: 0, "relu": 1, "silu": 2}[act]) + res
+    check_close(got, ref, dtype, f"conv_ex {dtype} v{variant} act={act}")
+    np.testing.assert_allclose(stats.cpu().numpy(), _np_stats(got, w.coords, 2, 32), rtol=1e-9, atol=1e-6)
+
+
+def test_conv_ex_residual_in_place(oracle_mod):
+    """y = conv + out: the residual may be the output buffer itself."""
+    w = workload("shell2")
+    m = build(w)
+    f, wt, b = _layer(w, "bf16", 4)
+    start = S.round_to(np.random.default_rng(32).standard_normal((w.n, w.cout)).astype(np.float32), "bf16")
+    out = dev(start, "bf16")
+    smc.conv(m, dev(f, "bf16"), dev(wt, "bf16"), dev(b, "bf16"), out=out, residual=out)
+    smc.status()
+    ref = oracle_mod.conv(w.coords, w.grid, f, wt, b, 3, 1, threads=THREADS) + start
+    check_close(host(out), ref, "bf16", "in-place residual")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_group_norm(oracle_mod, dtype):
+    w = workload("shell2")
+    rng = np.random.default_rng(33)
+    x = S.round_to((rng.standard_normal((w.n, 64)) * 2 + 0.5).astype(np.float32), dtype)
+    gamma = S.round_to(rng.standard_normal(64).astype(np.float32), dtype)
+    beta = S.round_to(rng.standard_normal(64).astype(np.float32), dtype)
+    coords = torch.from_numpy(w.coords).cuda()
+    st = smc.group_stats(dev(x, dtype), coords, 2, 32)
+    np.testing.assert_allclose(st.cpu().numpy(), _np_stats(x.astype(np.float64), w.coords, 2, 32), rtol=1e-9, atol=1e-6)
+    out = smc.group_norm(dev(x, dtype), coords, 2, 32, st, dev(gamma, dtype), dev(beta, dtype), 1e-5, act="silu")
+    smc.status()
+    ref = oracle_mod.group_norm(x, w.coords, 2, 32, gamma, beta, 1e-5, act=2)
+    check_close(host(out), ref, dtype, f"group_norm {dtype}")
+
+
+def test_resblock_chain(oracle_mod):
+    """A ResBlock on one cached map: GroupNorm32 + SiLU, conv (statistics of
+    its output fused), GroupNorm32 + SiLU, conv + skip.  Every step is checked
+    against the oracle fed the GPU's own input to that step."""
+    w = workload("shell2")
+    m = build(w)
+    coords = torch.from_numpy(w.coords).cuda()
+    rng = np.random.default_rng(34)
+    x = S.round_to(rng.standard_normal((w.n, 64)).astype(np.float32), "bf16")
+    _, w1, b1 = _layer(w, "bf16", 5)
+    _, w2, b2 = _layer(w, "bf16", 6)
+    xt = dev(x, "bf16")
+    st0 = smc.group_stats(xt, coords, 2, 32)
+    h = smc.group_norm(xt, coords, 2, 32, st0, act="silu")
+    check_close(host(h), oracle_mod.group_norm(x, w.coords, 2, 32, act=2), "bf16", "gn1")
+    st1 = torch.zeros((2, 32, 3), dtype=torch.float64, device="cuda")
+    h1 = smc.conv(m, h, dev(w1, "bf16"), dev(b1, "bf16"), coords=coords, stats=st1, groups=32)
+    check_close(host(h1), oracle_mod.conv(w.coords, w.grid, host(h), w1, b1, 3, 1, threads=THREADS), "bf16", "conv1")
+    np.testing.assert_allclose(st1.cpu().numpy(), _np_stats(host(h1), w.coords, 2, 32), rtol=1e-9, atol=1e-6)
+    h2 = smc.group_norm(h1, coords, 2, 32, st1, act="silu")
+    check_close(host(h2), oracle_mod.group_norm(host(h1), w.coords, 2, 32, act=2), "bf16", "gn2")
+    y = smc.conv(m, h2, dev(w2, "bf16"), dev(b2, "bf16"), residual=xt)
+    ref = oracle_mod.conv(w.coords, w.grid, host(h2), w2, b2, 3, 1, threads=THREADS) + x
+    check_close(host(y), ref, "bf16", "conv2 + skip")
+    smc.status()
+
+
 def test_conv_errors():
     w = workload("tiny")
     m = build(w)
