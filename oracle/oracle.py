@@ -14,6 +14,10 @@ subdivide(coords, keep=None)              -> int32 [M, 4] children, (parent row,
 activation(y, act)                        -> fp64, act 0 none / 1 ReLU / 2 SiLU
 group_stats(x, coords, batch, groups)     -> fp64 [batch, groups, 3] (sum, sum of squares, count)
 group_norm(x, coords, batch, groups, gamma, beta, eps, act) -> fp64 [N, C]
+downsample(coords, grid, feats=None, mode=POOL_MEAN, batch=None)
+                                          -> (parent coords [M, 4], pooled fp64 [M, C] or None,
+                                              subdivision mask uint8 [M, 8], parent row int32 [N])
+upsample(coords, mask, feats=None)        -> (child coords [K, 4], child feats fp64 [K, C] or None)
 
 The definition each follows is cited in smc_oracle.cpp.
 """
@@ -212,3 +216,93 @@ def group_norm(x, coords, batch: int, groups: int, gamma=None, beta=None, eps: f
     if beta is not None:
         y = y + np.asarray(beta, dtype=np.float64)[None, :]
     return activation(y, act)
+
+
+POOL_MAX, POOL_MEAN = 0, 1
+
+
+def subidx(dz, dy, dx) -> int:
+    """Child index inside a factor-2 parent as the subdivision mask numbers
+    it: the offset along spatial axis i is subidx // 2**i % 2, axis 0 (z)
+    varying fastest -- the reverse of the C order subdivide() uses (shared
+    sparse-core commit log, the masked-upsample entry)."""
+    return dz + 2 * dy + 4 * dx
+
+
+def downsample(coords, grid, feats=None, mode: int = POOL_MEAN, batch: Optional[int] = None):
+    """Pooling by 2 into parent voxels, SparseDownsample(2) (shared
+    sparse-core commit log: modes 'max' and 'mean'; Pixal3D MLX README
+    "Status").  Row i of (b, z, y, x) pools into the parent
+    (b, z // 2, y // 2, x // 2).  Parents are numbered in order of first
+    appearance: walking the rows in order, a parent not seen before takes the
+    next index.  Returns the parents' coordinates, their pooled features
+    (elementwise max, or the mean over the children present, in fp64), the
+    subdivision mask (mask[p, subidx] = 1 for every child present) and each
+    row's parent.  Coordinates outside (batch, grid) and repeated sites are
+    errors, as in the map build."""
+    c = _coords(coords).astype(np.int64)
+    g = _grid(grid)
+    n = c.shape[0]
+    nb = (int(c[:, 0].max()) + 1 if n else 1) if batch is None else batch
+    lo_ok = (c >= 0).all(axis=1)
+    hi_ok = (c[:, 0] < nb) & (c[:, 1] < g[0]) & (c[:, 2] < g[1]) & (c[:, 3] < g[2])
+    if n and not (lo_ok & hi_ok).all():
+        raise OracleError(-2)
+    index = {}
+    parent_coords = []
+    parent = np.empty(n, dtype=np.int32)
+    for i in range(n):
+        b, z, y, x = (int(v) for v in c[i])
+        key = (b, z // 2, y // 2, x // 2)
+        if key not in index:
+            index[key] = len(parent_coords)
+            parent_coords.append(key)
+        parent[i] = index[key]
+    m = len(parent_coords)
+    mask = np.zeros((m, 8), dtype=np.uint8)
+    for i in range(n):
+        j = subidx(int(c[i, 1]) % 2, int(c[i, 2]) % 2, int(c[i, 3]) % 2)
+        if mask[parent[i], j]:
+            raise OracleError(-3)
+        mask[parent[i], j] = 1
+    pc = np.array(parent_coords, dtype=np.int32).reshape(m, 4)
+    pooled = None
+    if feats is not None:
+        f = np.asarray(feats, dtype=np.float64)
+        if f.shape[0] != n:
+            raise ValueError("feats must have one row per coordinate")
+        if mode == POOL_MAX:
+            pooled = np.full((m, f.shape[1]), -np.inf)
+            np.maximum.at(pooled, parent, f)
+        elif mode == POOL_MEAN:
+            pooled = np.zeros((m, f.shape[1]))
+            np.add.at(pooled, parent, f)
+            pooled /= mask.sum(axis=1, dtype=np.float64)[:, None]
+        else:
+            raise ValueError("mode must be POOL_MAX (0) or POOL_MEAN (1)")
+    return pc, pooled, mask, parent
+
+
+def upsample(coords, mask, feats=None):
+    """Masked expansion by 2, SparseUpsample(2) (shared sparse-core commit
+    log, the masked-upsample entry; Pixal3D MLX README, remaining ops): parent
+    p emits the child at subidx j wherever mask[p, j] != 0 -- 0 to 8
+    children, unlike subdivide(), which always emits 8 -- at
+    (b, 2z + j % 2, 2y + j // 2 % 2, 2x + j // 4 % 2), listed parent by
+    parent, j ascending.  Each child carries its parent's features."""
+    c = _coords(coords).astype(np.int64)
+    n = c.shape[0]
+    mk = np.asarray(mask).reshape(n, 8) != 0
+    children, src = [], []
+    for p in range(n):
+        b, z, y, x = (int(v) for v in c[p])
+        for j in range(8):
+            if mk[p, j]:
+                children.append((b, 2 * z + j % 2, 2 * y + j // 2 % 2, 2 * x + j // 4 % 2))
+                src.append(p)
+    kids = np.array(children, dtype=np.int32).reshape(len(children), 4)
+    out = None
+    if feats is not None:
+        f = np.asarray(feats, dtype=np.float64)
+        out = f[np.array(src, dtype=np.int64)] if src else np.zeros((0, f.shape[1]))
+    return kids, out

@@ -71,3 +71,47 @@ def test_pins_reject_planted_mistake(name):
             got = _run(dll, coords, grid, feats, w, b, 3, s)
             caught |= not np.allclose(got, ref, rtol=1e-12, atol=1e-12)
         assert caught, f"planted mistake {name!r} passed the dense-equivalence pin"
+
+
+# Planted mistakes in the Python half of the oracle (resampling): each is
+# applied to a copy of oracle.py loaded as a throw-away module, and at least
+# one of the resampling pins must fail on it.
+PY_SRC = os.path.join(os.path.dirname(SRC), "oracle.py")
+PY_MUTATIONS = {
+    "subidx_c_order": ("return dz + 2 * dy + 4 * dx", "return 4 * dz + 2 * dy + dx"),
+    "upsample_c_order": ("(b, 2 * z + j % 2, 2 * y + j // 2 % 2, 2 * x + j // 4 % 2)",
+                         "(b, 2 * z + j // 4 % 2, 2 * y + j // 2 % 2, 2 * x + j % 2)"),
+    "parent_rounds_up": ("key = (b, z // 2, y // 2, x // 2)", "key = (b, (z + 1) // 2, y // 2, x // 2)"),
+    "mean_not_divided": ("pooled /= mask.sum(axis=1, dtype=np.float64)[:, None]", "pass"),
+    "max_sums": ("np.maximum.at(pooled, parent, f)", "pooled[:] = 0.0\n            np.add.at(pooled, parent, f)"),
+    "upsample_wrong_source": ("src.append(p)", "src.append(max(p - 1, 0))"),
+}
+RESAMPLE_PINS = ["test_golden_downsample_upsample", "test_downsample_matches_dense_pooling",
+                 "test_upsample_matches_nearest_interpolation", "test_upsample_index_is_subdivide_octant_reversed",
+                 "test_downsample_upsample_round_trip"]
+
+
+def _py_mutant(name):
+    import types
+    old, new = PY_MUTATIONS[name]
+    src = open(PY_SRC).read()
+    assert src.count(old) == 1, f"mutation {name} no longer applies"
+    mod = types.ModuleType(f"oracle_mutant_{name}")
+    mod.__file__ = PY_SRC
+    exec(compile(src.replace(old, new), PY_SRC, "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTATIONS))
+def test_resample_pins_reject_planted_mistake(name):
+    import tests.test_oracle_pins as pins
+    mod = _py_mutant(name)
+    failed = []
+    for pin in RESAMPLE_PINS:
+        fn = getattr(pins, pin)
+        args = [(6, 4, 8)] if pin == "test_downsample_matches_dense_pooling" else []
+        try:
+            fn(mod, *args)
+        except Exception:
+            failed.append(pin)
+    assert failed, f"planted mistake {name!r} passed every resampling pin"

@@ -17,7 +17,10 @@ one of them:
 * invariants: centre tap is the identity map, neighbour symmetry, batch
   isolation, linearity, brute-force all-pairs neighbour search;
 * subdivision: a hand-listed voxel, a full box that must become the full
-  doubled box, and parent/octant recovery from each child.
+  doubled box, and parent/octant recovery from each child;
+* downsample / upsample: a hand-worked example, dense max_pool3d and
+  avg_pool3d, nearest interpolation, the octant bit reversal against
+  subdivide, and the round trip.
 
 Grids are deliberately non-cubic and channel counts unequal so that an axis
 swap or an operand transposition cannot cancel out.
@@ -380,3 +383,120 @@ def test_group_stats_hand_example(oracle_mod):
     np.testing.assert_array_equal(st[0, 1], [3 + 4 + 2 - 2, 9 + 16 + 4 + 4, 4])
     np.testing.assert_array_equal(st[1, 0], [11, 61, 2])
     np.testing.assert_array_equal(st[1, 1], [15, 113, 2])
+
+
+# ------------------------------------------------------------------ downsample / upsample
+def test_golden_downsample_upsample(oracle_mod):
+    g = _golden("downsample_upsample.json")
+    coords, feats = np.array(g["coords"], np.int32), np.array(g["feats"])
+    pc, mx, mask, parent = oracle_mod.downsample(coords, g["grid"], feats, oracle_mod.POOL_MAX, g["batch"])
+    assert pc.tolist() == g["expected_parent_coords"]
+    assert parent.tolist() == g["expected_parent_of_row"]
+    assert mask.tolist() == g["expected_mask"]
+    np.testing.assert_array_equal(mx, g["expected_max"])
+    _, mean, _, _ = oracle_mod.downsample(coords, g["grid"], feats, oracle_mod.POOL_MEAN, g["batch"])
+    np.testing.assert_allclose(mean, np.array(g["expected_mean_num"]) / np.array(g["expected_mean_den"])[:, None],
+                               rtol=1e-15)
+    kids, kf = oracle_mod.upsample(pc, mask, np.array(g["upsample_feats"]))
+    assert kids.tolist() == g["expected_children"]
+    np.testing.assert_array_equal(kf, g["expected_child_feats"])
+
+
+def _dense_volume(coords, feats, grid, batch, fill):
+    vol = torch.full((batch, feats.shape[1], *grid), fill, dtype=torch.float64)
+    c = torch.from_numpy(coords.astype(np.int64))
+    vol[c[:, 0], :, c[:, 1], c[:, 2], c[:, 3]] = torch.from_numpy(feats)
+    return vol
+
+
+@pytest.mark.parametrize("grid", [(6, 4, 8), (5, 7, 3)])
+def test_downsample_matches_dense_pooling(oracle_mod, grid):
+    """On a dense grid, max pooling is max_pool3d(2, stride 2) with empty sites
+    at -inf, and mean pooling is avg_pool3d of the features over avg_pool3d
+    of the occupancy (both zero at empty sites); odd extents pool a partial
+    last window (ceil_mode)."""
+    rng = np.random.default_rng(21)
+    batch = 2
+    sites = np.array(list(itertools.product(range(batch), *(range(s) for s in grid))), np.int32)
+    coords = sites[rng.random(len(sites)) < 0.3]
+    coords = coords[rng.permutation(len(coords))]
+    feats = rng.standard_normal((len(coords), 3))
+    pool = dict(kernel_size=2, stride=2, ceil_mode=True)
+    pc, mx, mask, _ = oracle_mod.downsample(coords, grid, feats, oracle_mod.POOL_MAX, batch)
+    ref = torch.nn.functional.max_pool3d(_dense_volume(coords, feats, grid, batch, -np.inf), **pool)
+    b, z, y, x = (torch.from_numpy(pc[:, i].astype(np.int64)) for i in range(4))
+    np.testing.assert_array_equal(mx, ref[b, :, z, y, x].numpy())
+    _, mean, _, _ = oracle_mod.downsample(coords, grid, feats, oracle_mod.POOL_MEAN, batch)
+    num = torch.nn.functional.avg_pool3d(_dense_volume(coords, feats, grid, batch, 0.0), **pool)
+    occ = torch.nn.functional.avg_pool3d(_dense_volume(coords, np.ones((len(coords), 1)), grid, batch, 0.0), **pool)
+    np.testing.assert_allclose(mean, (num / occ)[b, :, z, y, x].numpy(), rtol=1e-12, atol=1e-14)
+    # every occupied window is a parent, once; its mask counts its sites
+    occupied = torch.nonzero(occ[:, 0] > 0).numpy()
+    assert sorted(map(tuple, pc.tolist())) == sorted(map(tuple, occupied.tolist()))
+    assert mask.sum() == len(coords)
+
+
+def test_upsample_matches_nearest_interpolation(oracle_mod):
+    """Each kept child carries its parent's features: nearest upsampling by 2
+    of the dense parent volume (interpolate, mode 'nearest') sampled at the
+    children; the children are exactly the masked sites of the doubled box."""
+    rng = np.random.default_rng(22)
+    grid, batch = (3, 4, 2), 2
+    sites = np.array(list(itertools.product(range(batch), *(range(s) for s in grid))), np.int32)
+    coords = sites[rng.random(len(sites)) < 0.6]
+    feats = rng.standard_normal((len(coords), 4))
+    mask = (rng.random((len(coords), 8)) < 0.5).astype(np.uint8)
+    kids, kf = oracle_mod.upsample(coords, mask, feats)
+    up = torch.nn.functional.interpolate(_dense_volume(coords, feats, grid, batch, 0.0), scale_factor=2,
+                                         mode="nearest")
+    b, z, y, x = (torch.from_numpy(kids[:, i].astype(np.int64)) for i in range(4))
+    np.testing.assert_array_equal(kf, up[b, :, z, y, x].numpy())
+    want = set()
+    for p, (cb, cz, cy, cx) in enumerate(coords.tolist()):
+        for dz, dy, dx in itertools.product(range(2), repeat=3):
+            if mask[p, dz + 2 * dy + 4 * dx]:
+                want.add((cb, 2 * cz + dz, 2 * cy + dy, 2 * cx + dx))
+    assert len(kids) == int(mask.sum()) and set(map(tuple, kids.tolist())) == want
+
+
+def test_upsample_index_is_subdivide_octant_reversed(oracle_mod):
+    """With every child kept, upsample lists each parent's children at subidx
+    j where subdivide lists them at the C-order octant whose three bits are
+    j's in reverse (the commit log notes the two orders are reverses)."""
+    coords = np.array([[0, 1, 2, 3], [1, 0, 5, 2]], np.int32)
+    kids, _ = oracle_mod.upsample(coords, np.ones((2, 8), np.uint8))
+    sub = oracle_mod.subdivide(coords)
+    rev = [int(f"{j:03b}"[::-1], 2) for j in range(8)]
+    for p in range(2):
+        assert kids[8 * p:8 * p + 8].tolist() == sub[8 * p + np.array(rev)].tolist()
+
+
+def test_downsample_upsample_round_trip(oracle_mod):
+    """Upsampling the parents with the mask the downsample recorded gives back
+    exactly the input sites; every row halves to its parent's coordinates."""
+    rng = np.random.default_rng(23)
+    coords = np.unique(rng.integers(0, 11, size=(300, 4)), axis=0).astype(np.int32)
+    coords[:, 0] %= 3
+    coords = np.unique(coords, axis=0)[rng.permutation(len(np.unique(coords, axis=0)))]
+    pc, _, mask, parent = oracle_mod.downsample(coords, (11, 11, 11))
+    kids, _ = oracle_mod.upsample(pc, mask)
+    assert sorted(map(tuple, kids.tolist())) == sorted(map(tuple, coords.tolist()))
+    np.testing.assert_array_equal(pc[parent, 0], coords[:, 0])
+    np.testing.assert_array_equal(pc[parent, 1:], coords[:, 1:] // 2)
+    # first-appearance numbering: parent indices first occur in increasing order
+    first = np.unique(parent, return_index=True)[1]
+    assert (np.diff(first) > 0).all() and parent[0] == 0
+
+
+def test_downsample_errors(oracle_mod):
+    c = np.array([[0, 0, 0, 0], [0, 0, 0, 0]], np.int32)
+    with pytest.raises(oracle_mod.OracleError) as e:
+        oracle_mod.downsample(c, (2, 2, 2))
+    assert e.value.code == -3
+    with pytest.raises(oracle_mod.OracleError) as e:
+        oracle_mod.downsample(np.array([[0, 2, 0, 0]], np.int32), (2, 2, 2))
+    assert e.value.code == -2
+    pc, pooled, mask, parent = oracle_mod.downsample(np.zeros((0, 4), np.int32), (2, 2, 2), np.zeros((0, 3)))
+    assert pc.shape == (0, 4) and pooled.shape == (0, 3) and mask.shape == (0, 8) and parent.shape == (0,)
+    kids, kf = oracle_mod.upsample(pc, mask, pooled)
+    assert kids.shape == (0, 4) and kf.shape == (0, 3)
