@@ -275,6 +275,55 @@ def subdivide_times(smc, torch, stream, flush, reps=5):
             "incremental": round(float(np.median(inc[1:])), 4), "full_build": round(float(np.median(full[1:])), 4)}
 
 
+def resample_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, peaks, reps=5):
+    """Median device time (ms) of the pooling and expansion calls on the
+    bench's voxels and features (bf16, Cin channels), each call whole
+    (scratch clears, all kernels, its host read of the count):
+    smc_downsample (max and mean) and smc_upsample of the parents with the
+    recorded mask, their features and the parents' map (child map included).
+    GB/s counts the algorithmic bytes of each call: coordinates, features,
+    mask and parent index read or written once.  Untimed for the bench value."""
+    c, es, n = feats_d.shape[1], feats_d.element_size(), w.n
+    out = {}
+    for mode in ("max", "mean"):
+        ts = []
+        for _ in range(reps + 1):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            pc, pooled, mask, parent = smc.downsample(coords_d, w.grid, feats_d, mode, batch=batch, stream=stream)
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ms = float(np.median(ts[1:]))
+        m = pc.shape[0]
+        nbytes = 16 * n + n * c * es + 16 * m + 8 * m + 4 * n + m * c * es
+        out[f"downsample_{mode}"] = {"ms": round(ms, 4), "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
+    half = tuple((g + 1) // 2 for g in w.grid)
+    pm = smc.build_map(pc, half, batch=batch, stream=stream)
+    ts = []
+    for _ in range(reps + 1):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        kids, kf, child = smc.upsample(pc, mask, pooled, parent=pm, stream=stream)
+        child.stream_wait(stream)
+        e1.record(stream)
+        e1.synchronize()
+        child.wait()
+        child.free()
+        ts.append(e0.elapsed_time(e1))
+    pm.free()
+    ms = float(np.median(ts[1:]))
+    k = kids.shape[0]
+    nbytes = 16 * m + 8 * m + m * c * es + 16 * k + k * c * es
+    out["upsample_with_child_map"] = {"ms": round(ms, 4), "gbs_features_and_coords": round(nbytes / (ms * 1e-3) / 1e9, 1)}
+    out["sizes"] = {"rows": n, "parents": m, "children": k, "channels": c, "dtype": "bf16"}
+    out["hbm_peak_gbs"] = peaks["hbm_gbs"]
+    smc.status(stream)
+    return out
+
+
 def run_gpu(args):
     import torch
 
@@ -385,6 +434,7 @@ def run_gpu(args):
     variants = conv_variant_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, w_d, b_d, out_d)
     subdiv = subdivide_times(smc, torch, stream, flush)
     epilogue = epilogue_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, w_d, b_d, out_d)
+    resample = resample_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, peaks)
 
     total_ms = reduce_max(sum(times), world, dev)
     conv_ms = reduce_max(sum(conv_times) / len(conv_times), world, dev)
@@ -439,6 +489,7 @@ def run_gpu(args):
             "conv_variants_ms": variants,
             "subdivide_map_ms": subdiv,
             "conv_epilogue_ms": epilogue,
+            "resample": resample,
             "roofline": {"kernel": "k_conv_tc", "bound": "tensor", "achieved": round(conv_tflops, 2),
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": round(conv_tflops / peaks["bf16_tflops"], 4), "traffic": traffic,

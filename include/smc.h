@@ -54,6 +54,9 @@ typedef enum { SMC_F32 = 0, SMC_BF16 = 1, SMC_F16 = 2 } smc_dtype;
 /* Activations of the fused epilogue and of smc_group_norm. */
 typedef enum { SMC_ACT_NONE = 0, SMC_ACT_RELU = 1, SMC_ACT_SILU = 2 } smc_act;
 
+/* Pooling of smc_downsample: elementwise max, or mean over the children present. */
+typedef enum { SMC_POOL_MAX = 0, SMC_POOL_MEAN = 1 } smc_pool;
+
 enum {
   SMC_OK = 0,
   SMC_E_ARG = -1,       /* null pointer, negative size, bad ksize/orientation/dtype value */
@@ -142,6 +145,73 @@ SMC_API int smc_map_wait(const smc_map* map);
  */
 SMC_API int smc_subdivide(const smc_map* parent, const int32_t* parent_coords, const uint8_t* keep,
                   int32_t* child_coords, int64_t* m, void* stream, smc_map** child);
+
+/*
+ * smc_downsample -- pooling by 2 into parent voxels (SparseDownsample(2);
+ * shared sparse-core commit log: modes 'max' and 'mean', which differ between
+ * the models; Pixal3D MLX README "Status").
+ *
+ * Row i at (b, z, y, x) pools into the parent (b, z/2, y/2, x/2) (integer
+ * halves; odd extents give a partial last window).  Parents are numbered in
+ * order of first appearance among the rows (the row order, not a sort).
+ *
+ * coords        : device int32 [n, 4], 16-byte aligned, inside
+ *                 [0, batch) x [0, grid[0]) x [0, grid[1]) x [0, grid[2]).
+ * grid          : host int32[3] (Z, Y, X) of the input.
+ * feats         : device [n, c] row-major, dtype `dtype`, or NULL (structure
+ *                 only; parent_feats must then be NULL too).
+ * mode          : SMC_POOL_MAX or SMC_POOL_MEAN (sum in fp32 over the children
+ *                 in index order, divided by their count, rounded to nearest
+ *                 even in the output type).
+ * parent_coords : device int32 [n, 4] capacity, 16-byte aligned; receives the
+ *                 m parents' (b, z, y, x) on the grid ((Z+1)/2, (Y+1)/2, (X+1)/2).
+ * parent_feats  : device [n, c] capacity, dtype `dtype`; must not overlap feats.
+ * mask          : device uint8 [n, 8] capacity, 8-byte aligned; receives the
+ *                 subdivision mask: mask[8p + j] = 1 if parent p has the child
+ *                 at index j = dz + 2 dy + 4 dx (z offset fastest), else 0.
+ *                 It is what smc_upsample takes to restore the children.
+ * parent        : device int32 [n] or NULL; receives each row's parent number.
+ * m             : host, receives the number of parents m (1 <= m <= n).
+ * Synchronises `stream` once, at the end, to read m and the error word; all
+ * outputs are complete on return.  Errors: SMC_E_ARG (also n >= 2^30),
+ * SMC_E_ALIGN, SMC_E_DTYPE, SMC_E_SHAPE (c < 1 or above 2^24), SMC_E_ALIAS,
+ * SMC_E_RANGE, SMC_E_DUPLICATE, SMC_E_OOM, SMC_E_CUDA, SMC_E_TIMEOUT; after an
+ * error the outputs are undefined (but every access stayed in bounds).
+ */
+SMC_API int smc_downsample(const int32_t* coords, int64_t n, int32_t batch, const int32_t grid[3],
+                   const void* feats, int64_t c, int32_t dtype, int32_t mode, int32_t* parent_coords,
+                   void* parent_feats, uint8_t* mask, int32_t* parent, int64_t* m, void* stream);
+
+/*
+ * smc_upsample -- masked expansion by 2 (SparseUpsample(2); shared sparse-core
+ * commit log: a voxel emits 0 to 8 children chosen by a 0/1 subdivision mask
+ * whose child index runs with the z offset fastest, the reverse of
+ * smc_subdivide's C order; Pixal3D MLX README, remaining ops).
+ *
+ * coords      : device int32 [n, 4], 16-byte aligned (the coarse voxels).
+ * mask        : device uint8 [n * 8], or NULL (every child): mask[8p + j] != 0
+ *               emits child j of parent p, the site
+ *               (b, 2z + j % 2, 2y + (j / 2) % 2, 2x + j / 4).
+ * feats       : device [n, c], dtype `dtype`, or NULL (coordinates only).
+ * map         : NULL, or the map built from `coords` (same n): then `child`
+ *               receives the children's map on the grid (2Z, 2Y, 2X), read off
+ *               this map without a lookup structure, as smc_subdivide does.
+ * child_coords: device int32 [8n, 4] capacity, 16-byte aligned; receives the
+ *               m children parent by parent, j ascending.
+ * child_feats : device [8n, c] capacity, dtype `dtype` (with feats); child r
+ *               receives its parent's row (nearest upsampling).  Must not
+ *               overlap feats.
+ * m           : host, receives m.
+ * child       : receives the child map (when map is given; may be NULL
+ *               otherwise), as a smc_build_map_async result.
+ * One host synchronisation of `stream` (to read m).  Without a map the
+ * children's coordinates are computed in int32 and not range-checked.
+ * Errors: SMC_E_ARG, SMC_E_ALIGN, SMC_E_DTYPE, SMC_E_SHAPE, SMC_E_ALIAS,
+ * SMC_E_OOM, SMC_E_CUDA, SMC_E_TIMEOUT, or the map's build error.
+ */
+SMC_API int smc_upsample(const int32_t* coords, int64_t n, const uint8_t* mask, const void* feats, int64_t c,
+                 int32_t dtype, const smc_map* map, int32_t* child_coords, void* child_feats, int64_t* m,
+                 void* stream, smc_map** child);
 
 /* Make `stream` wait (on the device, without blocking the host) until the
  * whole build has finished, pair lists included: work enqueued on `stream`

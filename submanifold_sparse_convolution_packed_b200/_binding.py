@@ -31,7 +31,7 @@ EXPORTS = [
     "smc_set_hash_capacity", "smc_set_profiling", "smc_map_timing", "smc_kernel_launches",
     "smc_build_map_async", "smc_map_wait", "smc_neighbour_map_noalloc", "smc_set_conv_variant",
     "smc_set_map_lookup", "smc_map_stream_wait", "smc_subdivide", "smc_conv_ex", "smc_group_stats",
-    "smc_group_norm",
+    "smc_group_norm", "smc_downsample", "smc_upsample",
 ]
 
 
@@ -61,6 +61,8 @@ def lib() -> ctypes.CDLL:
         L.smc_map_wait.argtypes = [P]
         L.smc_map_stream_wait.argtypes = [P, P]
         L.smc_subdivide.argtypes = [P, P, P, P, P, P, P]
+        L.smc_downsample.argtypes = [P, i64, i32, P, P, i64, i32, i32, P, P, P, P, P, P]
+        L.smc_upsample.argtypes = [P, i64, P, P, i64, i32, P, P, P, P, P, P]
         L.smc_conv_ex.argtypes = [P, P, i64, P, P, P, P, i64, i32, i32, i32, i32, P, P, i32, P]
         L.smc_group_stats.argtypes = [P, i64, i64, P, i32, i32, P, i32, P]
         L.smc_group_norm.argtypes = [P, i64, i64, P, i32, i32, P, P, P, ctypes.c_float, i32, P, i32, P]
@@ -260,6 +262,91 @@ def subdivide(parent: "Map", parent_coords: torch.Tensor, keep: Optional[torch.T
                                    _ptr(out), ctypes.byref(m), _stream(stream), ctypes.byref(h)), "smc_subdivide")
     grid = tuple(2 * int(g) for g in parent.grid)
     return out[: m.value], Map(h, int(m.value), parent.batch, grid, parent_coords.device)
+
+
+POOL_MODES = {"max": 0, "mean": 1}
+
+
+def _feats_arg(feats: Optional[torch.Tensor], n: int, device) -> int:
+    if feats is None:
+        return 0
+    if feats.dtype not in _DTYPES or feats.dim() != 2 or feats.shape[0] != n or not feats.is_cuda:
+        raise ValueError("feats must be a float32/bfloat16/float16 [N, C] CUDA tensor")
+    if feats.device != device:
+        raise ValueError("feats must be on the coordinates' device")
+    return _DTYPES[feats.dtype]
+
+
+def downsample(coords: torch.Tensor, grid: Sequence[int], feats: Optional[torch.Tensor] = None,
+               mode: str = "mean", batch: Optional[int] = None, stream=None):
+    """Pool by 2 into parent voxels (smc_downsample in include/smc.h; mode
+    "max" or "mean").  Returns (parent_coords int32 [M, 4], pooled [M, C] or
+    None, subdivision mask uint8 [M, 8], parent of each row int32 [N]);
+    parents are numbered in order of first appearance.  Synchronises the
+    stream once."""
+    if mode not in POOL_MODES:
+        raise ValueError("mode must be 'max' or 'mean'")
+    if coords.dtype != torch.int32 or coords.dim() != 2 or coords.shape[1] != 4 or not coords.is_cuda:
+        raise ValueError("coords must be an int32 [N, 4] CUDA tensor")
+    coords = coords.contiguous()
+    n = coords.shape[0]
+    if batch is None:
+        batch = int(coords[:, 0].max().item()) + 1 if n else 1
+    dt = _feats_arg(feats, n, coords.device)
+    if feats is not None:
+        feats = feats.contiguous()
+    dev = coords.device
+    pc = torch.empty((max(n, 1), 4), dtype=torch.int32, device=dev)
+    mask = torch.empty((max(n, 1), 8), dtype=torch.uint8, device=dev)
+    parent = torch.empty((n,), dtype=torch.int32, device=dev)
+    pooled = None if feats is None else torch.empty((max(n, 1), feats.shape[1]), dtype=feats.dtype, device=dev)
+    m = ctypes.c_int64()
+    g = (ctypes.c_int32 * 3)(*[int(x) for x in grid])
+    with torch.cuda.device(dev):
+        _check(lib().smc_downsample(_ptr(coords), n, int(batch), g, _ptr(feats),
+                                    0 if feats is None else feats.shape[1], dt, POOL_MODES[mode], _ptr(pc),
+                                    _ptr(pooled), _ptr(mask), _ptr(parent), ctypes.byref(m), _stream(stream)),
+               "smc_downsample")
+    k = int(m.value)
+    return pc[:k], None if pooled is None else pooled[:k], mask[:k], parent
+
+
+def upsample(coords: torch.Tensor, mask: Optional[torch.Tensor], feats: Optional[torch.Tensor] = None,
+             parent: Optional["Map"] = None, stream=None):
+    """Masked expansion by 2 (smc_upsample in include/smc.h): child j of
+    voxel p, at offset (j % 2, j // 2 % 2, j // 4) along (z, y, x), where
+    mask[p, j] != 0 (every child when mask is None), carrying p's features.
+    Returns (child_coords int32 [M, 4], child feats [M, C] or None, child Map
+    or None); the child map is built from `parent`, the map of `coords`, when
+    it is given."""
+    if coords.dtype != torch.int32 or coords.dim() != 2 or coords.shape[1] != 4 or not coords.is_cuda:
+        raise ValueError("coords must be an int32 [N, 4] CUDA tensor")
+    coords = coords.contiguous()
+    n = coords.shape[0]
+    if mask is not None:
+        if mask.dtype not in (torch.uint8, torch.bool) or mask.numel() != 8 * n or not mask.is_cuda:
+            raise ValueError("mask must be a uint8/bool CUDA tensor of N * 8 entries")
+        mask = mask.contiguous().view(torch.uint8)
+    dt = _feats_arg(feats, n, coords.device)
+    if feats is not None:
+        feats = feats.contiguous()
+    if parent is not None and parent.n != n:
+        raise ValueError("parent map must be the map of coords")
+    dev = coords.device
+    out = torch.empty((max(8 * n, 1), 4), dtype=torch.int32, device=dev)
+    kf = None if feats is None else torch.empty((max(8 * n, 1), feats.shape[1]), dtype=feats.dtype, device=dev)
+    m = ctypes.c_int64()
+    h = ctypes.c_void_p()
+    with torch.cuda.device(dev):
+        _check(lib().smc_upsample(_ptr(coords), n, _ptr(mask), _ptr(feats), 0 if feats is None else feats.shape[1],
+                                  dt, None if parent is None else parent.handle, _ptr(out), _ptr(kf),
+                                  ctypes.byref(m), _stream(stream), ctypes.byref(h) if parent is not None else None),
+               "smc_upsample")
+    k = int(m.value)
+    cm = None
+    if parent is not None:
+        cm = Map(h, k, parent.batch, tuple(2 * int(x) for x in parent.grid), dev)
+    return out[:k], None if kf is None else kf[:k], cm
 
 
 NOALLOC_MAX_N = 1 << 18

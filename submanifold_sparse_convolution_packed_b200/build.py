@@ -15,7 +15,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsmc.so")
-SOURCES = ["api.cu", "map_build.cu", "conv_simt.cu", "conv_tc.cu", "conv_offsets.cu", "norm.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "map_build.cu", "conv_simt.cu", "conv_tc.cu", "conv_offsets.cu", "norm.cu", "resample.cu",
+           "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

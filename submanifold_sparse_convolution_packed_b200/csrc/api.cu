@@ -560,30 +560,30 @@ int smc_map_wait(const smc_map* map) {
   return resolve(map);
 }
 
-int smc_subdivide(const smc_map* parent, const int32_t* parent_coords, const uint8_t* keep, int32_t* child_coords,
-                  int64_t* m_out, void* stream, smc_map** child) {
-  if (!child || !m_out) return SMC_E_ARG;
-  *child = nullptr;
-  *m_out = 0;
-  if (!parent) return SMC_E_ARG;
-  const int64_t n = parent->n;
-  if (n > 0 && (!parent_coords || !child_coords)) return SMC_E_ARG;
-  if (n > 0 && ((reinterpret_cast<uintptr_t>(parent_coords) & 15u) || (reinterpret_cast<uintptr_t>(child_coords) & 15u)))
-    return SMC_E_ALIGN;
-  int32_t grid2[3];
-  for (int i = 0; i < 3; ++i) {
-    if (parent->grid[i] > (1 << 30) - 1) return SMC_E_ARG;
-    grid2[i] = 2 * parent->grid[i];
+// Children of n parent rows (smc_subdivide, smc_upsample): per-parent child
+// bits and counts, their scan, one host read of the total m, the children's
+// coordinates in (parent, k) order (`order` as in launch_subdiv_emit), then
+// the rows of `feats` copied to the children (when feats is given) and the
+// children's map read off the parent map (when parent is given).
+static int spawn_children(const smc_map* parent, const int32_t* coords, int64_t n, const uint8_t* keep, int order,
+                   const void* feats, int64_t row_bytes, int elem_bytes, void* child_feats, int32_t* child_coords,
+                   int64_t* m_out, cudaStream_t s, smc_map** child) {
+  int32_t grid2[3] = {1, 1, 1};
+  if (parent) {
+    for (int i = 0; i < 3; ++i) {
+      if (parent->grid[i] > (1 << 30) - 1) return SMC_E_ARG;
+      grid2[i] = 2 * parent->grid[i];
+    }
+    const int rc = resolve(parent);  // the parent map must be complete (and sound)
+    if (rc != SMC_OK) return rc;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev != parent->device) return SMC_E_ARG;
   }
-  if (8 * n >= (1ll << 31) - 1) return SMC_E_ARG;  // child rows and parent slots are int32
-  const int rc = resolve(parent);  // the parent map must be complete (and sound)
-  if (rc != SMC_OK) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (n == 0) return parent ? build_async(nullptr, 0, parent->batch, grid2, s, child) : SMC_OK;
+  if (pending_cuda_error() != SMC_OK) return SMC_E_CUDA;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev != parent->device) return SMC_E_ARG;
-  if (n == 0) return build_async(nullptr, 0, parent->batch, grid2, s, child);
-  if (pending_cuda_error() != SMC_OK) return SMC_E_CUDA;
   cudaMemPool_t pool = device_pool(dev);
   HostSlot* slot = take_slot();
   if (!pool || !slot) {
@@ -618,7 +618,7 @@ int smc_subdivide(const smc_map* parent, const int32_t* parent_coords, const uin
   int32_t* src = reinterpret_cast<int32_t*>(S + o_src);
   // children per parent, then their first row; the total comes back to size the child map
   cudaError_t ce = cudaMemsetAsync(S + o_hdr, 0, zero_bytes, s);
-  if (ce == cudaSuccess) ce = smc::launch_subdiv_count(keep, n, bits, cnt, s);
+  if (ce == cudaSuccess) ce = smc::launch_subdiv_count(keep, n, order, bits, cnt, s);
   if (ce == cudaSuccess)
     ce = smc::launch_scan_counts(cnt, n, first, reinterpret_cast<unsigned long long*>(S + o_st),
                                  reinterpret_cast<uint32_t*>(S + o_tick), err, info, n, s);
@@ -637,13 +637,15 @@ int smc_subdivide(const smc_map* parent, const int32_t* parent_coords, const uin
     out = SMC_E_CUDA;
   }
   if (out == SMC_OK) {
-    ce = smc::launch_subdiv_emit(parent_coords, n, bits, first, child_coords, src, remap, s);
+    ce = smc::launch_subdiv_emit(coords, n, order, bits, first, child_coords, src, remap, s);
+    if (ce == cudaSuccess && feats)
+      ce = smc::launch_gather_rows(feats, row_bytes, src, m, child_feats, elem_bytes, s);
     if (ce != cudaSuccess) {
       cudaGetLastError();
       out = SMC_E_CUDA;
     }
   }
-  if (out == SMC_OK) {
+  if (out == SMC_OK && parent) {
     const SubdivSource sub{parent->nbr, src, remap};
     out = build_async(child_coords, m, parent->batch, grid2, s, child, &sub);
   }
@@ -651,6 +653,161 @@ int smc_subdivide(const smc_map* parent, const int32_t* parent_coords, const uin
   cudaGetLastError();
   if (out == SMC_OK) *m_out = m;
   return out;
+}
+
+int smc_subdivide(const smc_map* parent, const int32_t* parent_coords, const uint8_t* keep, int32_t* child_coords,
+                  int64_t* m_out, void* stream, smc_map** child) {
+  if (!child || !m_out) return SMC_E_ARG;
+  *child = nullptr;
+  *m_out = 0;
+  if (!parent) return SMC_E_ARG;
+  const int64_t n = parent->n;
+  if (n > 0 && (!parent_coords || !child_coords)) return SMC_E_ARG;
+  if (n > 0 && ((reinterpret_cast<uintptr_t>(parent_coords) & 15u) || (reinterpret_cast<uintptr_t>(child_coords) & 15u)))
+    return SMC_E_ALIGN;
+  if (8 * n >= (1ll << 31) - 1) return SMC_E_ARG;  // child rows and parent slots are int32
+  return spawn_children(parent, parent_coords, n, keep, 0, nullptr, 0, 0, nullptr, child_coords, m_out,
+                        static_cast<cudaStream_t>(stream), child);
+}
+
+int smc_upsample(const int32_t* coords, int64_t n, const uint8_t* mask, const void* feats, int64_t c, int32_t dtype,
+                 const smc_map* map, int32_t* child_coords, void* child_feats, int64_t* m_out, void* stream,
+                 smc_map** child) {
+  if (!m_out) return SMC_E_ARG;
+  *m_out = 0;
+  if (child) *child = nullptr;
+  if (map && !child) return SMC_E_ARG;
+  if (n < 0 || (map && map->n != n)) return SMC_E_ARG;
+  if (8 * n >= (1ll << 31) - 1) return SMC_E_ARG;  // child rows and parent slots are int32
+  int es = 0;
+  if (feats) {
+    if (dtype != SMC_F32 && dtype != SMC_BF16 && dtype != SMC_F16) return SMC_E_DTYPE;
+    es = dtype == SMC_F32 ? 4 : 2;
+    if (c < 1 || c > (1 << 24)) return SMC_E_SHAPE;
+    if (n > 0 && !child_feats) return SMC_E_ARG;
+    if ((reinterpret_cast<uintptr_t>(feats) | reinterpret_cast<uintptr_t>(child_feats)) & (es - 1)) return SMC_E_ALIGN;
+    if (n > 0 && ranges_overlap(feats, static_cast<size_t>(n) * c * es, child_feats, 8ull * n * c * es))
+      return SMC_E_ALIAS;
+  }
+  if (n > 0 && (!coords || !child_coords)) return SMC_E_ARG;
+  if (n > 0 && ((reinterpret_cast<uintptr_t>(coords) & 15u) || (reinterpret_cast<uintptr_t>(child_coords) & 15u)))
+    return SMC_E_ALIGN;
+  return spawn_children(map, coords, n, mask, 1, feats, feats ? c * es : 0, es, child_feats, child_coords, m_out,
+                        static_cast<cudaStream_t>(stream), child);
+}
+
+int smc_downsample(const int32_t* coords, int64_t n, int32_t batch, const int32_t grid[3], const void* feats,
+                   int64_t c, int32_t dtype, int32_t mode, int32_t* parent_coords, void* parent_feats,
+                   uint8_t* mask, int32_t* parent, int64_t* m_out, void* stream) {
+  if (!m_out) return SMC_E_ARG;
+  *m_out = 0;
+  if (!grid || n < 0 || batch < 1 || grid[0] < 1 || grid[1] < 1 || grid[2] < 1) return SMC_E_ARG;
+  if (mode != SMC_POOL_MAX && mode != SMC_POOL_MEAN) return SMC_E_ARG;
+  if (n >= (1ll << 30)) return SMC_E_ARG;  // rows are int32, hash slots below 2^31
+  if (n == 0) return SMC_OK;
+  if ((feats == nullptr) != (parent_feats == nullptr)) return SMC_E_ARG;
+  int es = 0;
+  if (feats) {
+    if (dtype != SMC_F32 && dtype != SMC_BF16 && dtype != SMC_F16) return SMC_E_DTYPE;
+    es = dtype == SMC_F32 ? 4 : 2;
+    if (c < 1 || c > (1 << 24)) return SMC_E_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(feats) | reinterpret_cast<uintptr_t>(parent_feats)) & (es - 1))
+      return SMC_E_ALIGN;
+    if (n > 0 && ranges_overlap(feats, static_cast<size_t>(n) * c * es, parent_feats, static_cast<size_t>(n) * c * es))
+      return SMC_E_ALIAS;
+  }
+  if (!coords || !parent_coords || !mask) return SMC_E_ARG;
+  if ((reinterpret_cast<uintptr_t>(coords) & 15u) || (reinterpret_cast<uintptr_t>(parent_coords) & 15u) ||
+      (reinterpret_cast<uintptr_t>(mask) & 7u) || (reinterpret_cast<uintptr_t>(parent) & 3u))
+    return SMC_E_ALIGN;
+  const double psites = static_cast<double>(batch) * ((grid[0] + 1) / 2) * ((grid[1] + 1) / 2) * ((grid[2] + 1) / 2);
+  if (psites >= 4.6e18) return SMC_E_ARG;
+  if (pending_cuda_error() != SMC_OK) return SMC_E_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaMemPool_t pool = device_pool(dev);
+  HostSlot* slot = take_slot();
+  if (!pool || !slot) {
+    give_slot(slot);
+    return SMC_E_OOM;
+  }
+  // Parent lookup: a dense grid over the parent box (8 bytes a site) when it
+  // holds at most 32 sites per row and 2^28 sites, else a hash at load <= 1/2.
+  const int lookup = g_map_lookup.load();
+  const bool dense = psites <= kDenseMaxSites && (lookup == 2 || (lookup == 0 && psites <= 32.0 * n));
+  int lg = 4;
+  while ((1ll << lg) < 2 * n) ++lg;
+  const size_t slots = dense ? static_cast<size_t>(psites) : (size_t(1) << lg);
+  Carve cv;
+  const size_t o_hdr = cv.take<HostSlot>(1);
+  const size_t o_tick = cv.take<uint32_t>(1);
+  const size_t o_st = cv.take<unsigned long long>(smc::scan_status_len(n));
+  const size_t o_bits = cv.take<uint32_t>(slots);
+  const size_t zero_bytes = cv.off - o_hdr;
+  const size_t o_first = cv.take<int32_t>(slots);
+  const size_t o_keys = dense ? 0 : cv.take<unsigned long long>(slots);
+  const size_t o_sor = cv.take<uint32_t>(n);
+  const size_t o_flags = cv.take<int32_t>(n);
+  const size_t o_pos = cv.take<int64_t>(n);
+  const size_t o_rows = cv.take<int32_t>(8 * n);
+  const size_t o_pbits = cv.take<uint8_t>(n);
+  void* sp = nullptr;
+  if (cudaMallocFromPoolAsync(&sp, cv.off, pool, s) != cudaSuccess) {
+    cudaGetLastError();
+    give_slot(slot);
+    return SMC_E_OOM;
+  }
+  char* S = static_cast<char*>(sp);
+  smc::DownArgs a{};
+  a.coords = coords;
+  a.n = n;
+  a.batch = batch;
+  a.Z = grid[0];
+  a.Y = grid[1];
+  a.X = grid[2];
+  a.keys = dense ? nullptr : reinterpret_cast<unsigned long long*>(S + o_keys);
+  a.lg = lg;
+  a.first = reinterpret_cast<int32_t*>(S + o_first);
+  a.bits = reinterpret_cast<uint32_t*>(S + o_bits);
+  a.slot_of_row = reinterpret_cast<uint32_t*>(S + o_sor);
+  a.flags = reinterpret_cast<int32_t*>(S + o_flags);
+  a.pos = reinterpret_cast<int64_t*>(S + o_pos);
+  a.scan_status = reinterpret_cast<unsigned long long*>(S + o_st);
+  a.scan_ticket = reinterpret_cast<uint32_t*>(S + o_tick);
+  a.err = reinterpret_cast<uint32_t*>(S + o_hdr + offsetof(HostSlot, err));
+  a.info = reinterpret_cast<int64_t*>(S + o_hdr + offsetof(HostSlot, info));
+  a.child_rows = reinterpret_cast<int32_t*>(S + o_rows);
+  a.pbits = reinterpret_cast<uint8_t*>(S + o_pbits);
+  a.parent_coords = parent_coords;
+  a.mask = mask;
+  a.parent = parent;
+  a.feats = feats;
+  a.out = parent_feats;
+  a.c = static_cast<int>(c);
+  a.dtype = dtype;
+  a.mode = mode;
+  cudaError_t ce = cudaMemsetAsync(S + o_hdr, 0, zero_bytes, s);
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(a.first, 0x7F, slots * sizeof(int32_t), s);
+  if (ce == cudaSuccess && !dense) ce = cudaMemsetAsync(a.keys, 0xFF, slots * sizeof(unsigned long long), s);
+  if (ce == cudaSuccess) ce = smc::launch_downsample(a, s);
+  if (ce == cudaSuccess) ce = cudaMemcpyAsync(slot, S + o_hdr, sizeof(HostSlot), cudaMemcpyDeviceToHost, s);
+  if (ce == cudaSuccess) ce = cudaStreamSynchronize(s);
+  const uint32_t e = slot->err;
+  const int64_t m = slot->info[27];
+  give_slot(slot);
+  cudaFreeAsync(sp, s);
+  if (ce != cudaSuccess) {
+    cudaGetLastError();
+    return SMC_E_CUDA;
+  }
+  if (e & smc::kErrRange) return SMC_E_RANGE;
+  if (e & smc::kErrDuplicate) return SMC_E_DUPLICATE;
+  if (e & smc::kErrCapacity) return SMC_E_CAPACITY;
+  if (e & smc::kErrTimeout) return SMC_E_TIMEOUT;
+  if (m < 1 || m > n) return SMC_E_CUDA;
+  *m_out = m;
+  return SMC_OK;
 }
 
 int smc_group_stats(const void* x, int64_t n, int64_t c, const int32_t* coords, int32_t batch, int32_t groups,

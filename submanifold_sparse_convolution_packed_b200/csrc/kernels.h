@@ -75,11 +75,48 @@ cudaError_t launch_scan_counts(const int32_t* in, int64_t L, int64_t* out, unsig
 // Subdivision: children per parent (bit mask and count), the children's
 // coordinates with their (parent, octant) and the parent-slot -> child-row
 // remap, then the children's map rows from the parent map.
-cudaError_t launch_subdiv_count(const uint8_t* keep, int64_t n, uint8_t* bits, int32_t* cnt, cudaStream_t s);
-cudaError_t launch_subdiv_emit(const int32_t* coords, int64_t n, const uint8_t* bits, const int64_t* first,
-                               int32_t* child_coords, int32_t* child_src, int32_t* remap, cudaStream_t s);
+// `order` numbers the children and lists them: 0 = C-order octant
+// o = 4a + 2c + e (subdivide), 1 = the upsample mask's index
+// j = a + 2c + 4e (z offset fastest).  child_src always holds 8 * parent + o.
+cudaError_t launch_subdiv_count(const uint8_t* keep, int64_t n, int order, uint8_t* bits, int32_t* cnt,
+                                cudaStream_t s);
+cudaError_t launch_subdiv_emit(const int32_t* coords, int64_t n, int order, const uint8_t* bits,
+                               const int64_t* first, int32_t* child_coords, int32_t* child_src, int32_t* remap,
+                               cudaStream_t s);
 cudaError_t launch_subdiv_lookups(const MapBuildArgs& a, const int32_t* parent_nbr, const int32_t* child_src,
                                   const int32_t* remap, cudaStream_t s);
+
+// Downsample by 2 (resample.cu): parents numbered in order of first
+// appearance, their coordinates, subdivision mask, each row's parent, and the
+// pooled features.
+struct DownArgs {
+  const int32_t* coords;  // [n, 4] (b, z, y, x)
+  int64_t n;
+  int32_t batch, Z, Y, X;
+  unsigned long long* keys;  // hash: 2^lg parent keys pre-filled with ~0; null: dense parent grid
+  int lg;
+  int32_t* first;          // per slot, pre-filled with 0x7F7F7F7F: smallest row of the parent
+  uint32_t* bits;          // per slot, zeroed: children present (bit j)
+  uint32_t* slot_of_row;   // [n]
+  int32_t* flags;          // [n]
+  int64_t* pos;            // [n]
+  unsigned long long* scan_status;  // [scan_status_len(n)], zeroed
+  uint32_t* scan_ticket;   // zeroed
+  uint32_t* err;           // error bits, zeroed
+  int64_t* info;           // [28]: info[27] receives the parent count M
+  int32_t* child_rows;     // [8 n]: row of child j of parent p at 8 p + j (where present)
+  uint8_t* pbits;          // [n]: children present per parent
+  int32_t* parent_coords;  // [n, 4] capacity
+  uint8_t* mask;           // [n, 8] capacity, 8-byte aligned
+  int32_t* parent;         // [n] or null
+  const void* feats;       // [n, c] or null (no pooling)
+  void* out;               // [n, c] capacity
+  int c, dtype, mode;      // mode 0 max, 1 mean
+};
+cudaError_t launch_downsample(const DownArgs& a, cudaStream_t s);
+// out[r] = rows[src[r] >> 3] for r < m, rows of row_bytes bytes of elem_bytes-byte elements.
+cudaError_t launch_gather_rows(const void* rows, int64_t row_bytes, const int32_t* src, int64_t m, void* out,
+                               int elem_bytes, cudaStream_t s);
 
 // GroupNorm over a sparse tensor (norm.cu): statistics of x per (batch item,
 // channel group) added into stats [batch, groups, 3], and the normalisation

@@ -302,9 +302,14 @@ __global__ void __launch_bounds__(kMapBlock) k_neighbours(
 }
 
 // ------------------------------------------------------------ subdivision
-// The children of parent row v are the sites (b, 2z+a, 2y+c, 2x+e) of octant
-// o = 4a + 2c + e (C order), kept where keep[8v+o] is nonzero (all when keep
-// is null) and numbered in (parent row, octant) order.
+// The children of parent row v are the sites (b, 2z+a, 2y+c, 2x+e), kept
+// where keep[8v + k] is nonzero (all when keep is null) and numbered in
+// (parent row, k) order, where k is the octant o = 4a + 2c + e (C order,
+// subdivide) or, for order 1, the upsample mask's index j = a + 2c + 4e.
+__device__ __forceinline__ int octant_of(int k, int order) {
+  return order ? ((k & 1) << 2) | (k & 2) | ((k >> 2) & 1) : k;
+}
+
 __global__ void k_subdiv_count(const uint8_t* __restrict__ keep, int64_t n, uint8_t* __restrict__ bits,
                                int32_t* __restrict__ cnt) {
   for (int64_t v = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; v < n;
@@ -313,14 +318,14 @@ __global__ void k_subdiv_count(const uint8_t* __restrict__ keep, int64_t n, uint
     if (keep) {
       b = 0;
 #pragma unroll
-      for (int o = 0; o < 8; ++o) b |= static_cast<uint32_t>(keep[8 * v + o] != 0) << o;
+      for (int k = 0; k < 8; ++k) b |= static_cast<uint32_t>(keep[8 * v + k] != 0) << k;
     }
     bits[v] = static_cast<uint8_t>(b);
     cnt[v] = __popc(b);
   }
 }
 
-__global__ void k_subdiv_emit(const int4* __restrict__ coords, int64_t n, const uint8_t* __restrict__ bits,
+__global__ void k_subdiv_emit(const int4* __restrict__ coords, int64_t n, int order, const uint8_t* __restrict__ bits,
                               const int64_t* __restrict__ first, int4* __restrict__ child_coords,
                               int32_t* __restrict__ child_src, int32_t* __restrict__ remap) {
   for (int64_t v = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; v < n;
@@ -329,8 +334,9 @@ __global__ void k_subdiv_emit(const int4* __restrict__ coords, int64_t n, const 
     const uint32_t b = bits[v];
     int64_t r = first[v];
 #pragma unroll
-    for (int o = 0; o < 8; ++o) {
-      if ((b >> o) & 1u) {
+    for (int k = 0; k < 8; ++k) {
+      const int o = octant_of(k, order);
+      if ((b >> k) & 1u) {
         child_coords[r] = make_int4(c.x, 2 * c.y + (o >> 2), 2 * c.z + ((o >> 1) & 1), 2 * c.w + (o & 1));
         child_src[r] = static_cast<int32_t>(8 * v + o);
         remap[8 * v + o] = static_cast<int32_t>(r);
@@ -711,7 +717,9 @@ cudaError_t launch_scan_counts(const int32_t* in, int64_t L, int64_t* out, unsig
   return scan_i32(in, L, out, status, ticket, err, info, stride, s);
 }
 
-cudaError_t launch_subdiv_count(const uint8_t* keep, int64_t n, uint8_t* bits, int32_t* cnt, cudaStream_t s) {
+cudaError_t launch_subdiv_count(const uint8_t* keep, int64_t n, int order, uint8_t* bits, int32_t* cnt,
+                                cudaStream_t s) {
+  (void)order;  // the mask's bit k is child k in either numbering
   if (n == 0) return cudaSuccess;
   const int64_t blocks = (n + 255) / 256;
   k_subdiv_count<<<static_cast<unsigned>(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, s>>>(keep, n, bits, cnt);
@@ -719,12 +727,13 @@ cudaError_t launch_subdiv_count(const uint8_t* keep, int64_t n, uint8_t* bits, i
   return cudaGetLastError();
 }
 
-cudaError_t launch_subdiv_emit(const int32_t* coords, int64_t n, const uint8_t* bits, const int64_t* first,
-                               int32_t* child_coords, int32_t* child_src, int32_t* remap, cudaStream_t s) {
+cudaError_t launch_subdiv_emit(const int32_t* coords, int64_t n, int order, const uint8_t* bits,
+                               const int64_t* first, int32_t* child_coords, int32_t* child_src, int32_t* remap,
+                               cudaStream_t s) {
   if (n == 0) return cudaSuccess;
   const int64_t blocks = (n + 255) / 256;
   k_subdiv_emit<<<static_cast<unsigned>(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, s>>>(
-      reinterpret_cast<const int4*>(coords), n, bits, first, reinterpret_cast<int4*>(child_coords), child_src,
+      reinterpret_cast<const int4*>(coords), n, order, bits, first, reinterpret_cast<int4*>(child_coords), child_src,
       remap);
   count_launches(1);
   return cudaGetLastError();

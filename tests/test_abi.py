@@ -55,3 +55,30 @@ def test_argument_errors_without_gpu():
     assert h.value is None
     assert lib.smc_conv(None, None, 1, None, None, None, 1, 3, 1, 0, None) == -1
     assert lib.smc_free_map(None) == 0
+
+
+def test_resample_argument_errors_without_gpu():
+    import ctypes
+    lib = smc.lib()
+    m = ctypes.c_int64(7)
+    grid = (ctypes.c_int32 * 3)(4, 4, 4)
+    P = ctypes.c_void_p
+    a16 = P(16)
+    # downsample: no m, bad mode, feats without an output, bad dtype, misaligned coords
+    assert lib.smc_downsample(None, 1, 1, grid, None, 0, 0, 0, None, None, None, None, None, None) == -1
+    assert lib.smc_downsample(a16, 1, 1, grid, None, 0, 0, 2, a16, None, a16, None, ctypes.byref(m), None) == -1
+    assert m.value == 0
+    assert lib.smc_downsample(a16, 1, 1, grid, a16, 4, 0, 0, a16, None, a16, None, ctypes.byref(m), None) == -1
+    assert lib.smc_downsample(a16, 1, 1, grid, a16, 4, 7, 0, a16, P(4096), a16, None, ctypes.byref(m), None) == -4
+    assert lib.smc_downsample(P(8), 1, 1, grid, None, 0, 0, 0, a16, None, a16, None, ctypes.byref(m), None) == -11
+    assert lib.smc_downsample(a16, 1, 0, grid, None, 0, 0, 0, a16, None, a16, None, ctypes.byref(m), None) == -1
+    assert lib.smc_downsample(None, 0, 1, grid, None, 0, 0, 1, None, None, None, None, ctypes.byref(m), None) == 0
+    # pooled output overlapping the input
+    assert lib.smc_downsample(a16, 4, 1, grid, P(4096), 8, 0, 0, a16, P(4096 + 64), a16, None,
+                              ctypes.byref(m), None) == -6
+    # upsample: no m, a map without somewhere to put the child map, bad dtype, misaligned coords
+    assert lib.smc_upsample(a16, 1, None, None, 0, 0, None, a16, None, None, None, None) == -1
+    assert lib.smc_upsample(a16, 1, None, None, 0, 0, P(64), a16, None, ctypes.byref(m), None, None) == -1
+    assert lib.smc_upsample(a16, 1, None, a16, 4, 9, None, a16, P(4096), ctypes.byref(m), None, None) == -4
+    assert lib.smc_upsample(P(4), 1, None, None, 0, 0, None, a16, None, ctypes.byref(m), None, None) == -11
+    assert lib.smc_upsample(None, 0, None, None, 0, 0, None, None, None, ctypes.byref(m), None, None) == 0

@@ -619,3 +619,152 @@ def test_async_build_reports_errors_late():
     assert e.value.name == "SMC_E_DUPLICATE"
     m.free()
     smc.status()
+
+
+# ------------------------------------------------------------------ downsample / upsample
+def _shuffled(w, seed):
+    """The workload's rows in a seeded random order, so that first-appearance
+    numbering differs from any sorted order."""
+    perm = np.random.default_rng(seed).permutation(w.n)
+    return np.ascontiguousarray(w.coords[perm])
+
+
+def _pool_ref_check(got, ref, dtype, mode, what):
+    if mode == "max":  # one of the inputs, exactly
+        np.testing.assert_array_equal(got, S.round_to(ref, dtype).astype(np.float64), err_msg=what)
+    else:
+        check_close(got, ref, dtype, what)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("mode", ["max", "mean"])
+@pytest.mark.parametrize("c", [128, 3])
+def test_downsample_matches_oracle(oracle_mod, map_lookup, dtype, mode, c):
+    """Two-item shell workload in shuffled row order: parent coordinates,
+    subdivision mask and parent of each row bit-exact; max pooling exact, mean
+    within the dtype's bar (16-byte vector path at 128 channels, scalar at 3)."""
+    w = workload("shell2")
+    coords = _shuffled(w, 31)
+    f = S.features(w.n, c, np.random.default_rng(32), dtype)
+    pc, pooled, mask, parent = smc.downsample(torch.from_numpy(coords).cuda(), w.grid, dev(f, dtype), mode, batch=2)
+    rpc, rpooled, rmask, rparent = oracle_mod.downsample(coords, w.grid, f, oracle_mod.POOL_MAX if mode == "max"
+                                                         else oracle_mod.POOL_MEAN, 2)
+    np.testing.assert_array_equal(pc.cpu().numpy(), rpc)
+    np.testing.assert_array_equal(mask.cpu().numpy(), rmask)
+    np.testing.assert_array_equal(parent.cpu().numpy(), rparent)
+    _pool_ref_check(host(pooled), rpooled, dtype, mode, f"{mode} pooling")
+    smc.status()
+
+
+def test_downsample_full128_sampled(oracle_mod):
+    """The 128^3 full grid (2,097,152 rows, bf16, 128 channels), shuffled:
+    structure bit-exact against the oracle, pooled features (max and mean)
+    checked on 2048 sampled parents, each recomputed by the oracle from just
+    its own children."""
+    w = workload("full128")
+    coords = _shuffled(w, 33)
+    f = S.features(w.n, 128, np.random.default_rng(34), "bf16")
+    ct, ft = torch.from_numpy(coords).cuda(), dev(f, "bf16")
+    rpc, _, rmask, rparent = oracle_mod.downsample(coords, w.grid)
+    rows_of = None
+    for mode in ("max", "mean"):
+        pc, pooled, mask, parent = smc.downsample(ct, w.grid, ft, mode, batch=1)
+        np.testing.assert_array_equal(pc.cpu().numpy(), rpc)
+        np.testing.assert_array_equal(mask.cpu().numpy(), rmask)
+        np.testing.assert_array_equal(parent.cpu().numpy(), rparent)
+        ps = sample_rows(len(rpc), 2048, 35)
+        if rows_of is None:
+            rows_of = np.flatnonzero(np.isin(rparent, ps))
+        spc, sp, _, _ = oracle_mod.downsample(coords[rows_of], w.grid, f[rows_of],
+                                              oracle_mod.POOL_MAX if mode == "max" else oracle_mod.POOL_MEAN, 1)
+        # the subset's parents are the sampled parents, in the same relative order
+        np.testing.assert_array_equal(spc, rpc[ps])
+        _pool_ref_check(host(pooled)[ps], sp, "bf16", mode, f"{mode} pooling, sampled parents")
+    smc.status()
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("with_map", [False, True], ids=["no_map", "child_map"])
+def test_upsample_matches_oracle(oracle_mod, dtype, with_map):
+    """Masked expansion of the shell workload with a random mask: children's
+    coordinates (parent by parent, z-fastest index ascending) and features
+    bit-exact; with the parent's map, the children's map, pair lists and
+    schedule bit-exact against a map the oracle builds from scratch."""
+    w = workload("shell2")
+    mask = (np.random.default_rng(36).random((w.n, 8)) < 0.4).astype(np.uint8)
+    c = 128 if dtype != "f32" else 5
+    f = S.features(w.n, c, np.random.default_rng(37), dtype)
+    ct = torch.from_numpy(w.coords).cuda()
+    parent = build(w) if with_map else None
+    kids, kf, child = smc.upsample(ct, torch.from_numpy(mask).cuda(), dev(f, dtype), parent=parent)
+    rk, rf = oracle_mod.upsample(w.coords, mask, f)
+    np.testing.assert_array_equal(kids.cpu().numpy(), rk)
+    np.testing.assert_array_equal(host(kf), rf)
+    if with_map:
+        grid2 = tuple(2 * g for g in w.grid)
+        assert child.n == len(rk) and child.grid == grid2
+        ref = oracle_mod.neighbour_map(rk, grid2)
+        np.testing.assert_array_equal(child.nbr().cpu().numpy(), ref)
+        counts, _, in_idx, out_idx = oracle_mod.pair_lists(ref)
+        gi, go, _ = child.pairs()
+        np.testing.assert_array_equal(gi.cpu().numpy(), in_idx)
+        np.testing.assert_array_equal(go.cpu().numpy(), out_idx)
+        np.testing.assert_array_equal(child.schedule().cpu().numpy(), expected_schedule(ref))
+    else:
+        assert child is None
+    smc.status()
+
+
+def test_downsample_upsample_round_trip_gpu(oracle_mod):
+    """Downsample the shuffled shell workload, build the parents' map, then
+    upsample with the recorded mask: the children are the input sites again,
+    their map is exact, and a conv over it meets the bf16 bar."""
+    w = workload("shell2")
+    coords = _shuffled(w, 38)
+    pc, _, mask, _ = smc.downsample(torch.from_numpy(coords).cuda(), w.grid, None, "max", batch=2)
+    half = tuple((g + 1) // 2 for g in w.grid)
+    pm = smc.build_map(pc, half, batch=2)
+    kids, _, child = smc.upsample(pc, mask, None, parent=pm)
+    got = kids.cpu().numpy()
+    assert sorted(map(tuple, got.tolist())) == sorted(map(tuple, coords.tolist()))
+    rk, _ = oracle_mod.upsample(pc.cpu().numpy(), mask.cpu().numpy())
+    np.testing.assert_array_equal(got, rk)
+    grid2 = tuple(2 * g for g in half)
+    np.testing.assert_array_equal(child.nbr().cpu().numpy(), oracle_mod.neighbour_map(rk, grid2))
+    sub = S.Workload("round_trip", rk, grid2, 64, 64, ("bf16",))
+    f, wt, b = _layer(sub, "bf16")
+    rows = sample_rows(sub.n, 2048, 39)
+    out = smc.conv(child, dev(f, "bf16"), dev(wt, "bf16"), dev(b, "bf16"))
+    ref = oracle_mod.conv(rk, grid2, f, wt, b, 3, 1, rows=rows, threads=THREADS)
+    check_close(host(out)[rows], ref, "bf16", "conv on the upsampled map")
+    smc.status()
+
+
+def test_resample_errors_and_edges(oracle_mod, map_lookup):
+    d = "cuda"
+    dup = torch.tensor([[0, 1, 1, 1], [0, 2, 2, 2], [0, 1, 1, 1]], dtype=torch.int32, device=d)
+    with pytest.raises(smc.SmcError) as e:
+        smc.downsample(dup, (4, 4, 4), batch=1)
+    assert e.value.name == "SMC_E_DUPLICATE"
+    far = torch.tensor([[0, 1, 1, 1], [0, 1, 4, 1]], dtype=torch.int32, device=d)
+    with pytest.raises(smc.SmcError) as e:
+        smc.downsample(far, (4, 4, 4), torch.ones((2, 8), device=d), batch=1)
+    assert e.value.name == "SMC_E_RANGE"
+    empty = torch.zeros((0, 4), dtype=torch.int32, device=d)
+    pc, pooled, mask, parent = smc.downsample(empty, (4, 4, 4), torch.zeros((0, 8), device=d), "mean", batch=1)
+    assert pc.shape == (0, 4) and pooled.shape == (0, 8) and mask.shape == (0, 8) and parent.shape == (0,)
+    kids, kf, child = smc.upsample(empty, None, torch.zeros((0, 8), device=d))
+    assert kids.shape == (0, 4) and kf.shape == (0, 8) and child is None
+    # odd extents: the last window is partial; one voxel per parent keeps its features
+    one = torch.tensor([[0, 4, 1, 0], [1, 0, 0, 6]], dtype=torch.int32, device=d)
+    x = torch.tensor([[1.5, -2.0], [3.0, 4.25]], device=d)
+    pc, pooled, mask, _ = smc.downsample(one, (5, 3, 7), x, "mean", batch=2)
+    assert pc.tolist() == [[0, 2, 0, 0], [1, 0, 0, 3]]
+    assert pooled.tolist() == x.tolist()
+    assert mask.tolist() == [[0, 0, 1, 0, 0, 0, 0, 0], [1, 0, 0, 0, 0, 0, 0, 0]]
+    # a mask of all zeros emits nothing; a null mask emits all eight
+    kids, _, _ = smc.upsample(pc, torch.zeros_like(mask))
+    assert kids.shape == (0, 4)
+    kids, _, _ = smc.upsample(pc, None)
+    np.testing.assert_array_equal(kids.cpu().numpy(), oracle_mod.upsample(pc.cpu().numpy(), np.ones((2, 8)))[0])
+    smc.status()
