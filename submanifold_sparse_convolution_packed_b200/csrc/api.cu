@@ -639,7 +639,7 @@ static int spawn_children(const smc_map* parent, const int32_t* coords, int64_t 
   if (out == SMC_OK) {
     ce = smc::launch_subdiv_emit(coords, n, order, bits, first, child_coords, src, remap, s);
     if (ce == cudaSuccess && feats)
-      ce = smc::launch_gather_rows(feats, row_bytes, src, m, child_feats, elem_bytes, s);
+      ce = smc::launch_expand_rows(feats, row_bytes, first, bits, n, child_feats, elem_bytes, s);
     if (ce != cudaSuccess) {
       cudaGetLastError();
       out = SMC_E_CUDA;

@@ -114,9 +114,10 @@ struct DownArgs {
   int c, dtype, mode;      // mode 0 max, 1 mean
 };
 cudaError_t launch_downsample(const DownArgs& a, cudaStream_t s);
-// out[r] = rows[src[r] >> 3] for r < m, rows of row_bytes bytes of elem_bytes-byte elements.
-cudaError_t launch_gather_rows(const void* rows, int64_t row_bytes, const int32_t* src, int64_t m, void* out,
-                               int elem_bytes, cudaStream_t s);
+// Row p of `rows` (row_bytes bytes of elem_bytes-byte elements) copied to
+// output rows first[p] .. first[p] + popc(bits[p]) - 1, for p < n.
+cudaError_t launch_expand_rows(const void* rows, int64_t row_bytes, const int64_t* first, const uint8_t* bits,
+                               int64_t n, void* out, int elem_bytes, cudaStream_t s);
 
 // GroupNorm over a sparse tensor (norm.cu): statistics of x per (batch item,
 // channel group) added into stats [batch, groups, 3], and the normalisation

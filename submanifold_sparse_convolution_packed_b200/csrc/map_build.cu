@@ -325,25 +325,55 @@ __global__ void k_subdiv_count(const uint8_t* __restrict__ keep, int64_t n, uint
   }
 }
 
-__global__ void k_subdiv_emit(const int4* __restrict__ coords, int64_t n, int order, const uint8_t* __restrict__ bits,
-                              const int64_t* __restrict__ first, int4* __restrict__ child_coords,
-                              int32_t* __restrict__ child_src, int32_t* __restrict__ remap) {
-  for (int64_t v = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; v < n;
-       v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+// One block of kEmitBlock parents: their children form one contiguous run of
+// the output, staged in shared memory and stored coalesced.
+constexpr int kEmitBlock = 256;
+
+__global__ void __launch_bounds__(kEmitBlock) k_subdiv_emit(const int4* __restrict__ coords, int64_t n, int order,
+                                                            const uint8_t* __restrict__ bits,
+                                                            const int64_t* __restrict__ first,
+                                                            int4* __restrict__ child_coords,
+                                                            int32_t* __restrict__ child_src,
+                                                            int32_t* __restrict__ remap) {
+  __shared__ int4 s_coords[8 * kEmitBlock];
+  __shared__ int32_t s_src[8 * kEmitBlock];
+  __shared__ int s_total;
+  const int tid = threadIdx.x;
+  const int64_t v0 = static_cast<int64_t>(blockIdx.x) * kEmitBlock;
+  const int64_t v = v0 + tid;
+  const int64_t base = first[v0];
+  if (tid == 0) s_total = 0;
+  __syncthreads();
+  if (v < n) {
     const int4 c = coords[v];
     const uint32_t b = bits[v];
-    int64_t r = first[v];
+    const int64_t local = first[v] - base;
+    // always in range, unless the scan gave up on a wait (error bit set)
+    const bool ok = local >= 0 && local + __popc(b) <= 8 * kEmitBlock;
+    int r = static_cast<int>(ok ? local : 0);
+    int32_t rm[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int o = octant_of(k, order);
-      if ((b >> k) & 1u) {
-        child_coords[r] = make_int4(c.x, 2 * c.y + (o >> 2), 2 * c.z + ((o >> 1) & 1), 2 * c.w + (o & 1));
-        child_src[r] = static_cast<int32_t>(8 * v + o);
-        remap[8 * v + o] = static_cast<int32_t>(r);
+      rm[o] = -1;
+      if (ok && ((b >> k) & 1u)) {
+        s_coords[r] = make_int4(c.x, 2 * c.y + (o >> 2), 2 * c.z + ((o >> 1) & 1), 2 * c.w + (o & 1));
+        s_src[r] = static_cast<int32_t>(8 * v + o);
+        rm[o] = static_cast<int32_t>(base + r);
         ++r;
-      } else {
-        remap[8 * v + o] = -1;
       }
+    }
+    reinterpret_cast<int4*>(remap)[2 * v] = make_int4(rm[0], rm[1], rm[2], rm[3]);
+    reinterpret_cast<int4*>(remap)[2 * v + 1] = make_int4(rm[4], rm[5], rm[6], rm[7]);
+    if (ok) atomicMax(&s_total, r);
+  }
+  __syncthreads();
+  const int total = s_total;
+  const int64_t cap = 8 * n;
+  for (int i = tid; i < total; i += kEmitBlock) {
+    if (base + i < cap) {
+      child_coords[base + i] = s_coords[i];
+      child_src[base + i] = s_src[i];
     }
   }
 }
@@ -731,8 +761,7 @@ cudaError_t launch_subdiv_emit(const int32_t* coords, int64_t n, int order, cons
                                const int64_t* first, int32_t* child_coords, int32_t* child_src, int32_t* remap,
                                cudaStream_t s) {
   if (n == 0) return cudaSuccess;
-  const int64_t blocks = (n + 255) / 256;
-  k_subdiv_emit<<<static_cast<unsigned>(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, s>>>(
+  k_subdiv_emit<<<static_cast<unsigned>((n + kEmitBlock - 1) / kEmitBlock), kEmitBlock, 0, s>>>(
       reinterpret_cast<const int4*>(coords), n, order, bits, first, reinterpret_cast<int4*>(child_coords), child_src,
       remap);
   count_launches(1);

@@ -18,7 +18,8 @@
 //   k_down_pool    one thread per (parent, 16-byte vector of channels): max
 //                  or mean over the children present, j ascending, in fp32.
 // Upsample: the children's coordinates come from the subdivision kernels of
-// map_build.cu in mask order; k_gather_rows copies each child's parent row.
+// map_build.cu in mask order; k_expand_rows copies each parent's row to its
+// children.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -32,6 +33,10 @@ namespace smc {
 namespace {
 
 constexpr int kThreads = 256;
+#ifndef SMC_POOL_BLOCKS_PER_SM
+#define SMC_POOL_BLOCKS_PER_SM 3
+#endif
+constexpr int kPoolBlocksPerSm = SMC_POOL_BLOCKS_PER_SM;  // 85 registers a thread: no spills
 constexpr uint32_t kNoSlot = 0xFFFFFFFFu;
 constexpr unsigned long long kFree = ~0ull;
 constexpr uint64_t kFibHash = 0x9E3779B97F4A7C15ull;
@@ -140,28 +145,45 @@ template <> struct Lanes<__half> {
 };
 
 // kV channels per thread: 16 / sizeof(T) (one 16-byte load per child) or 1.
+// The grid-stride loop is software-pipelined: the next item's child list
+// (rows and mask) is loaded before this item's features, so that its latency
+// overlaps theirs.
 template <typename T, int kV>
-__global__ void __launch_bounds__(kThreads) k_down_pool(const T* __restrict__ feats, int c,
-                                                        const int32_t* __restrict__ child_rows,
-                                                        const uint8_t* __restrict__ pbits,
-                                                        const int64_t* __restrict__ count, int64_t n, int mode,
-                                                        T* __restrict__ out) {
+__global__ void __launch_bounds__(kThreads, kPoolBlocksPerSm) k_down_pool(const T* __restrict__ feats, int c,
+                                                                          const int32_t* __restrict__ child_rows,
+                                                                          const uint8_t* __restrict__ pbits,
+                                                                          const int64_t* __restrict__ count,
+                                                                          int64_t n, int mode, T* __restrict__ out) {
   using Vec = typename std::conditional<kV == 1, T, uint4>::type;
   const int64_t m = *count < n ? *count : n;
   const int nv = c / kV;
   const int64_t total = m * nv;
-  for (int64_t t = blockIdx.x * static_cast<int64_t>(kThreads) + threadIdx.x; t < total;
-       t += static_cast<int64_t>(gridDim.x) * kThreads) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
+  int64_t t = blockIdx.x * static_cast<int64_t>(kThreads) + threadIdx.x;
+  int4 r0 = make_int4(0, 0, 0, 0), r1 = r0;
+  uint32_t b = 0;
+  if (t < total) {
+    const int64_t p = t / nv;
+    b = pbits[p];
+    r0 = reinterpret_cast<const int4*>(child_rows)[2 * p];
+    r1 = reinterpret_cast<const int4*>(child_rows)[2 * p + 1];
+  }
+  for (; t < total; t += stride) {
     const int64_t p = t / nv;
     const int q = static_cast<int>(t - p * nv);
-    const uint32_t b = pbits[p];
-    const int4 r0 = reinterpret_cast<const int4*>(child_rows)[2 * p];
-    const int4 r1 = reinterpret_cast<const int4*>(child_rows)[2 * p + 1];
+    const uint32_t bc = b;
     const int32_t row[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+    const int64_t tn = t + stride;
+    if (tn < total) {
+      const int64_t pn = tn / nv;
+      b = pbits[pn];
+      r0 = reinterpret_cast<const int4*>(child_rows)[2 * pn];
+      r1 = reinterpret_cast<const int4*>(child_rows)[2 * pn + 1];
+    }
     Vec u[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-      if (((b >> j) & 1u) && static_cast<uint64_t>(row[j]) < static_cast<uint64_t>(n))  // rows are valid unless
+      if (((bc >> j) & 1u) && static_cast<uint64_t>(row[j]) < static_cast<uint64_t>(n))  // rows are valid unless
         u[j] = __ldg(reinterpret_cast<const Vec*>(feats + static_cast<int64_t>(row[j]) * c) + q);  // the call fails
     float acc[kV];
 #pragma unroll
@@ -169,7 +191,7 @@ __global__ void __launch_bounds__(kThreads) k_down_pool(const T* __restrict__ fe
     bool any = false;  // a parent has at least one child
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      if (((b >> j) & 1u) && static_cast<uint64_t>(row[j]) < static_cast<uint64_t>(n)) {
+      if (((bc >> j) & 1u) && static_cast<uint64_t>(row[j]) < static_cast<uint64_t>(n)) {
         const T* x = reinterpret_cast<const T*>(&u[j]);
 #pragma unroll
         for (int e = 0; e < kV; ++e) {
@@ -180,7 +202,7 @@ __global__ void __launch_bounds__(kThreads) k_down_pool(const T* __restrict__ fe
       }
     }
     if (mode == 1) {
-      const float cnt = static_cast<float>(__popc(b));
+      const float cnt = static_cast<float>(__popc(bc));
 #pragma unroll
       for (int e = 0; e < kV; ++e) acc[e] = acc[e] / cnt;
     }
@@ -192,30 +214,59 @@ __global__ void __launch_bounds__(kThreads) k_down_pool(const T* __restrict__ fe
   }
 }
 
-// out[r] = rows[src[r] >> 3] for r < m: whole rows of `units` elements of U.
+// Parent p's row copied to its children, rows first[p] .. first[p] + cnt - 1
+// of the output (children are listed parent by parent): one thread per
+// (parent, unit of U), one load and up to eight stores; each store
+// instruction of a warp writes whole runs of child rows.
 template <typename U>
-__global__ void __launch_bounds__(kThreads) k_gather_rows(const U* __restrict__ rows, int64_t units,
-                                                          const int32_t* __restrict__ src, int64_t m,
+__global__ void __launch_bounds__(kThreads) k_expand_rows(const U* __restrict__ rows, int64_t units,
+                                                          const int64_t* __restrict__ first,
+                                                          const uint8_t* __restrict__ bits, int64_t n, int64_t cap,
                                                           U* __restrict__ out) {
-  const int64_t total = m * units;
+  const int64_t total = n * units;
   for (int64_t t = blockIdx.x * static_cast<int64_t>(kThreads) + threadIdx.x; t < total;
        t += static_cast<int64_t>(gridDim.x) * kThreads) {
-    const int64_t r = t / units;
-    const int64_t q = t - r * units;
-    out[t] = __ldg(rows + static_cast<int64_t>(src[r] >> 3) * units + q);
+    const int64_t p = t / units;
+    const int64_t q = t - p * units;
+    const int64_t r0 = first[p];
+    const int cnt = __popc(static_cast<uint32_t>(bits[p]));
+    if (cnt == 0 || r0 < 0 || r0 + cnt > cap) continue;  // out of range only if the scan failed
+    const U x = __ldg(rows + t);
+    U* dst = out + r0 * units + q;
+    for (int i = 0; i < cnt; ++i) dst[i * units] = x;
   }
+}
+
+// Grid of a grid-stride kernel: as many blocks as fit on the device at once
+// (blocks per SM from the occupancy calculator, times the SM count), capped
+// by the work.
+template <typename K>
+unsigned resident_grid(K kernel, int64_t work) {
+  static int per_sm = 0, sms = 0;
+  if (per_sm == 0) {
+    int dev = 0, b = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, kThreads, 0);
+    sms = n > 0 ? n : 148;
+    per_sm = b > 0 ? b : 1;
+  }
+  const int64_t blocks = (work + kThreads - 1) / kThreads;
+  const int64_t cap = static_cast<int64_t>(per_sm) * sms;
+  return static_cast<unsigned>(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
 }
 
 template <typename T>
 void pool_launch(const DownArgs& a, cudaStream_t s, bool vec) {
   constexpr int kV = 16 / sizeof(T);
-  const unsigned g = grid_of(a.n * (vec ? a.c / kV : a.c));
   const T* f = static_cast<const T*>(a.feats);
   T* o = static_cast<T*>(a.out);
   if (vec)
-    k_down_pool<T, kV><<<g, kThreads, 0, s>>>(f, a.c, a.child_rows, a.pbits, a.info + kTaps, a.n, a.mode, o);
+    k_down_pool<T, kV><<<resident_grid(k_down_pool<T, kV>, a.n * (a.c / kV)), kThreads, 0, s>>>(
+        f, a.c, a.child_rows, a.pbits, a.info + kTaps, a.n, a.mode, o);
   else
-    k_down_pool<T, 1><<<g, kThreads, 0, s>>>(f, a.c, a.child_rows, a.pbits, a.info + kTaps, a.n, a.mode, o);
+    k_down_pool<T, 1><<<resident_grid(k_down_pool<T, 1>, a.n * a.c), kThreads, 0, s>>>(
+        f, a.c, a.child_rows, a.pbits, a.info + kTaps, a.n, a.mode, o);
 }
 
 }  // namespace
@@ -248,23 +299,24 @@ cudaError_t launch_downsample(const DownArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_gather_rows(const void* rows, int64_t row_bytes, const int32_t* src, int64_t m, void* out,
-                               int elem_bytes, cudaStream_t s) {
-  if (m == 0 || row_bytes == 0) return cudaSuccess;
+cudaError_t launch_expand_rows(const void* rows, int64_t row_bytes, const int64_t* first, const uint8_t* bits,
+                               int64_t n, void* out, int elem_bytes, cudaStream_t s) {
+  if (n == 0 || row_bytes == 0) return cudaSuccess;
   const bool vec = row_bytes % 16 == 0 && (reinterpret_cast<uintptr_t>(rows) & 15u) == 0 &&
                    (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
+  const int64_t cap = 8 * n;
   if (vec) {
     const int64_t units = row_bytes / 16;
-    k_gather_rows<uint4><<<grid_of(m * units), kThreads, 0, s>>>(static_cast<const uint4*>(rows), units, src, m,
-                                                                 static_cast<uint4*>(out));
+    k_expand_rows<uint4><<<resident_grid(k_expand_rows<uint4>, n * units), kThreads, 0, s>>>(
+        static_cast<const uint4*>(rows), units, first, bits, n, cap, static_cast<uint4*>(out));
   } else if (elem_bytes == 4) {
     const int64_t units = row_bytes / 4;
-    k_gather_rows<uint32_t><<<grid_of(m * units), kThreads, 0, s>>>(static_cast<const uint32_t*>(rows), units, src,
-                                                                    m, static_cast<uint32_t*>(out));
+    k_expand_rows<uint32_t><<<resident_grid(k_expand_rows<uint32_t>, n * units), kThreads, 0, s>>>(
+        static_cast<const uint32_t*>(rows), units, first, bits, n, cap, static_cast<uint32_t*>(out));
   } else {
     const int64_t units = row_bytes / 2;
-    k_gather_rows<uint16_t><<<grid_of(m * units), kThreads, 0, s>>>(static_cast<const uint16_t*>(rows), units, src,
-                                                                    m, static_cast<uint16_t*>(out));
+    k_expand_rows<uint16_t><<<resident_grid(k_expand_rows<uint16_t>, n * units), kThreads, 0, s>>>(
+        static_cast<const uint16_t*>(rows), units, first, bits, n, cap, static_cast<uint16_t*>(out));
   }
   count_launches(1);
   return cudaGetLastError();
