@@ -518,8 +518,13 @@ def run_gpu(args):
 
 
 def run_e2e(w, f, wt, b, batch, dev, stream, args):
-    """Same step through the public API, with the step's inputs copied from
-    pinned host memory and the result copied back inside the timed region."""
+    """Same step through the public API, with each step's inputs copied from
+    pinned host memory and its result copied back inside the timed region.
+    Steps are pipelined the way a serving loop runs them: inputs go up on a
+    copy stream, the build and the conv run on the compute stream, the result
+    comes back on a second copy stream, and two device slots let step k's
+    copy-back overlap step k+1's upload and compute.  Timed from the first
+    upload to the last copy-back, on the device; ms = that time / steps."""
     import torch
 
     import submanifold_sparse_convolution_packed_b200 as smc
@@ -527,28 +532,67 @@ def run_e2e(w, f, wt, b, batch, dev, stream, args):
     feats_h = torch.from_numpy(f).to(torch.bfloat16).pin_memory()
     w_h = torch.from_numpy(wt).to(torch.bfloat16).pin_memory()
     b_h = torch.from_numpy(b).to(torch.bfloat16).pin_memory()
-    out_h = torch.empty((w.n, w.cout), dtype=torch.bfloat16).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (coords_h, feats_h, w_h, b_h))
-    d2h = out_h.numel() * out_h.element_size()
-    times = []
+    depth = 2
+    outs_h = [torch.empty((w.n, w.cout), dtype=torch.bfloat16).pin_memory() for _ in range(depth)]
+    d2h = outs_h[0].numel() * outs_h[0].element_size()
+    slots = [dict(c=torch.empty_like(coords_h, device=dev), x=torch.empty_like(feats_h, device=dev),
+                  w=torch.empty_like(w_h, device=dev), b=torch.empty_like(b_h, device=dev),
+                  y=torch.empty((w.n, w.cout), dtype=torch.bfloat16, device=dev)) for _ in range(depth)]
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    inputs_free = [None] * depth   # compute consumed the slot's inputs
+    output_free = [None] * depth   # copy-back of the slot's output done
+    maps = []
+
+    def step(i):
+        k = i % depth
+        sl = slots[k]
+        with torch.cuda.stream(up):
+            if inputs_free[k] is not None:
+                up.wait_event(inputs_free[k])
+            for name, src in (("c", coords_h), ("x", feats_h), ("w", w_h), ("b", b_h)):
+                sl[name].copy_(src, non_blocking=True)
+            ready = ev()
+            ready.record(up)
+        stream.wait_event(ready)
+        if output_free[k] is not None:
+            stream.wait_event(output_free[k])
+        m = smc.build_map(sl["c"], w.grid, batch=batch, stream=stream, sync=False)
+        smc.conv(m, sl["x"], sl["w"], sl["b"], ksize=3, orientation=1, out=sl["y"], stream=stream)
+        done = ev()
+        done.record(stream)
+        inputs_free[k] = done
+        with torch.cuda.stream(down):
+            down.wait_event(done)
+            outs_h[k].copy_(sl["y"], non_blocking=True)
+            back = ev()
+            back.record(down)
+        output_free[k] = back
+        maps.append((m, back))
+        while len(maps) > depth:  # retire old steps: check the build, free its map
+            old, e = maps.pop(0)
+            e.synchronize()
+            old.wait()
+            old.free()
+
     n = max(3, min(args.steps, 50))
-    for i in range(n + 3):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        c = coords_h.to(dev, non_blocking=True)
-        x = feats_h.to(dev, non_blocking=True)
-        ww = w_h.to(dev, non_blocking=True)
-        bb = b_h.to(dev, non_blocking=True)
-        m = smc.build_map(c, w.grid, batch=batch, stream=stream, sync=False)
-        y = smc.conv(m, x, ww, bb, ksize=3, orientation=1, stream=stream)
-        out_h.copy_(y, non_blocking=True)
-        e1.record(stream)
-        e1.synchronize()
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(up)
+    for i in range(3, 3 + n):
+        step(i)
+    down.wait_stream(stream)
+    e1.record(down)
+    e1.synchronize()
+    for m, e in maps:
+        e.synchronize()
         m.wait()
         m.free()
-        if i >= 3:
-            times.append(e0.elapsed_time(e1))
-    return {"ms": sum(times) / len(times), "h2d": h2d, "d2h": d2h}
+    torch.cuda.synchronize(dev)
+    return {"ms": e0.elapsed_time(e1) / n, "h2d": h2d, "d2h": d2h}
 
 
 # ------------------------------------------------------------- CPU oracle
