@@ -768,3 +768,34 @@ def test_resample_errors_and_edges(oracle_mod, map_lookup):
     kids, _, _ = smc.upsample(pc, None)
     np.testing.assert_array_equal(kids.cpu().numpy(), oracle_mod.upsample(pc.cpu().numpy(), np.ones((2, 8)))[0])
     smc.status()
+
+
+def test_downsample_upsample_varlen4_sampled(oracle_mod, map_lookup):
+    """Four items of 300k-600k voxels on a 256^3 grid (fp16, 64 channels),
+    shuffled, under each lookup structure: structure bit-exact, mean pooling
+    on 2048 sampled parents (each recomputed from its own children), and the
+    expansion back with the children's map bit-exact against the oracle's."""
+    w = workload("varlen4")
+    coords = _shuffled(w, 41)
+    f = S.features(w.n, 64, np.random.default_rng(42), "f16")
+    ct = torch.from_numpy(coords).cuda()
+    pc, pooled, mask, parent = smc.downsample(ct, w.grid, dev(f, "f16"), "mean", batch=4)
+    rpc, _, rmask, rparent = oracle_mod.downsample(coords, w.grid, None, oracle_mod.POOL_MEAN, 4)
+    np.testing.assert_array_equal(pc.cpu().numpy(), rpc)
+    np.testing.assert_array_equal(mask.cpu().numpy(), rmask)
+    np.testing.assert_array_equal(parent.cpu().numpy(), rparent)
+    ps = sample_rows(len(rpc), 2048, 43)
+    rows_of = np.flatnonzero(np.isin(rparent, ps))
+    spc, sp, _, _ = oracle_mod.downsample(coords[rows_of], w.grid, f[rows_of], oracle_mod.POOL_MEAN, 4)
+    np.testing.assert_array_equal(spc, rpc[ps])
+    check_close(host(pooled)[ps], sp, "f16", "mean pooling, sampled parents")
+    half = tuple((g + 1) // 2 for g in w.grid)
+    pm = smc.build_map(pc, half, batch=4)
+    kids, kf, child = smc.upsample(pc, mask, pooled, parent=pm)
+    rk, _ = oracle_mod.upsample(rpc, rmask)
+    np.testing.assert_array_equal(kids.cpu().numpy(), rk)
+    np.testing.assert_array_equal(kf.cpu().numpy()[:: 97], pooled.cpu().numpy()[np.repeat(np.arange(len(rpc)), rmask.sum(1).astype(np.int64))][:: 97])
+    rows = sample_rows(len(rk), 4096, 44)
+    ref = oracle_mod.neighbour_map(rk, w.grid)
+    np.testing.assert_array_equal(child.nbr().cpu().numpy()[rows], ref[rows])
+    smc.status()
