@@ -101,7 +101,11 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
   const uint32_t b_bytes = static_cast<uint32_t>(bn_cta) * row_bytes;
   const int kblocks = (p.cin + p.kb_elems - 1) / p.kb_elems;
   const int last_ksteps = (p.cin - (kblocks - 1) * p.kb_elems + 15) / 16;
-  const int64_t unit = kPair ? blockIdx.x / 2 : blockIdx.x;
+  // One-CTA launches take the schedule's tiles last to first: the schedule
+  // sorts rows by ascending corner/edge key, so the tiles with the most taps
+  // come last, and launching them first leaves the lighter tiles to fill the
+  // final partial wave.
+  const int64_t unit = kPair ? blockIdx.x / 2 : gridDim.x - 1 - blockIdx.x;
   const int64_t tile0 = (unit / p.nsplit) * (kPair ? 2 : 1);  // first tile of the unit
   const int64_t tile = tile0 + rank;
   const int n0 = static_cast<int>(unit % p.nsplit) * p.bn;
