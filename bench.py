@@ -205,35 +205,42 @@ def conv_variant_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, w
 
 def epilogue_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, w_d, b_d, out_d, reps=5):
     """Median device time (ms) of one conv on the bench's map: plain; with
-    SiLU and a residual fused into the epilogue; the same plus the GroupNorm-32
-    statistics of its output (smc_conv_ex, a statistics pass behind the conv);
-    and plain followed by the statistics pass.  Untimed for the bench value."""
+    SiLU and a residual (smc_conv_ex: the conv, then one row pass that applies
+    them in row order); the same plus the GroupNorm-32 statistics of the
+    output (in the same row pass); the same SiLU and residual done inside the
+    conv's epilogue instead (smc_set_conv_epilogue(1)); and plain followed by
+    a statistics pass.  Untimed for the bench value."""
     m = smc.build_map(coords_d, w.grid, batch=batch, stream=stream)
     residual = torch.randn(out_d.shape, device=out_d.device).to(out_d.dtype)
     stats = torch.zeros((batch, 32, 3), dtype=torch.float64, device=out_d.device)
+    silu_res = lambda: smc.conv(m, feats_d, w_d, b_d, out=out_d, stream=stream, residual=residual, act="silu")
     runs = {
-        "plain": lambda: smc.conv(m, feats_d, w_d, b_d, out=out_d, stream=stream),
-        "silu_residual_fused": lambda: smc.conv(m, feats_d, w_d, b_d, out=out_d, stream=stream,
-                                                residual=residual, act="silu"),
-        "silu_residual_fused_with_stats": lambda: smc.conv(m, feats_d, w_d, b_d, out=out_d, stream=stream,
-                                                           residual=residual, act="silu", coords=coords_d,
-                                                           stats=stats, groups=32),
-        "plain_then_stats_pass": lambda: (smc.conv(m, feats_d, w_d, b_d, out=out_d, stream=stream),
-                                          smc.group_stats(out_d, coords_d, batch, 32, stats, stream=stream)),
+        "plain": (0, lambda: smc.conv(m, feats_d, w_d, b_d, out=out_d, stream=stream)),
+        "silu_residual": (0, silu_res),
+        "silu_residual_with_stats": (0, lambda: smc.conv(m, feats_d, w_d, b_d, out=out_d, stream=stream,
+                                                         residual=residual, act="silu", coords=coords_d,
+                                                         stats=stats, groups=32)),
+        "silu_residual_in_conv_epilogue": (1, silu_res),
+        "plain_then_stats_pass": (0, lambda: (smc.conv(m, feats_d, w_d, b_d, out=out_d, stream=stream),
+                                              smc.group_stats(out_d, coords_d, batch, 32, stats, stream=stream))),
     }
     res = {}
-    for name, fn in runs.items():
-        ts = []
-        for _ in range(reps + 1):
-            flush.zero_()
-            stats.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            fn()
-            e1.record(stream)
-            e1.synchronize()
-            ts.append(e0.elapsed_time(e1))
-        res[name] = round(float(np.median(ts[1:])), 4)
+    try:
+        for name, (where, fn) in runs.items():
+            smc.set_conv_epilogue(where)
+            ts = []
+            for _ in range(reps + 1):
+                flush.zero_()
+                stats.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+                e1.synchronize()
+                ts.append(e0.elapsed_time(e1))
+            res[name] = round(float(np.median(ts[1:])), 4)
+    finally:
+        smc.set_conv_epilogue(0)
     m.free()
     smc.status(stream)
     return res

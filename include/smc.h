@@ -401,6 +401,15 @@ SMC_API int smc_set_profiling(int32_t on);
 SMC_API int smc_map_timing(const smc_map* map, float ms[3]);
 SMC_API int smc_kernel_launches(int64_t* count);
 SMC_API int smc_set_conv_variant(int32_t variant);
+/* smc_set_conv_epilogue: where smc_conv_ex applies the activation and the
+ *   residual for the tensor-core conv: 0 = a row pass behind the conv, in
+ *   row order, with the GroupNorm statistics in the same pass (default;
+ *   measured faster; a residual that is the output buffer itself always
+ *   goes through the epilogue), 1 = in the conv's own epilogue.  Results
+ *   agree to rounding: the row pass sees the conv's stored (rounded) output,
+ *   as a separate activation layer would.  Used to test and measure the two.  SMC_E_ARG for any other
+ *   value. */
+SMC_API int smc_set_conv_epilogue(int32_t where);
 SMC_API int smc_set_map_lookup(int32_t mode);
 
 #ifdef __cplusplus

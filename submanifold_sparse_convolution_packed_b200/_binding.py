@@ -31,7 +31,7 @@ EXPORTS = [
     "smc_set_hash_capacity", "smc_set_profiling", "smc_map_timing", "smc_kernel_launches",
     "smc_build_map_async", "smc_map_wait", "smc_neighbour_map_noalloc", "smc_set_conv_variant",
     "smc_set_map_lookup", "smc_map_stream_wait", "smc_subdivide", "smc_conv_ex", "smc_group_stats",
-    "smc_group_norm", "smc_downsample", "smc_upsample",
+    "smc_group_norm", "smc_downsample", "smc_upsample", "smc_set_conv_epilogue",
 ]
 
 
@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
         L.smc_map_timing.argtypes = [P, P]
         L.smc_kernel_launches.argtypes = [P]
         L.smc_set_conv_variant.argtypes = [i32]
+        L.smc_set_conv_epilogue.argtypes = [i32]
         L.smc_set_map_lookup.argtypes = [i32]
         for name in EXPORTS:
             if name != "smc_strerror":
@@ -483,6 +484,13 @@ def group_norm(x: torch.Tensor, coords: torch.Tensor, batch: int, groups: int, s
 def status(stream=None) -> None:
     """Synchronise the stream and raise if a conv kernel reported a timeout."""
     _check(lib().smc_status(_stream(stream)), "smc_status")
+
+
+def set_conv_epilogue(where: int) -> None:
+    """Where conv(..., act=, residual=) applies them on the tensor-core
+    kernel: 0 = a row pass behind the conv (default), 1 = the conv's own
+    epilogue (smc_set_conv_epilogue)."""
+    _check(lib().smc_set_conv_epilogue(int(where)), "smc_set_conv_epilogue")
 
 
 def set_conv_variant(variant: int) -> None:

@@ -539,6 +539,12 @@ int smc_set_map_lookup(int32_t mode) {
   return SMC_OK;
 }
 
+int smc_set_conv_epilogue(int32_t where) {
+  if (where != 0 && where != 1) return SMC_E_ARG;
+  smc::set_conv_epilogue(where);
+  return SMC_OK;
+}
+
 int smc_set_conv_variant(int32_t variant) {
   if (variant < 0 || variant > 3) return SMC_E_ARG;
   smc::set_conv_variant(variant);
@@ -944,6 +950,16 @@ int smc_conv_ex(const smc_map* map, const void* feats, int64_t cin, const void* 
     cudaGetLastError();
     return SMC_E_CUDA;
   }
+  // The tensor-core kernel leaves activation and residual to a row pass
+  // behind it (unless set to do them itself, or unless the residual is the
+  // output buffer, which the conv overwrites: then its epilogue reads each
+  // row's residual before storing the row); so do the statistics.
+  const bool pass = tc && !per_offset && smc::conv_epilogue() == 0 && (act != SMC_ACT_NONE || residual) &&
+                    residual != out;
+  if (pass) {
+    a.ep.residual = nullptr;
+    a.ep.act = SMC_ACT_NONE;
+  }
   cudaError_t e;
   if (per_offset) {
     void* acc = nullptr;
@@ -961,9 +977,24 @@ int smc_conv_ex(const smc_map* map, const void* feats, int64_t cin, const void* 
     cudaGetLastError();
     return SMC_E_CUDA;
   }
-  // Group statistics of the stored output: a pass right behind the conv on
-  // the same stream (measured faster than folding them into the conv's
-  // epilogue, see conv_tc.cu).
+  // Group statistics of the stored output: in the row pass, or a statistics
+  // pass right behind the conv on the same stream (both measured faster than
+  // folding them into the conv's epilogue, see conv_tc.cu).
+  if (pass) {
+    smc::Epilogue ep;
+    ep.batch = map->batch;
+    ep.groups = stats ? groups : 1;
+    ep.stripes = kStatStripes;
+    if (stats) {
+      const int rc = stats_begin(dev, s, map->batch, groups, &ep.stats);
+      if (rc != SMC_OK) return rc;
+    }
+    e = smc::launch_rows_pass(out, out, residual, act, n, static_cast<int>(cout), coords, ep, dtype, s);
+    if (e != cudaSuccess) cudaGetLastError();
+    const int rc2 = stats ? stats_end(ep.stats, map->batch, groups, stats, s, e == cudaSuccess) : SMC_OK;
+    if (e != cudaSuccess) return SMC_E_CUDA;
+    return rc2;
+  }
   if (stats) return smc_group_stats(out, n, cout, coords, map->batch, groups, stats, dtype, stream);
   return SMC_OK;
 }

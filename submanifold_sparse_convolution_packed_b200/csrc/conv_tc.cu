@@ -73,11 +73,12 @@ struct TcParams {
 // consecutive schedule tiles, the union of their tap masks); it loads its own
 // 128 gathered rows and half of the weight block's N columns, and every load
 // and arrival counts on the even CTA's full barriers.
-// kEpi: 0 = bias only; 1 = activation and residual.  Separate instances keep
-// the plain conv free of the extra epilogue code, which measured 5-19% slower
-// even when unused.  (Group statistics of the output are a separate pass,
-// k_group_stats: folded into this epilogue they measured slower than the
-// pass, by the registers and the reduction work they add to every CTA.)
+// kEpi: 0 = bias only; 1 = activation and residual, used only when
+// set_conv_epilogue(1) asks for them here: by default a row pass behind the
+// conv applies them (k_rows_pass), which measured faster, since everything in
+// this epilogue lengthens the tile's hold on its SM slot and the residual rows
+// are read in schedule order.  Separate instances keep the plain conv free of
+// the extra epilogue code, which measured 5-19% slower even when unused.
 template <bool kPair, int kEpi>
 __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant__ CUtensorMap fmap,
                                                         const __grid_constant__ CUtensorMap wmap,
@@ -266,14 +267,34 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
     }
     // ---------------------------------------------------------- epilogue
     // y = act(acc + bias) + residual, rounded and stored as 16-byte vectors.
+    constexpr bool extra = kEpi >= 1;  // activation and residual
+    const uint16_t* res = static_cast<const uint16_t*>(p.ep.residual);
+    // Residual of 32 output columns from c0 (4 x 16 bytes; zeros past the
+    // row's columns).  The first chunk's is loaded before the accumulator is
+    // ready (while the last MMAs run) and each later chunk's one chunk ahead;
+    // a thread reads and writes only its own row, and loads a column before
+    // storing it, so this holds for a residual that is the output buffer.
+    auto load_res = [&](int c0, uint4 (&r)[4]) {
+      int nc = p.bn - c0 < 32 ? p.bn - c0 : 32;
+      if (p.cout - (n0 + c0) < nc) nc = p.cout - (n0 + c0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        r[j] = make_uint4(0, 0, 0, 0);
+        if (extra && res && v >= 0 && 8 * j < nc)
+          r[j] = *reinterpret_cast<const uint4*>(res + static_cast<int64_t>(v) * p.cout + n0 + c0 + 8 * j);
+      }
+    };
+    uint4 rcur[4], rnext[4];
+    if constexpr (extra) load_res(0, rcur);
     const bool ready = mbar_wait_bounded(bar_acc, 0, p.err) && !s_misc[1];
     tc_fence_after();
     if (ready) {
       const bool bf = p.is_bf16 != 0;
-      constexpr bool extra = kEpi >= 1;  // activation and residual
-      const uint16_t* res = static_cast<const uint16_t*>(p.ep.residual);
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
       for (int c0 = 0; c0 < p.bn; c0 += 32) {
+        if constexpr (extra) {
+          if (c0 + 32 < p.bn) load_res(c0 + 32, rnext);
+        }
         float acc[32];
         tmem_ld_32cols(t_row + c0, acc);
         int ncols = p.bn - c0 < 32 ? p.bn - c0 : 32;
@@ -284,9 +305,13 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
             if (j >= ncols) break;
             const int col = n0 + c0 + j;
             const int64_t at = static_cast<int64_t>(v) * p.cout + col;
-            uint4 rv = make_uint4(0, 0, 0, 0);
-            if (extra && res) rv = *reinterpret_cast<const uint4*>(res + at);
-            const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
+            uint32_t rw[4] = {0u, 0u, 0u, 0u};
+            if constexpr (extra) {
+              rw[0] = rcur[j / 8].x;
+              rw[1] = rcur[j / 8].y;
+              rw[2] = rcur[j / 8].z;
+              rw[3] = rcur[j / 8].w;
+            }
             uint32_t packed[4];
 #pragma unroll
             for (int e = 0; e < 8; e += 2) {
@@ -308,6 +333,10 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
             }
             *reinterpret_cast<uint4*>(p.out + at) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
           }
+        }
+        if constexpr (extra) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) rcur[j] = rnext[j];
         }
       }
     }
@@ -402,6 +431,10 @@ static TcShape choose_shape(int cin, int cout, int64_t ntiles) {
 }
 
 void set_conv_variant(int v) { g_conv_variant.store(v); }
+
+static std::atomic<int> g_conv_epilogue{0};
+void set_conv_epilogue(int where) { g_conv_epilogue.store(where); }
+int conv_epilogue() { return g_conv_epilogue.load(); }
 int conv_variant() { return g_conv_variant.load(); }
 
 cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s) {

@@ -124,6 +124,14 @@ cudaError_t launch_expand_rows(const void* rows, int64_t row_bytes, const int64_
 // y = act(gamma * (x - mean) / sqrt(var + eps) + beta) from such statistics.
 cudaError_t launch_group_stats(const void* x, int64_t n, int c, const int32_t* coords, const Epilogue& ep, int dtype,
                                cudaStream_t s);
+// y = act(x) + residual (residual may be null; y may be x, and so may the
+// residual), in row order, with the statistics of y when ep.stats is set.
+cudaError_t launch_rows_pass(const void* x, void* y, const void* residual, int act, int64_t n, int c,
+                             const int32_t* coords, const Epilogue& ep, int dtype, cudaStream_t s);
+// Where the tensor-core conv applies activation and residual: 0 = a row pass
+// behind it (default), 1 = its own epilogue.
+void set_conv_epilogue(int where);
+int conv_epilogue();
 // stats[i] += sum over s < stripes of copies[s * len + i]
 cudaError_t launch_stats_fold(const double* copies, int stripes, int64_t len, double* stats, cudaStream_t s);
 cudaError_t launch_group_norm(const void* x, int64_t n, int c, const int32_t* coords, int batch, int groups,

@@ -432,9 +432,18 @@ def _np_stats(x, coords, batch, groups):
     return st
 
 
+@pytest.fixture(params=[0, 1], ids=["row_pass", "in_conv"])
+def conv_epilogue(request):
+    """Runs a test with the tensor-core conv's activation and residual applied
+    by the row pass behind it, and inside its own epilogue."""
+    smc.set_conv_epilogue(request.param)
+    yield request.param
+    smc.set_conv_epilogue(0)
+
+
 @pytest.mark.parametrize("dtype,variant", [("bf16", 1), ("bf16", 2), ("bf16", 3), ("f32", 1), ("f16", 1)])
 @pytest.mark.parametrize("act", [None, "relu", "silu"])
-def test_conv_ex_epilogue(oracle_mod, dtype, variant, act):
+def test_conv_ex_epilogue(oracle_mod, dtype, variant, act, conv_epilogue):
     """out = act(conv + bias) + residual, and the GroupNorm statistics of the
     stored output: the output against the oracle, the statistics against
     fp64 sums of that very output (the two-item shell workload, 64 -> 64
@@ -461,7 +470,7 @@ def test_conv_ex_epilogue(oracle_mod, dtype, variant, act):
     np.testing.assert_allclose(stats.cpu().numpy(), _np_stats(got, w.coords, 2, 32), rtol=1e-9, atol=1e-6)
 
 
-def test_conv_ex_residual_in_place(oracle_mod):
+def test_conv_ex_residual_in_place(oracle_mod, conv_epilogue):
     """y = conv + out: the residual may be the output buffer itself."""
     w = workload("shell2")
     m = build(w)
@@ -490,7 +499,7 @@ def test_group_norm(oracle_mod, dtype):
     check_close(host(out), ref, dtype, f"group_norm {dtype}")
 
 
-def test_resblock_chain(oracle_mod):
+def test_resblock_chain(oracle_mod, conv_epilogue):
     """A ResBlock on one cached map: GroupNorm32 + SiLU, conv (statistics of
     its output fused), GroupNorm32 + SiLU, conv + skip.  Every step is checked
     against the oracle fed the GPU's own input to that step."""
@@ -799,3 +808,32 @@ def test_downsample_upsample_varlen4_sampled(oracle_mod, map_lookup):
     ref = oracle_mod.neighbour_map(rk, w.grid)
     np.testing.assert_array_equal(child.nbr().cpu().numpy()[rows], ref[rows])
     smc.status()
+
+
+@pytest.mark.parametrize("dtype,cout,groups", [("bf16", 128, 32), ("bf16", 256, 8), ("f32", 128, 32), ("f16", 128, 128)])
+def test_row_pass_shuffled_items(oracle_mod, dtype, cout, groups):
+    """The row pass behind a tensor-core or FMA conv on the two-item shell
+    workload with its rows shuffled (batch items alternate row by row):
+    act(conv) + residual against the oracle, the GroupNorm statistics against
+    fp64 sums of the stored output, and the statistics-only pass alike."""
+    w0 = workload("shell2")
+    perm = np.random.default_rng(51).permutation(w0.n)
+    coords = np.ascontiguousarray(w0.coords[perm])
+    w = S.Workload("shell2_shuffled", coords, w0.grid, 64, cout, (dtype,))
+    m = build(w)
+    f, wt, b = _layer(w, dtype, 0, 3, 64, cout)
+    res = S.round_to(np.random.default_rng(52).standard_normal((w.n, cout)).astype(np.float32), dtype)
+    ct = torch.from_numpy(coords).cuda()
+    stats = torch.zeros((2, groups, 3), dtype=torch.float64, device="cuda")
+    out = smc.conv(m, dev(f, dtype), dev(wt, dtype), dev(b, dtype), residual=dev(res, dtype), act="silu",
+                   coords=ct, stats=stats, groups=groups)
+    smc.status()
+    got = host(out)
+    rows = sample_rows(w.n, 4096, 53)
+    ref = oracle_mod.activation(oracle_mod.conv(coords, w.grid, f, wt, b, 3, 1, rows=rows, threads=THREADS), 2)
+    check_close(got[rows], ref + res[rows], dtype, f"row pass {dtype} {cout}")
+    np.testing.assert_allclose(stats.cpu().numpy(), _np_stats(got, coords, 2, groups), rtol=1e-9, atol=1e-6)
+    st2 = torch.zeros_like(stats)
+    smc.group_stats(out, ct, 2, groups, st2)
+    smc.status()
+    np.testing.assert_allclose(st2.cpu().numpy(), _np_stats(got, coords, 2, groups), rtol=1e-9, atol=1e-6)
