@@ -248,23 +248,32 @@ SMC_API int smc_conv(const smc_map* map, const void* feats, int64_t cin, const v
              int32_t dtype, void* stream);
 
 /*
- * smc_conv_ex -- smc_conv with a fused epilogue for the layers around the
+ * smc_conv_ex -- smc_conv with the epilogue of the layers around the
  * decoders' convs (norms, activations and ResBlocks: Pixal3D MLX README
  * "Status"; SparseGroupNorm32 and activations: LATO.2 MLX port README
  * "Status"):
  *
  *   out = round(act(bias + conv(feats)) + residual)
  *
+ * On the tensor-core kernel the activation, the residual and the statistics
+ * are applied by one row pass enqueued right behind the conv, which sees the
+ * conv's stored (rounded) output (smc_set_conv_epilogue selects the conv's
+ * own epilogue instead; a residual that is `out` itself always uses it); the
+ * FMA kernel applies them in its epilogue and the per-offset variant in its
+ * final pass.
+ *
  * residual : device [n, cout] in the output type, or NULL; it may be `out`
  *            itself (y = conv + out) but must not otherwise overlap it.
  * act      : SMC_ACT_NONE, SMC_ACT_RELU (max(y, 0)) or SMC_ACT_SILU
- *            (y / (1 + exp(-y))), applied before the residual.
+ *            (y / (1 + exp(-y)), in fp32 with the fast exponential),
+ *            applied before the residual.
  * stats    : device fp64 [batch, groups, 3] or NULL: for every batch item b
  *            and channel group g (cout / groups channels each), the sum, the
  *            sum of squares and the number of the stored output values of
  *            the item's rows are ADDED (the caller zeroes it) -- what a
- *            following smc_group_norm normalises with.  Computed by the
- *            smc_group_stats pass over `out`, enqueued right behind the conv.
+ *            following smc_group_norm normalises with.  Computed in the
+ *            row pass, or by the smc_group_stats pass over `out` enqueued
+ *            right behind the conv.
  * coords   : device int32 [n, 4], the map's coordinates (the batch index of
  *            each row); needed with stats.
  * groups   : >= 1 and dividing cout; used with stats.

@@ -257,6 +257,7 @@ __global__ void k_stats_fold(const double* __restrict__ copies, int stripes, int
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < len;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     double t = 0.0;
+#pragma unroll 8
     for (int s = 0; s < stripes; ++s) t += copies[s * len + i];
     stats[i] += t;
   }
