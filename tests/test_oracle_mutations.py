@@ -89,11 +89,31 @@ PY_MUTATIONS = {
 RESAMPLE_PINS = ["test_golden_downsample_upsample", "test_downsample_matches_dense_pooling",
                  "test_upsample_matches_nearest_interpolation", "test_upsample_index_is_subdivide_octant_reversed",
                  "test_downsample_upsample_round_trip"]
+# the same for subdivision, the activations and GroupNorm, against their pins
+OTHER_MUTATIONS = {
+    "subdivide_axes_swapped": ("a, cc, e = o >> 2, (o >> 1) & 1, o & 1", "e, cc, a = o >> 2, (o >> 1) & 1, o & 1"),
+    "subdivide_not_doubled": ("children[:, o, 2] = 2 * c[:, 2] + cc", "children[:, o, 2] = c[:, 2] + cc"),
+    "silu_sign": ("return y / (1.0 + np.exp(-y))", "return y / (1.0 + np.exp(y))"),
+    "relu_leaky": ("return np.maximum(y, 0.0)", "return np.maximum(y, 0.01 * y)"),
+    "stats_ignore_item": ("rows = xg[b == item]", "rows = xg"),
+    "variance_unbiased": ("var = st[:, :, 1] / cnt - mean * mean", "var = (st[:, :, 1] - cnt * mean * mean) / (cnt - 1)"),
+    "eps_outside_sqrt": ("/ np.sqrt(var[b][:, g_of_c] + eps)", "/ (np.sqrt(var[b][:, g_of_c]) + eps)"),
+    "gamma_after_beta": ("""    if gamma is not None:
+        y = y * np.asarray(gamma, dtype=np.float64)[None, :]
+    if beta is not None:
+        y = y + np.asarray(beta, dtype=np.float64)[None, :]""", """    if beta is not None:
+        y = y + np.asarray(beta, dtype=np.float64)[None, :]
+    if gamma is not None:
+        y = y * np.asarray(gamma, dtype=np.float64)[None, :]"""),
+}
+OTHER_PINS = ["test_golden_subdivide_one_voxel", "test_subdivide_full_box_is_full_doubled_box",
+              "test_subdivide_parent_and_octant_recovery", "test_activation_matches_torch",
+              "test_group_norm_matches_torch_per_item", "test_group_stats_hand_example"]
 
 
 def _py_mutant(name):
     import types
-    old, new = PY_MUTATIONS[name]
+    old, new = PY_MUTATIONS[name] if name in PY_MUTATIONS else OTHER_MUTATIONS[name]
     src = open(PY_SRC).read()
     assert src.count(old) == 1, f"mutation {name} no longer applies"
     mod = types.ModuleType(f"oracle_mutant_{name}")
@@ -115,3 +135,16 @@ def test_resample_pins_reject_planted_mistake(name):
         except Exception:
             failed.append(pin)
     assert failed, f"planted mistake {name!r} passed every resampling pin"
+
+
+@pytest.mark.parametrize("name", sorted(OTHER_MUTATIONS))
+def test_subdivide_and_norm_pins_reject_planted_mistake(name):
+    import tests.test_oracle_pins as pins
+    mod = _py_mutant(name)
+    failed = []
+    for pin in OTHER_PINS:
+        try:
+            getattr(pins, pin)(mod)
+        except Exception:
+            failed.append(pin)
+    assert failed, f"planted mistake {name!r} passed every subdivision / norm pin"
