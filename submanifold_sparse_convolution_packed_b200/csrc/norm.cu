@@ -142,8 +142,14 @@ __global__ void __launch_bounds__(kNormThreads) k_rows_pass(const T* x, T* y, co
 // kG: channels per group when every group of the unit is whole and
 // lies in it or holds it (a power of two; kG >= kU: the unit lies in one
 // group), else 0 (sums per channel, added to their groups at a flush).
+// Accumulator slots of a k_rows_flat thread with statistics (see kSlots).
+constexpr int flat_slots(int u, int g) { return g == 0 ? u : u / (g < u ? g : u); }
+
+// With statistics and at most four accumulator slots the kernel is held to
+// 64 registers (four blocks per SM): measured faster than 74 registers at
+// three blocks.  With more slots (one channel per group) that would spill.
 template <typename T, bool kStats, int kU, int kG>
-__global__ void __launch_bounds__(kNormThreads) k_rows_flat(const T* x, T* y, const T* residual, int act, int64_t n,
+__global__ void __launch_bounds__(kNormThreads, kStats && flat_slots(kU, kG) <= 4 ? 4 : 1) k_rows_flat(const T* x, T* y, const T* residual, int act, int64_t n,
                                                             int c, const int32_t* __restrict__ coords, Epilogue ep) {
   extern __shared__ double s_acc[];
   constexpr int kWarps = kNormThreads / 32;
@@ -333,9 +339,12 @@ cudaError_t launch_rows_pass(const void* x, void* y, const void* residual, int a
   int64_t blocks = (want < cap ? want : cap + step - 1) / step * step;
   if (blocks < step) blocks = step;
   const size_t flat_smem = static_cast<size_t>(entries) * kWarps * sizeof(double);
-  // With statistics and rows under 256 bytes the per-row kernel measured
-  // faster (a thread keeps its whole row in flight): 64-channel bf16/fp16.
-  const bool flat = step <= cap && flat_smem <= 48 * 1024 && (!ep.stats || static_cast<int64_t>(c) * es >= 256);
+  // For statistics alone on rows under 256 bytes (64-channel bf16/fp16) the
+  // per-row kernel measured faster (decoder stage 3: 113 vs 123 us; a thread
+  // keeps its whole row in flight); with the transform too, this one (721 vs
+  // 772 us for the conv and the pass).
+  const bool flat = step <= cap && flat_smem <= 48 * 1024 &&
+                    (!ep.stats || y != nullptr || static_cast<int64_t>(c) * es >= 256);
   if (flat) {
     const unsigned g = static_cast<unsigned>(blocks);
     auto run = [&](auto tag, auto per) {
