@@ -51,7 +51,7 @@ typedef struct smc_map smc_map;
 /* Storage type of feats, weight, bias and out in smc_conv. */
 typedef enum { SMC_F32 = 0, SMC_BF16 = 1, SMC_F16 = 2 } smc_dtype;
 
-/* Activations of the fused epilogue and of smc_group_norm. */
+/* Activations of the conv epilogue (smc_conv_ex) and of smc_group_norm. */
 typedef enum { SMC_ACT_NONE = 0, SMC_ACT_RELU = 1, SMC_ACT_SILU = 2 } smc_act;
 
 /* Pooling of smc_downsample: elementwise max, or mean over the children present. */

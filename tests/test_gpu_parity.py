@@ -420,7 +420,7 @@ def test_conv_variants_agree(name, dtype):
     smc.status()
 
 
-# ------------------------------------------------------------------ fused epilogue / GroupNorm
+# ------------------------------------------------------------------ epilogue (row pass / in the conv) and GroupNorm
 def _np_stats(x, coords, batch, groups):
     """fp64 (sum, sum of squares, count) per (item, group), summed directly."""
     n, c = x.shape
