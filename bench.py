@@ -112,14 +112,37 @@ class ClockSampler:
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{device_index}.csv")
 
     def start(self):
+        """Start sampling every 20 ms and wait (at most 3 s) for the first
+        sample, so that a short timed region that follows is covered."""
+        self.mark_at = 0
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.id}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+                 "-lms", "20"], stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < 3.0 and not self._rows():
+            time.sleep(0.01)
+
+    def mark(self):
+        """The timed region starts now: later samples are the ones reported."""
+        self.mark_at = len(self._rows())
+
+    def _rows(self):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                        rows.append(parts)
+        except OSError:
+            pass
+        return rows
 
     def stop(self):
         if self.proc is None:
@@ -130,12 +153,17 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.fh.close()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
-                    rows.append(parts)
+        return self.summary(self._rows(), self.mark_at)
+
+    @staticmethod
+    def summary(all_rows, mark_at):
+        """Median SM clock, max clock and throttle reasons of the samples
+        taken after mark_at; when the region was too short for one, the last
+        sample before it, flagged."""
+        rows = all_rows[mark_at:]
+        before = False
+        if not rows and all_rows:
+            rows, before = all_rows[-1:], True
         if not rows:
             return None
         sm = [float(r[1]) for r in rows]
@@ -145,8 +173,11 @@ class ClockSampler:
             for name, val in zip(names, r[5:9]):
                 if val.lower() == "active":
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "samples": len(rows),
-                "reasons": sorted(reasons)}
+        out = {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "samples": 0 if before else len(rows),
+               "reasons": sorted(reasons)}
+        if before:
+            out["note"] = "timed region shorter than the sampling interval: the last sample before it"
+        return out
 
 
 def tap_efficiency(perm: np.ndarray, nbr: np.ndarray, tile: int = 128) -> float:
@@ -414,6 +445,7 @@ def run_gpu(args):
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
+    clocks.mark()
     t_wall0 = time.perf_counter()
     launches_before = smc.kernel_launches()
     run = Steps()
