@@ -837,3 +837,32 @@ def test_row_pass_shuffled_items(oracle_mod, dtype, cout, groups):
     smc.group_stats(out, ct, 2, groups, st2)
     smc.status()
     np.testing.assert_allclose(st2.cpu().numpy(), _np_stats(got, coords, 2, groups), rtol=1e-9, atol=1e-6)
+
+
+def test_slab_conv_two_ranks_in_one_process():
+    """The per-rank side of z-slab sharding on the GPU: two ranks' local maps
+    (slab plus halo planes) built by the library, the halo rows copied from
+    the neighbour's boundary rows by hand (the collective is tested with gloo
+    on the CPU), two stacked bf16 layers: each rank's own rows equal the
+    unsharded conv's, bit for bit (a row's taps are summed in the same order
+    whatever tile it lands in)."""
+    from submanifold_sparse_convolution_packed_b200.shard import SlabConv
+    w = workload("shells6")
+    f, w1, b1 = _layer(w, "bf16", 0)
+    _, w2, b2 = _layer(w, "bf16", 1)
+    full = build(w)
+    ref = smc.conv(full, smc.conv(full, dev(f, "bf16"), dev(w1, "bf16"), dev(b1, "bf16")),
+                   dev(w2, "bf16"), dev(b2, "bf16"))
+    ranks = [SlabConv(w.coords, w.grid, 2, r, batch=1, device="cuda") for r in range(2)]
+    x = [r.local_features(dev(f, "bf16")) for r in ranks]
+    for wt, b in ((w1, b1), (w2, b2)):
+        lo, hi = ranks[0].plan, ranks[1].plan
+        # rank 0's top plane -> rank 1's halo below; rank 1's bottom plane -> rank 0's halo above
+        x[1][hi.n_owned:hi.n_owned + hi.halo_lo.size] = x[0][torch.from_numpy(lo.send_hi).cuda()]
+        x[0][lo.n_owned + lo.halo_lo.size:] = x[1][torch.from_numpy(hi.send_lo).cuda()]
+        x = [smc.conv(r.map, xi, dev(wt, "bf16"), dev(b, "bf16")) for r, xi in zip(ranks, x)]
+    got = torch.empty_like(ref)
+    for r, xi in zip(ranks, x):
+        got[torch.from_numpy(r.plan.owned).cuda()] = xi[:r.plan.n_owned]
+    assert torch.equal(got, ref)
+    smc.status()
