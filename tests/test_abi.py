@@ -84,3 +84,22 @@ def test_resample_argument_errors_without_gpu():
     assert lib.smc_upsample(a16, 1, None, a16, 4, 9, None, a16, P(4096), ctypes.byref(m), None, None) == -4
     assert lib.smc_upsample(P(4), 1, None, None, 0, 0, None, a16, None, ctypes.byref(m), None, None) == -11
     assert lib.smc_upsample(None, 0, None, None, 0, 0, None, None, None, ctypes.byref(m), None, None) == 0
+
+
+def test_binding_rejects_bad_tensors_without_gpu():
+    """The Python binding checks dtypes, shapes and devices before any call
+    into the library, so these raise on a CPU machine."""
+    import pytest
+    import torch
+    c = torch.zeros((4, 4), dtype=torch.int32)  # a CPU tensor
+    with pytest.raises(ValueError):
+        smc.downsample(c, (4, 4, 4))                      # not on a CUDA device
+    with pytest.raises(ValueError):
+        smc.downsample(c.float(), (4, 4, 4))              # not int32
+    with pytest.raises(ValueError):
+        smc.downsample(c, (4, 4, 4), mode="median")       # unknown pooling
+    with pytest.raises(ValueError):
+        smc.upsample(c[:, :3], None)                      # not [N, 4]
+    with pytest.raises(ValueError):
+        smc.neighbour_map_noalloc(c, (4, 4, 4))           # not on a CUDA device
+    assert set(smc.POOL_MODES) == {"max", "mean"}
