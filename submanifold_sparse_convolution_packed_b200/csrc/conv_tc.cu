@@ -40,7 +40,7 @@ constexpr int kTcThreads = 192;
 constexpr int kMaxStages = 8;
 
 struct TcSmemLayout {
-  uint32_t a_off, b_off, bar_off, misc_off, total;
+  uint32_t a_off, b_off, bar_off, misc_off, bias_off, total;
 };
 
 __host__ __device__ inline TcSmemLayout tc_layout(int stages, int bn, int kb_elems) {
@@ -51,7 +51,8 @@ __host__ __device__ inline TcSmemLayout tc_layout(int stages, int bn, int kb_ele
   L.b_off = L.a_off + stages * a_bytes;
   L.bar_off = L.b_off + stages * b_bytes;
   L.misc_off = L.bar_off + (2 * kMaxStages + 2) * 8;
-  L.total = L.misc_off + 32;
+  L.bias_off = L.misc_off + 32;  // the unit's BN bias values (bf16/fp16 bits), 16-byte aligned
+  L.total = L.bias_off + 512;
   return L;
 }
 
@@ -65,6 +66,8 @@ struct TcParams {
   int64_t n;
   int64_t ntiles;
   int cin, cout, taps, orientation, bn, nsplit, stages, is_bf16, kb_elems;
+  int bias_vec;  // bias present and 16-byte aligned: read 8 values per load
+  int stage_out;  // plain epilogue staged through the (then free) stage buffers
   uint32_t tmem_cols;
   Epilogue ep;  // activation and residual
 };
@@ -117,6 +120,37 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
     if (p.orientation < 0) mask = mirror27(mask);
   }
 
+  // The gather / epilogue warps (2-5) own tile row r: its output row v and,
+  // for k = 3, its 27 neighbour rows, loaded here so that the loads overlap
+  // the barrier set-up and the TMEM allocation below.
+  const int q = warp & 3;       // TMEM lane quarter of warps 2..5
+  const int r = q * 32 + lane;  // tile row
+  int32_t v = -1;
+  int32_t nb[kTaps];
+  // The unit's bias values go to shared memory once, so that the epilogue
+  // reads them from there: read from global memory chunk by chunk, their
+  // latency was most of the epilogue's time.
+  uint16_t* s_bias = reinterpret_cast<uint16_t*>(smem + L.bias_off);
+  if (warp >= 2 && p.bias) {
+    const int t = tid - 64;
+    const int nb_cols = p.cout - n0 < p.bn ? p.cout - n0 : p.bn;
+    if (p.bias_vec) {
+      if (8 * t < nb_cols) reinterpret_cast<uint4*>(s_bias)[t] = __ldg(reinterpret_cast<const uint4*>(p.bias + n0) + t);
+    } else {
+      for (int c = t; c < nb_cols; c += 128) s_bias[c] = __ldg(p.bias + n0 + c);
+    }
+  }
+  if (warp >= 2) {
+    const int64_t g = tile * kTileRows + r;
+    v = g < p.n ? (k3 ? __ldg(p.perm + g) : static_cast<int32_t>(g)) : -1;
+    if (v >= p.n) v = -1;  // a schedule left incomplete by a failed build is skipped, never followed
+    if (k3) {
+      const int32_t* row = p.nbr + static_cast<int64_t>(v < 0 ? 0 : v) * kTaps;
+#pragma unroll
+      for (int d = 0; d < kTaps; ++d) nb[d] = v >= 0 ? __ldg(row + (p.orientation > 0 ? d : kTaps - 1 - d)) : -1;
+    }
+  }
+
   if (tid == 0) {
     prefetch_tmap(&fmap);
     prefetch_tmap(&wmap);
@@ -149,15 +183,19 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
 
   if (warp == 0) {
     // ---------------------------------------------------------- weight loader
-    if (lane == 0) {
+    // The whole warp runs the loop (warp-uniform values); lane 0 waits, the
+    // warp agrees on the outcome, and one elected lane issues the loads.
+    {
       uint32_t it = 0;
       bool ok = true;
       for (uint32_t m = mask; m && ok; m &= m - 1) {
         const int d = __ffs(m) - 1;
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const uint32_t stage = it % p.stages, phase = (it / p.stages) & 1u;
-          if (!mbar_wait_bounded(bar_empty + 8 * stage, phase ^ 1u, p.err) || s_misc[1]) {
-            s_misc[1] = 1;
+          int w_ok = 1;
+          if (lane == 0) w_ok = mbar_wait_bounded(bar_empty + 8 * stage, phase ^ 1u, p.err) && !s_misc[1];
+          if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
+            if (lane == 0) s_misc[1] = 1;
             ok = false;
             break;
           }
@@ -165,22 +203,28 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
           const uint32_t a_dst = sbase + L.a_off + stage * a_bytes, b_dst = sbase + L.b_off + stage * b_bytes;
           const int32_t a_row = static_cast<int32_t>(tile * kTileRows);
           const int32_t b_row = n0 + static_cast<int32_t>(rank) * bn_cta;
-          if (kPair) {
-            mbar_arrive_expect_tx_cluster(full, b_bytes + (k3 ? 0u : a_bytes));
-            if (!k3) tma_load_2d_pair(a_dst, &fmap, full, kb * p.kb_elems, a_row);
-            tma_load_3d_pair(b_dst, &wmap, full, kb * p.kb_elems, k3 ? d : 0, b_row);
-          } else {
-            mbar_arrive_expect_tx(full, b_bytes + (k3 ? 0u : a_bytes));
-            if (!k3) tma_load_2d(a_dst, &fmap, full, kb * p.kb_elems, a_row);
-            tma_load_3d(b_dst, &wmap, full, kb * p.kb_elems, k3 ? d : 0, b_row);
+          if (elect_one()) {
+            if (kPair) {
+              mbar_arrive_expect_tx_cluster(full, b_bytes + (k3 ? 0u : a_bytes));
+              if (!k3) tma_load_2d_pair(a_dst, &fmap, full, kb * p.kb_elems, a_row);
+              tma_load_3d_pair(b_dst, &wmap, full, kb * p.kb_elems, k3 ? d : 0, b_row);
+            } else {
+              mbar_arrive_expect_tx(full, b_bytes + (k3 ? 0u : a_bytes));
+              if (!k3) tma_load_2d(a_dst, &fmap, full, kb * p.kb_elems, a_row);
+              tma_load_3d(b_dst, &wmap, full, kb * p.kb_elems, k3 ? d : 0, b_row);
+            }
           }
+          __syncwarp();
         }
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    // (for a pair only the even CTA issues; the odd one only holds TMEM)
-    if (lane == 0 && rank == 0) {
+    // The whole warp runs the loop with warp-uniform values and one elected
+    // lane issues each MMA and commit: measured on B200, a lone thread in a
+    // lane-divergent branch issues MMAs about half as fast.  (For a pair only
+    // the even CTA issues; the odd one only holds TMEM.)
+    if (rank == 0) {
       const uint32_t idesc =
           idesc_f16(static_cast<uint32_t>(p.is_bf16), static_cast<uint32_t>(p.bn), kPair ? 256u : 128u);
       uint32_t it = 0;
@@ -188,8 +232,9 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
       for (uint32_t m = mask; m && ok; m &= m - 1) {
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const uint32_t stage = it % p.stages, phase = (it / p.stages) & 1u;
-          if (!mbar_wait_bounded(bar_full + 8 * stage, phase, p.err) || s_misc[1]) {
-            s_misc[1] = 1;
+          const bool w_ok = mbar_wait_bounded(bar_full + 8 * stage, phase, p.err);
+          if (!__all_sync(0xffffffffu, w_ok && !s_misc[1])) {
+            if (lane == 0) s_misc[1] = 1;
             ok = false;
             break;
           }
@@ -198,23 +243,20 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
           const uint64_t bdesc = kmajor_desc(sbase + L.b_off + stage * b_bytes, row_bytes);
           const int ksteps = kb == kblocks - 1 ? last_ksteps : p.kb_elems / 16;
           for (int k = 0; k < ksteps; ++k) {
-            if (kPair) umma_f16_pair(tmem_base, adesc + 2 * k, bdesc + 2 * k, idesc, (it > 0 || k > 0) ? 1u : 0u);
-            else umma_f16(tmem_base, adesc + 2 * k, bdesc + 2 * k, idesc, (it > 0 || k > 0) ? 1u : 0u);
+            if (kPair)
+              umma_f16_pair_elect(tmem_base, adesc + 2 * k, bdesc + 2 * k, idesc, (it > 0 || k > 0) ? 1u : 0u);
+            else
+              umma_f16_elect(tmem_base, adesc + 2 * k, bdesc + 2 * k, idesc, (it > 0 || k > 0) ? 1u : 0u);
           }
-          if (kPair) umma_commit_pair(bar_empty + 8 * stage, 3);
-          else umma_commit(bar_empty + 8 * stage);
+          if (kPair) umma_commit_pair_elect(bar_empty + 8 * stage, 3);
+          else umma_commit_elect(bar_empty + 8 * stage);
         }
       }
-      if (kPair) umma_commit_pair(bar_acc, 3);
-      else umma_commit(bar_acc);
+      if (kPair) umma_commit_pair_elect(bar_acc, 3);
+      else umma_commit_elect(bar_acc);
     }
   } else {
-    // Gather / epilogue warps: this thread's tile row and its neighbour rows.
-    const int q = warp & 3;       // TMEM lane quarter of warps 2..5
-    const int r = q * 32 + lane;  // tile row
-    const int64_t g = tile * kTileRows + r;
-    int32_t v = g < p.n ? (k3 ? __ldg(p.perm + g) : static_cast<int32_t>(g)) : -1;
-    if (v >= p.n) v = -1;  // a schedule left incomplete by a failed build is skipped, never followed
+    // Gather / epilogue warps: this thread's tile row v and its neighbour rows nb.
     if constexpr (kEpi >= 1) {
       // the epilogue reads this row's residual: bring it into L2 now, while
       // the tile's taps are gathered and multiplied
@@ -226,10 +268,6 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
     }
     // ---------------------------------------------------------- A gather (k=3)
     if (k3) {
-      int32_t nb[kTaps];
-      const int32_t* row = p.nbr + static_cast<int64_t>(v < 0 ? 0 : v) * kTaps;
-#pragma unroll
-      for (int d = 0; d < kTaps; ++d) nb[d] = v >= 0 ? __ldg(row + (p.orientation > 0 ? d : kTaps - 1 - d)) : -1;
       uint32_t it = 0;
       bool ok = true;
 #pragma unroll
@@ -274,21 +312,75 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
     // ready (while the last MMAs run) and each later chunk's one chunk ahead;
     // a thread reads and writes only its own row, and loads a column before
     // storing it, so this holds for a residual that is the output buffer.
-    auto load_res = [&](int c0, uint4 (&r)[4]) {
+    auto load_res = [&](int c0, uint4 (&rq)[4]) {
       int nc = p.bn - c0 < 32 ? p.bn - c0 : 32;
       if (p.cout - (n0 + c0) < nc) nc = p.cout - (n0 + c0);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        r[j] = make_uint4(0, 0, 0, 0);
+        rq[j] = make_uint4(0, 0, 0, 0);
         if (extra && res && v >= 0 && 8 * j < nc)
-          r[j] = *reinterpret_cast<const uint4*>(res + static_cast<int64_t>(v) * p.cout + n0 + c0 + 8 * j);
+          rq[j] = *reinterpret_cast<const uint4*>(res + static_cast<int64_t>(v) * p.cout + n0 + c0 + 8 * j);
       }
     };
     uint4 rcur[4], rnext[4];
     if constexpr (extra) load_res(0, rcur);
     const bool ready = mbar_wait_bounded(bar_acc, 0, p.err) && !s_misc[1];
     tc_fence_after();
-    if (ready) {
+    if (!extra && ready && p.stage_out) {
+      // Plain epilogue through shared memory: the accumulator is complete, so
+      // every MMA has consumed its operands and the stage buffers are free.
+      // Each warp converts its 32 rows (bias in fp32, rounding) into its own
+      // padded row block, then writes whole output rows with coalesced
+      // 16-byte stores (a row's bytes are contiguous in `out`), instead of 32
+      // scattered rows per store instruction.
+      const bool bf = p.is_bf16 != 0;
+      const uint32_t pitch = static_cast<uint32_t>(p.bn) * 2u + 16u;
+      uint8_t* blk = smem + L.a_off + static_cast<uint32_t>(q) * 32u * pitch;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      int ncols_all = p.cout - n0 < p.bn ? p.cout - n0 : p.bn;
+      for (int c0 = 0; c0 < ncols_all; c0 += 32) {
+        float acc[32];
+        tmem_ld_32cols(t_row + c0, acc);
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+          if (c0 + j >= ncols_all) break;
+          float bv[8];
+          if (p.bias) {
+            const uint4 bq = *reinterpret_cast<const uint4*>(s_bias + c0 + j);
+            const uint32_t bw[4] = {bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              bv[2 * e] = half_bits_to_float(static_cast<uint16_t>(bw[e] & 0xFFFFu), bf);
+              bv[2 * e + 1] = half_bits_to_float(static_cast<uint16_t>(bw[e] >> 16), bf);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) bv[e] = 0.f;
+          }
+          uint32_t packed[4];
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            const uint16_t h0 = float_to_half_bits(acc[j + e] + bv[e], bf);
+            const uint16_t h1 = float_to_half_bits(acc[j + e + 1] + bv[e + 1], bf);
+            packed[e / 2] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+          }
+          *reinterpret_cast<uint4*>(blk + lane * pitch + (c0 + j) * 2) =
+              make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        }
+      }
+      __syncwarp();
+      // copy out: `cpr` 16-byte chunks per row, 32 / cpr rows per pass
+      const int cpr = ncols_all / 8;
+      const int rpp = 32 / cpr > 0 ? 32 / cpr : 1;
+      for (int r0 = 0; r0 < 32; r0 += rpp) {
+        const int rr = r0 + lane / cpr, ch = lane % cpr;
+        const int32_t vr = __shfl_sync(0xffffffffu, v, rr < 32 ? rr : 31);
+        if (lane < rpp * cpr && rr < 32 && vr >= 0) {
+          const uint4 x = *reinterpret_cast<const uint4*>(blk + rr * pitch + ch * 16);
+          *reinterpret_cast<uint4*>(p.out + static_cast<int64_t>(vr) * p.cout + n0 + ch * 8) = x;
+        }
+      }
+    } else if (ready) {
       const bool bf = p.is_bf16 != 0;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
       for (int c0 = 0; c0 < p.bn; c0 += 32) {
@@ -312,14 +404,24 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
               rw[2] = rcur[j / 8].z;
               rw[3] = rcur[j / 8].w;
             }
+            // the 8 bias values of these columns, from shared memory
+            float bv[8];
+            if (p.bias) {
+              const uint4 bq = *reinterpret_cast<const uint4*>(s_bias + c0 + j);
+              const uint32_t bw[4] = {bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                bv[2 * e] = half_bits_to_float(static_cast<uint16_t>(bw[e] & 0xFFFFu), bf);
+                bv[2 * e + 1] = half_bits_to_float(static_cast<uint16_t>(bw[e] >> 16), bf);
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) bv[e] = 0.f;
+            }
             uint32_t packed[4];
 #pragma unroll
             for (int e = 0; e < 8; e += 2) {
-              float x0 = acc[j + e], x1 = acc[j + e + 1];
-              if (p.bias) {
-                x0 += half_bits_to_float(__ldg(p.bias + col + e), bf);
-                x1 += half_bits_to_float(__ldg(p.bias + col + e + 1), bf);
-              }
+              float x0 = acc[j + e] + bv[e], x1 = acc[j + e + 1] + bv[e + 1];
               if constexpr (extra) {
                 x0 = apply_act(x0, p.ep.act);
                 x1 = apply_act(x1, p.ep.act);
@@ -476,6 +578,15 @@ cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s) {
   p.perm = a.perm;
   p.tile_mask = a.tile_mask;
   p.bias = static_cast<const uint16_t*>(a.bias);
+  p.bias_vec = a.bias && aligned16(a.bias) ? 1 : 0;
+  {
+    // the staged epilogue needs 4 warps x 32 rows x (row bytes + 16) of the
+    // stage buffers (A and B regions, contiguous); rows hold at most 32 chunks
+    const uint32_t need = 4u * 32u * (static_cast<uint32_t>(t.bn) * 2u + 16u);
+    const uint32_t have =
+        static_cast<uint32_t>(t.stages) * (static_cast<uint32_t>(kTileRows + t.bn) * t.kb_elems * 2u);
+    p.stage_out = !t.pair && need <= have ? 1 : 0;
+  }
   p.out = static_cast<uint16_t*>(a.out);
   p.err = a.err;
   p.n = a.n;
