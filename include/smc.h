@@ -394,10 +394,12 @@ SMC_API const char* smc_strerror(int code);
  *          the error word (SMC_E_RANGE, SMC_E_DUPLICATE as for smc_build_map).
  *
  * Scratch: one file-scope device array of about 9.5 MB, which every GPU that
- * loads the library holds until the process exits; no cudaMalloc, cudaFree or
- * other allocating call is made.  The first call on a device looks up the
- * array's device address (cudaGetSymbolAddress) with that device current;
- * make that first call before any stream capture.  Every call shares the
+ * loads the library holds until the process exits; no cudaMalloc or other
+ * allocating call is made.  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current and caches
+ * it with the device's current context; make that first call before any
+ * stream capture.  After cudaDeviceReset (a new context) the next call looks
+ * the address up again, so it too should come before any capture.  Every call shares the
  * array and clears what it reads; calls whose work overlaps on the GPU
  * (different streams or host threads) race on it and must be serialised by
  * the caller.  No pair lists or tile schedule are produced.
@@ -420,6 +422,27 @@ SMC_API int smc_set_conv_variant(int32_t variant);
  *   value. */
 SMC_API int smc_set_conv_epilogue(int32_t where);
 SMC_API int smc_set_map_lookup(int32_t mode);
+
+/*
+ * Failure-path test hooks (host side: no GPU fault is involved).
+ * smc_set_alloc_fail_after: k >= 1 makes the k-th device allocation the
+ *   library asks its pool for, counted from this call, report failure once;
+ *   the entry point that asked returns SMC_E_OOM, leaves its handle output
+ *   NULL and releases whatever it had allocated.  0 disarms the hook.
+ *   SMC_E_ARG for k < 0.
+ * smc_set_wait_limit_ns: bound, in nanoseconds, of the single-pass scans'
+ *   device-side waits on earlier segments (every build, subdivision,
+ *   upsample and downsample runs such scans); 0 restores the default 2 s.
+ *   SMC_E_ARG for ns < 0.
+ * smc_set_scan_hold: in every later scan, the segment with this ticket
+ *   (0-based, in start order) publishes nothing, so the waits of the
+ *   segments after it run out and the call reports SMC_E_TIMEOUT; every
+ *   access stays in bounds and the device stays usable.  -1 (default) turns
+ *   it off; SMC_E_ARG below -1.  Meant for use with a short wait limit.
+ */
+SMC_API int smc_set_alloc_fail_after(int64_t k);
+SMC_API int smc_set_wait_limit_ns(int64_t ns);
+SMC_API int smc_set_scan_hold(int64_t ticket);
 
 #ifdef __cplusplus
 }

@@ -32,6 +32,7 @@ EXPORTS = [
     "smc_build_map_async", "smc_map_wait", "smc_neighbour_map_noalloc", "smc_set_conv_variant",
     "smc_set_map_lookup", "smc_map_stream_wait", "smc_subdivide", "smc_conv_ex", "smc_group_stats",
     "smc_group_norm", "smc_downsample", "smc_upsample", "smc_set_conv_epilogue",
+    "smc_set_alloc_fail_after", "smc_set_wait_limit_ns", "smc_set_scan_hold",
 ]
 
 
@@ -83,6 +84,9 @@ def lib() -> ctypes.CDLL:
         L.smc_set_conv_variant.argtypes = [i32]
         L.smc_set_conv_epilogue.argtypes = [i32]
         L.smc_set_map_lookup.argtypes = [i32]
+        L.smc_set_alloc_fail_after.argtypes = [i64]
+        L.smc_set_wait_limit_ns.argtypes = [i64]
+        L.smc_set_scan_hold.argtypes = [i64]
         for name in EXPORTS:
             if name != "smc_strerror":
                 getattr(L, name).restype = ctypes.c_int
@@ -502,6 +506,23 @@ def set_conv_variant(variant: int) -> None:
 def set_map_lookup(mode: int) -> None:
     """Lookup structure of later builds: 0 by size, 1 hash table, 2 dense grid."""
     _check(lib().smc_set_map_lookup(int(mode)), "smc_set_map_lookup")
+
+
+def set_alloc_fail_after(k: int) -> None:
+    """Test hook: the k-th device allocation of the library from now on
+    reports failure, once (0 disarms it; smc_set_alloc_fail_after)."""
+    _check(lib().smc_set_alloc_fail_after(int(k)), "smc_set_alloc_fail_after")
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Bound of the scans' device-side waits, in ns (0 = the default 2 s)."""
+    _check(lib().smc_set_wait_limit_ns(int(ns)), "smc_set_wait_limit_ns")
+
+
+def set_scan_hold(ticket: int) -> None:
+    """Test hook: the scan segment with this ticket publishes nothing, so the
+    later segments' waits run out (-1 turns it off; smc_set_scan_hold)."""
+    _check(lib().smc_set_scan_hold(int(ticket)), "smc_set_scan_hold")
 
 
 def set_hash_capacity(slots: int) -> None:

@@ -53,6 +53,10 @@ struct smc_map {
 namespace {
 
 std::atomic<int64_t> g_capacity_override{0};
+// Test hooks of the failure paths (smc_set_alloc_fail_after, smc_set_wait_limit_ns, smc_set_scan_hold).
+std::atomic<int64_t> g_alloc_fail_after{0};
+std::atomic<int64_t> g_wait_limit_ns{static_cast<int64_t>(smc::kWaitLimitNs)};
+std::atomic<int64_t> g_scan_hold{-1};
 std::atomic<long long> g_launches{0};
 std::atomic<int32_t> g_profiling{0};
 std::atomic<int32_t> g_map_lookup{0};
@@ -171,6 +175,23 @@ void give_slot(HostSlot* s) {
   if (!s) return;
   std::lock_guard<std::mutex> lk(g_slot_mu);
   g_free_slots.push_back(s);
+}
+
+// Every device allocation of the library goes through here: stream-ordered,
+// from the library's pool.  When smc_set_alloc_fail_after(k) is armed, the
+// k-th allocation from then on reports failure instead (once), which is how
+// the SMC_E_OOM paths are exercised without exhausting a GPU.
+cudaError_t pool_alloc(void** p, size_t bytes, cudaMemPool_t pool, cudaStream_t s) {
+  *p = nullptr;
+  if (!pool) return cudaErrorMemoryAllocation;
+  int64_t k = g_alloc_fail_after.load();
+  while (k > 0) {
+    if (g_alloc_fail_after.compare_exchange_weak(k, k - 1)) {
+      if (k == 1) return cudaErrorMemoryAllocation;
+      break;
+    }
+  }
+  return cudaMallocFromPoolAsync(p, bytes, pool, s);
 }
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -355,7 +376,7 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   const size_t zero_bytes = tmp.off - o_err;
 
   void* tp = nullptr;
-  if (cudaMallocFromPoolAsync(&m->keep, keep.off, pool, s) != cudaSuccess) {
+  if (pool_alloc(&m->keep, keep.off, pool, s) != cudaSuccess) {
     cudaGetLastError();
     m->keep = nullptr;
     give_event(m->device, ev_fork);
@@ -363,7 +384,7 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
     release_map(m);
     return SMC_E_OOM;
   }
-  if (cudaMallocFromPoolAsync(&tp, tmp.off, pool, s) != cudaSuccess) {
+  if (pool_alloc(&tp, tmp.off, pool, s) != cudaSuccess) {
     cudaGetLastError();
     give_event(m->device, ev_fork);
     give_event(m->device, ev_sched);
@@ -477,7 +498,7 @@ int stats_begin(int dev, cudaStream_t s, int batch, int groups, double** copies)
   const size_t bytes = static_cast<size_t>(kStatStripes) * batch * groups * 3 * sizeof(double);
   cudaMemPool_t pool = device_pool(dev);
   void* p = nullptr;
-  if (!pool || cudaMallocFromPoolAsync(&p, bytes, pool, s) != cudaSuccess) {
+  if (pool_alloc(&p, bytes, pool, s) != cudaSuccess) {
     cudaGetLastError();
     return SMC_E_OOM;
   }
@@ -505,6 +526,8 @@ int stats_end(double* copies, int batch, int groups, double* stats, cudaStream_t
 
 namespace smc {
 void count_launches(int k) { g_launches.fetch_add(k, std::memory_order_relaxed); }
+uint64_t scan_wait_limit_ns() { return static_cast<uint64_t>(g_wait_limit_ns.load()); }
+int64_t scan_hold_ticket() { return g_scan_hold.load(); }
 }  // namespace smc
 
 extern "C" {
@@ -530,6 +553,24 @@ const char* smc_strerror(int code) {
 int smc_set_hash_capacity(int64_t slots) {
   if (slots < 0) return SMC_E_ARG;
   g_capacity_override.store(slots);
+  return SMC_OK;
+}
+
+int smc_set_alloc_fail_after(int64_t k) {
+  if (k < 0) return SMC_E_ARG;
+  g_alloc_fail_after.store(k);
+  return SMC_OK;
+}
+
+int smc_set_wait_limit_ns(int64_t ns) {
+  if (ns < 0) return SMC_E_ARG;
+  g_wait_limit_ns.store(ns == 0 ? static_cast<int64_t>(smc::kWaitLimitNs) : ns);
+  return SMC_OK;
+}
+
+int smc_set_scan_hold(int64_t ticket) {
+  if (ticket < -1) return SMC_E_ARG;
+  g_scan_hold.store(ticket);
   return SMC_OK;
 }
 
@@ -609,7 +650,7 @@ static int spawn_children(const smc_map* parent, const int32_t* coords, int64_t 
   const size_t o_remap = c.take<int32_t>(8 * n);
   const size_t o_src = c.take<int32_t>(8 * n);
   void* sp = nullptr;
-  if (cudaMallocFromPoolAsync(&sp, c.off, pool, s) != cudaSuccess) {
+  if (pool_alloc(&sp, c.off, pool, s) != cudaSuccess) {
     cudaGetLastError();
     give_slot(slot);
     return SMC_E_OOM;
@@ -759,7 +800,7 @@ int smc_downsample(const int32_t* coords, int64_t n, int32_t batch, const int32_
   const size_t o_rows = cv.take<int32_t>(8 * n);
   const size_t o_pbits = cv.take<uint8_t>(n);
   void* sp = nullptr;
-  if (cudaMallocFromPoolAsync(&sp, cv.off, pool, s) != cudaSuccess) {
+  if (pool_alloc(&sp, cv.off, pool, s) != cudaSuccess) {
     cudaGetLastError();
     give_slot(slot);
     return SMC_E_OOM;
@@ -870,6 +911,8 @@ int smc_map_stream_wait(const smc_map* map, void* stream) {
 
 int smc_build_map(const int32_t* coords, int64_t n, int32_t batch, const int32_t grid[3], void* stream,
                   smc_map** out) {
+  if (!out) return SMC_E_ARG;
+  *out = nullptr;
   smc_map* m = nullptr;
   int rc = build_async(coords, n, batch, grid, static_cast<cudaStream_t>(stream), &m);
   if (rc != SMC_OK) return rc;
@@ -964,7 +1007,7 @@ int smc_conv_ex(const smc_map* map, const void* feats, int64_t cin, const void* 
   if (per_offset) {
     void* acc = nullptr;
     cudaMemPool_t pool = device_pool(dev);
-    if (!pool || cudaMallocFromPoolAsync(&acc, static_cast<size_t>(n) * cout * sizeof(float), pool, s) != cudaSuccess) {
+    if (pool_alloc(&acc, static_cast<size_t>(n) * cout * sizeof(float), pool, s) != cudaSuccess) {
       cudaGetLastError();
       return SMC_E_OOM;
     }

@@ -59,6 +59,10 @@ int map_nblocks(int64_t n);
 int radix_nblocks(int64_t n);
 int radix_bins();
 int64_t scan_status_len(int64_t L);
+// Bound of the look-back scans' waits on their predecessors (2 s unless a
+// test sets it) and the test hook that holds one scan segment back (-1 = none).
+uint64_t scan_wait_limit_ns();
+int64_t scan_hold_ticket();
 
 // Hash insert + neighbour lookups (map, schedule keys, block counts, first
 // radix histogram), then, on any stream ordered after them, the pair lists.

@@ -517,8 +517,10 @@ __device__ __forceinline__ int64_t block_exclusive_scan(int64_t x, int64_t* s_wa
 // own inclusive prefix.  Statuses are one word each: flag (aggregate /
 // prefix) in bits 63..62, value below, so no fence orders them.  A block waits
 // only on segments with smaller tickets, which are resident and running, so
-// every wait ends; it is still bounded (kWaitLimitNs), after which the error
-// word gets kErrTimeout and the offsets are not to be trusted.
+// every wait ends; it is still bounded (wait_ns, 2 s unless a test sets it),
+// after which the error word gets kErrTimeout and the offsets are not to be
+// trusted.  The segment whose ticket is `hold` (a test hook; -1 = none)
+// publishes nothing, so the waits of the segments after it run out.
 //
 // When `info` is given, the offsets at positions d * stride (d < 27) -- the
 // starts of the per-offset pair lists -- and the grand total go to info[0..27].
@@ -526,7 +528,7 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_lookback(const int32_t* _
                                                                 int64_t* __restrict__ out,
                                                                 unsigned long long* status, uint32_t* ticket,
                                                                 uint32_t* err, int64_t* __restrict__ info,
-                                                                int64_t stride) {
+                                                                int64_t stride, uint64_t wait_ns, int64_t hold) {
   __shared__ int64_t s_warp[32];
   __shared__ int64_t s_t;
   __shared__ int s_first;
@@ -550,7 +552,7 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_lookback(const int32_t* _
   }
   int64_t tot;
   const int64_t mine = block_exclusive_scan(sum, s_warp, &tot);
-  if (tid == 0)
+  if (tid == 0 && t != hold)
     st_relaxed_gpu(&status[t], (t == 0 ? kFlagPrefix : kFlagAggregate) | static_cast<unsigned long long>(tot));
   int64_t excl = 0;
   if (t > 0) {
@@ -567,7 +569,7 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_lookback(const int32_t* _
         // a predecessor up to that prefix has not published yet: read again
         if (tid == 0) {
           s_first = kScanThreads;
-          if (globaltimer_ns() - t_start > kWaitLimitNs) {
+          if (globaltimer_ns() - t_start > wait_ns) {
             atomicOr(err, kErrTimeout);
             s_abort = 1;
           }
@@ -582,7 +584,7 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_lookback(const int32_t* _
       if (first < kScanThreads) break;
       top -= kScanThreads;
     }
-    if (tid == 0) st_relaxed_gpu(&status[t], kFlagPrefix | static_cast<unsigned long long>(excl + tot));
+    if (tid == 0 && t != hold) st_relaxed_gpu(&status[t], kFlagPrefix | static_cast<unsigned long long>(excl + tot));
   }
   int64_t run = excl + mine;
 #pragma unroll
@@ -700,7 +702,8 @@ static cudaError_t scan_i32(const int32_t* in, int64_t L, int64_t* out, unsigned
   const int64_t nseg = (L + kScanSeg - 1) / kScanSeg;
   if (nseg == 0) return cudaSuccess;
   k_scan_lookback<<<static_cast<unsigned>(nseg), kScanThreads, 0, s>>>(in, L, out, status, ticket, err, info,
-                                                                       stride);
+                                                                       stride, scan_wait_limit_ns(),
+                                                                       scan_hold_ticket());
   count_launches(1);
   return cudaGetLastError();
 }

@@ -13,10 +13,14 @@
 //
 // The array's name is a host-side stand-in in host code, not a device
 // address; the first call on each device looks the address up with
-// cudaGetSymbolAddress while that device is current and caches it.  All calls
-// share the one array and it keeps the last call's contents, so the table and
-// the error word are cleared on every call, and calls whose work overlaps on
-// the GPU (different streams, or several host threads) race with each other.
+// cudaGetSymbolAddress while that device is current and caches it together
+// with the device's current context.  A call that finds another context
+// current (after cudaDeviceReset, or a re-created primary context) looks the
+// address up again, so a cached address never outlives its context.  All
+// calls share the one array and it keeps the last call's contents, so the
+// table and the error word are cleared on every call, and calls whose work
+// overlaps on the GPU (different streams, or several host threads) race with
+// each other.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -44,20 +48,46 @@ static __device__ __align__(256) NoAllocScratch g_noalloc_scratch;
 
 constexpr int kMaxDevices = 64;
 NoAllocScratch* g_scratch_addr[kMaxDevices] = {};
+void* g_scratch_ctx[kMaxDevices] = {};  // the context the cached address belongs to
 std::mutex g_scratch_mu;
 
-// Device address of the scratch array on `dev` (the current device), looked
-// up once per device.
+// The driver's cuCtxGetCurrent, reached through the runtime (the library
+// links only the CUDA runtime).
+using CtxGetCurrentFn = int (*)(void**);
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// Device address of the scratch array on `dev` (the current device): looked
+// up once per device and context, and again whenever the current context is
+// not the one the cached address was found in.
 NoAllocScratch* scratch_on(int dev) {
   if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  CtxGetCurrentFn get_ctx = ctx_get_current();
+  if (!get_ctx) return nullptr;
+  void* ctx = nullptr;  // null before the runtime has made the device's context current
+  if (get_ctx(&ctx) != 0) return nullptr;
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  if (!ctx || !g_scratch_addr[dev] || g_scratch_ctx[dev] != ctx) {
+    g_scratch_addr[dev] = nullptr;
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
       cudaGetLastError();
       return nullptr;
     }
+    if (get_ctx(&ctx) != 0 || !ctx) return nullptr;  // current now: the lookup needed it
     g_scratch_addr[dev] = static_cast<NoAllocScratch*>(ptr);
+    g_scratch_ctx[dev] = ctx;
   }
   return g_scratch_addr[dev];
 }

@@ -309,7 +309,7 @@ def test_conv_shells6_bf16(oracle_mod, orientation, conv_variant):
     check_close(got, ref, "bf16", f"shells6 s={orientation}")
 
 
-def test_conv_full128_bf16_sampled(oracle_mod):
+def test_conv_full128_bf16_sampled(oracle_mod, conv_variant):
     w = workload("full128")
     m = build(w)
     f, wt, b = _layer(w, "bf16")
@@ -421,17 +421,6 @@ def test_conv_variants_agree(name, dtype):
 
 
 # ------------------------------------------------------------------ epilogue (row pass / in the conv) and GroupNorm
-def _np_stats(x, coords, batch, groups):
-    """fp64 (sum, sum of squares, count) per (item, group), summed directly."""
-    n, c = x.shape
-    xg = x.reshape(n, groups, c // groups)
-    st = np.zeros((batch, groups, 3))
-    for b in range(batch):
-        r = xg[coords[:, 0] == b]
-        st[b, :, 0], st[b, :, 1], st[b, :, 2] = r.sum(axis=(0, 2)), (r * r).sum(axis=(0, 2)), r.shape[0] * (c // groups)
-    return st
-
-
 @pytest.fixture(params=[0, 1], ids=["row_pass", "in_conv"])
 def conv_epilogue(request):
     """Runs a test with the tensor-core conv's activation and residual applied
@@ -467,7 +456,7 @@ def test_conv_ex_epilogue(oracle_mod, dtype, variant, act, conv_epilogue):
     ref = oracle_mod.activation(oracle_mod.conv(w.coords, w.grid, f, wt, b, 3, 1, threads=THREADS),
                                 {None: 0, "relu": 1, "silu": 2}[act]) + res
     check_close(got, ref, dtype, f"conv_ex {dtype} v{variant} act={act}")
-    np.testing.assert_allclose(stats.cpu().numpy(), _np_stats(got, w.coords, 2, 32), rtol=1e-9, atol=1e-6)
+    np.testing.assert_allclose(stats.cpu().numpy(), oracle_mod.group_stats(got, w.coords, 2, 32), rtol=1e-9, atol=1e-6)
 
 
 def test_conv_ex_residual_in_place(oracle_mod, conv_epilogue):
@@ -492,7 +481,7 @@ def test_group_norm(oracle_mod, dtype):
     beta = S.round_to(rng.standard_normal(64).astype(np.float32), dtype)
     coords = torch.from_numpy(w.coords).cuda()
     st = smc.group_stats(dev(x, dtype), coords, 2, 32)
-    np.testing.assert_allclose(st.cpu().numpy(), _np_stats(x.astype(np.float64), w.coords, 2, 32), rtol=1e-9, atol=1e-6)
+    np.testing.assert_allclose(st.cpu().numpy(), oracle_mod.group_stats(x.astype(np.float64), w.coords, 2, 32), rtol=1e-9, atol=1e-6)
     out = smc.group_norm(dev(x, dtype), coords, 2, 32, st, dev(gamma, dtype), dev(beta, dtype), 1e-5, act="silu")
     smc.status()
     ref = oracle_mod.group_norm(x, w.coords, 2, 32, gamma, beta, 1e-5, act=2)
@@ -517,7 +506,7 @@ def test_resblock_chain(oracle_mod, conv_epilogue):
     st1 = torch.zeros((2, 32, 3), dtype=torch.float64, device="cuda")
     h1 = smc.conv(m, h, dev(w1, "bf16"), dev(b1, "bf16"), coords=coords, stats=st1, groups=32)
     check_close(host(h1), oracle_mod.conv(w.coords, w.grid, host(h), w1, b1, 3, 1, threads=THREADS), "bf16", "conv1")
-    np.testing.assert_allclose(st1.cpu().numpy(), _np_stats(host(h1), w.coords, 2, 32), rtol=1e-9, atol=1e-6)
+    np.testing.assert_allclose(st1.cpu().numpy(), oracle_mod.group_stats(host(h1), w.coords, 2, 32), rtol=1e-9, atol=1e-6)
     h2 = smc.group_norm(h1, coords, 2, 32, st1, act="silu")
     check_close(host(h2), oracle_mod.group_norm(host(h1), w.coords, 2, 32, act=2), "bf16", "gn2")
     y = smc.conv(m, h2, dev(w2, "bf16"), dev(b2, "bf16"), residual=xt)
@@ -832,11 +821,11 @@ def test_row_pass_shuffled_items(oracle_mod, dtype, cout, groups):
     rows = sample_rows(w.n, 4096, 53)
     ref = oracle_mod.activation(oracle_mod.conv(coords, w.grid, f, wt, b, 3, 1, rows=rows, threads=THREADS), 2)
     check_close(got[rows], ref + res[rows], dtype, f"row pass {dtype} {cout}")
-    np.testing.assert_allclose(stats.cpu().numpy(), _np_stats(got, coords, 2, groups), rtol=1e-9, atol=1e-6)
+    np.testing.assert_allclose(stats.cpu().numpy(), oracle_mod.group_stats(got, coords, 2, groups), rtol=1e-9, atol=1e-6)
     st2 = torch.zeros_like(stats)
     smc.group_stats(out, ct, 2, groups, st2)
     smc.status()
-    np.testing.assert_allclose(st2.cpu().numpy(), _np_stats(got, coords, 2, groups), rtol=1e-9, atol=1e-6)
+    np.testing.assert_allclose(st2.cpu().numpy(), oracle_mod.group_stats(got, coords, 2, groups), rtol=1e-9, atol=1e-6)
 
 
 def test_slab_conv_two_ranks_in_one_process():

@@ -61,6 +61,35 @@ def test_noalloc_matches_build_map_twice():
                                   _reference(w.coords, w.grid, batch))
 
 
+def test_noalloc_matches_oracle(oracle_mod):
+    """Bit for bit against the CPU oracle's neighbour map, not only against
+    the other GPU entry point."""
+    for name in ("tiny", "shell2"):
+        w = S.workload(name)
+        batch = int(w.coords[:, 0].max()) + 1
+        got = _noalloc_via_cabi(w.coords, list(w.grid), batch)
+        np.testing.assert_array_equal(got, oracle_mod.neighbour_map(w.coords, w.grid))
+
+
+def test_noalloc_out_of_range_row():
+    """A coordinate outside the box is reported as SMC_E_RANGE and its row of
+    the map is left all -1 (it is never a neighbour of anything)."""
+    w = S.workload("tiny")
+    coords = w.coords.copy()
+    bad = 7
+    coords[bad, 3] = w.grid[2]  # x one past the last plane
+    c = torch.from_numpy(coords).cuda()
+    out = torch.full((coords.shape[0], 27), -7, dtype=torch.int32, device="cuda")
+    g = (ctypes.c_int32 * 3)(*w.grid)
+    rc = smc.lib().smc_neighbour_map_noalloc(ctypes.c_void_p(c.data_ptr()), coords.shape[0], 1, g,
+                                             ctypes.c_void_p(out.data_ptr()), None)
+    assert rc == -2  # SMC_E_RANGE
+    got = out.cpu().numpy()
+    assert (got[bad] == -1).all()
+    assert not (got == bad).any()
+    assert ((got >= -1) & (got < coords.shape[0])).all()
+
+
 def test_noalloc_limits_and_errors():
     lib = smc.lib()
     g = (ctypes.c_int32 * 3)(8, 8, 8)
