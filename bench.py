@@ -24,9 +24,11 @@ import argparse
 import hashlib
 import json
 import os
+import platform
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -95,7 +97,8 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """nvidia-smi clock / throttle sampling during the timed region (samples
+    go to a temporary file that is removed when sampling stops)."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -109,14 +112,15 @@ class ClockSampler:
             self.id = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
         except Exception:
             self.id = str(device_index)
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{device_index}.csv")
+        fd, self.path = tempfile.mkstemp(prefix=f"smc_clocks_{device_index}_", suffix=".csv")
+        os.close(fd)
 
     def start(self):
         """Start sampling every 20 ms and wait (at most 3 s) for the first
         sample, so that a short timed region that follows is covered."""
         self.mark_at = 0
+        self.end_at = None
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.id}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
@@ -132,6 +136,14 @@ class ClockSampler:
         """The timed region starts now: later samples are the ones reported."""
         self.mark_at = len(self._rows())
 
+    def mark_end(self):
+        """The timed region ended now; samples taken after this belong to the
+        window of the same work that may follow it."""
+        self.end_at = len(self._rows())
+
+    def region_samples(self) -> int:
+        return max(0, (self.end_at if self.end_at is not None else len(self._rows())) - self.mark_at)
+
     def _rows(self):
         rows = []
         try:
@@ -144,7 +156,7 @@ class ClockSampler:
             pass
         return rows
 
-    def stop(self):
+    def stop(self, window_note=None):
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -153,17 +165,26 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.fh.close()
-        return self.summary(self._rows(), self.mark_at)
+        rows = self._rows()
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        return self.summary(rows, self.mark_at, self.end_at, window_note)
 
     @staticmethod
-    def summary(all_rows, mark_at):
+    def summary(all_rows, mark_at, end_at=None, window_note=None):
         """Median SM clock, max clock and throttle reasons of the samples
-        taken after mark_at; when the region was too short for one, the last
-        sample before it, flagged."""
-        rows = all_rows[mark_at:]
+        taken in the timed region (from mark_at to end_at) and, when a window
+        of the same work followed it (window_note), of that window too; with
+        neither, the last sample before the region, flagged."""
+        end = len(all_rows) if end_at is None else end_at
+        region = all_rows[mark_at:end]
+        window = all_rows[end:] if (end_at is not None and window_note) else []
+        rows = region + window
         before = False
         if not rows and all_rows:
-            rows, before = all_rows[-1:], True
+            rows, before = all_rows[max(0, mark_at - 1):mark_at] or all_rows[-1:], True
         if not rows:
             return None
         sm = [float(r[1]) for r in rows]
@@ -173,8 +194,11 @@ class ClockSampler:
             for name, val in zip(names, r[5:9]):
                 if val.lower() == "active":
                     reasons.add(name)
-        out = {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "samples": 0 if before else len(rows),
-               "reasons": sorted(reasons)}
+        out = {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+               "samples": 0 if before else len(region), "reasons": sorted(reasons)}
+        if window:
+            out["window_samples"] = len(window)
+            out["window"] = window_note
         if before:
             out["note"] = "timed region shorter than the sampling interval: the last sample before it"
         return out
@@ -356,10 +380,149 @@ def resample_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, peaks
     k = kids.shape[0]
     nbytes = 16 * m + 8 * m + m * c * es + 16 * k + k * c * es
     out["upsample_with_child_map"] = {"ms": round(ms, 4), "gbs_features_and_coords": round(nbytes / (ms * 1e-3) / 1e9, 1)}
-    out["sizes"] = {"rows": n, "parents": m, "children": k, "channels": c, "dtype": "bf16"}
+    out["sizes"] = {"rows": n, "parents": m, "children": k, "channels": c, "dtype": str(feats_d.dtype).replace("torch.", "")}
     out["hbm_peak_gbs"] = peaks["hbm_gbs"]
     smc.status(stream)
     return out
+
+
+class StepRunner:
+    """Steps enqueued up to DEPTH ahead of the host, as a job would run them:
+    each step is the asynchronous map build and the conv behind it on one
+    stream, bracketed by its own CUDA events (an L2 flush sits between steps,
+    outside them).  A step is retired DEPTH steps later: its map's outcome is
+    checked, its event times are read and the map is freed (stream-ordered)."""
+    DEPTH = 4
+
+    def __init__(self, smc, torch, stream, flush, coords_d, grid, batch, feats_d, w_d, b_d, out_d, profile=False):
+        self.smc, self.torch, self.stream, self.flush = smc, torch, stream, flush
+        self.coords_d, self.grid, self.batch = coords_d, grid, batch
+        self.feats_d, self.w_d, self.b_d, self.out_d = feats_d, w_d, b_d, out_d
+        self.profile = profile  # read the library's per-phase timing of each build
+        self.pending = []
+        self.times, self.conv_times, self.map_times = [], [], []
+
+    def submit(self, flush=True):
+        torch, smc, stream = self.torch, self.smc, self.stream
+        if flush:
+            self.flush.zero_()
+        e0, e1, ec, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
+        e0.record(stream)
+        m = smc.build_map(self.coords_d, self.grid, batch=self.batch, stream=stream, sync=False)
+        e1.record(stream)
+        smc.conv(m, self.feats_d, self.w_d, self.b_d, ksize=3, orientation=1, out=self.out_d, stream=stream)
+        ec.record(stream)
+        m.stream_wait(stream)  # the step ends when the whole build (pair lists too) is done
+        e2.record(stream)
+        self.pending.append((e0, e1, ec, e2, m))
+        if len(self.pending) > self.DEPTH:
+            self.retire()
+
+    def retire(self):
+        e0, e1, ec, e2, m = self.pending.pop(0)
+        e2.synchronize()
+        m.wait()  # raises if the build failed on the device
+        self.times.append(e0.elapsed_time(e2))
+        self.conv_times.append(e1.elapsed_time(ec))
+        if self.profile:
+            self.map_times.append(m.timing())
+        m.free()
+
+    def drain(self):
+        while self.pending:
+            self.retire()
+
+
+def conv_alone_times(smc, torch, stream, flush, m, feats_d, w_d, b_d, out_d, reps=10):
+    """Median device time (ms) of one conv on a built map, with L2 flushed
+    before it (flushed) and right after an identical conv (L2 warm: the
+    features, weights and map it reads are where the previous one left them).
+    Each conv is queued behind device work, so no host latency is timed."""
+    cold, warm = [], []
+    for _ in range(reps + 1):
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        smc.conv(m, feats_d, w_d, b_d, ksize=3, orientation=1, out=out_d, stream=stream)
+        ev[1].record(stream)
+        ev[2].record(stream)
+        smc.conv(m, feats_d, w_d, b_d, ksize=3, orientation=1, out=out_d, stream=stream)
+        ev[3].record(stream)
+        ev[3].synchronize()
+        cold.append(ev[0].elapsed_time(ev[1]))
+        warm.append(ev[2].elapsed_time(ev[3]))
+    smc.status(stream)
+    return float(np.median(cold[1:])), float(np.median(warm[1:]))
+
+
+def measure_config(smc, torch, stream, flush, dev, peaks, name, dtype, steps, world, wl=None):
+    """One workload measured the way the headline is: timed steps (build +
+    conv, L2 flushed between steps), the conv alone flushed and L2-warm, and
+    the map phases from the library's own events; with the SM clocks sampled
+    while it runs.  Returns a sub-record for the bench line."""
+    w = wl if wl is not None else get_workload(name)
+    tdt = {"bf16": torch.bfloat16, "f16": torch.float16}[dtype]
+    f, wt, b = S.layer_tensors(w, dtype)
+    coords_d = torch.from_numpy(w.coords).to(dev)
+    feats_d = torch.from_numpy(f).to(tdt).to(dev)
+    w_d = torch.from_numpy(wt).to(tdt).to(dev)
+    b_d = torch.from_numpy(b).to(tdt).to(dev)
+    out_d = torch.empty((w.n, w.cout), dtype=tdt, device=dev)
+    batch = int(w.coords[:, 0].max()) + 1
+    del f
+    args = (smc, torch, stream, flush, coords_d, w.grid, batch, feats_d, w_d, b_d, out_d)
+    warm = StepRunner(*args)
+    for _ in range(3):
+        warm.submit()
+    warm.drain()
+    clocks = ClockSampler(dev.index or 0)
+    clocks.start()
+    clocks.mark()
+    run = StepRunner(*args)
+    t0 = time.perf_counter()
+    while len(run.times) + len(run.pending) < steps or time.perf_counter() - t0 < 0.3:
+        run.submit()
+    run.drain()
+    clocks.mark_end()
+    clk = clocks.stop()
+    prof = StepRunner(*args, profile=True)
+    smc.set_profiling(True)
+    for _ in range(min(steps, 20)):
+        prof.submit()
+    prof.drain()
+    smc.set_profiling(False)
+    m = smc.build_map(coords_d, w.grid, batch=batch, stream=stream)
+    P = m.pairs_total
+    conv_cold, conv_warm = conv_alone_times(smc, torch, stream, flush, m, feats_d, w_d, b_d, out_d)
+    m.free()
+    step_ms = reduce_max(float(np.median(run.times)), world, dev)
+    conv_ms = reduce_max(float(np.median(run.conv_times)), world, dev)
+    look = reduce_max(float(np.median([t[0] for t in prof.map_times])), world, dev)
+    sched = reduce_max(float(np.median([t[1] for t in prof.map_times])), world, dev)
+    pairs_ms = reduce_max(float(np.median([t[2] for t in prof.map_times])), world, dev)
+    flops = pair_flops(P, w.cin, w.cout)
+    map_bytes = algorithmic_map_bytes(w.n, P)
+    tfl = flops / (conv_ms * 1e-3) / 1e12
+    gbs = map_bytes / ((look + pairs_ms) * 1e-3) / 1e9
+    rec = {
+        "workload": f"{w.name}: {w.note}", "dtype": dtype, "n_voxels": w.n, "pairs": P,
+        "steps_timed": len(run.times), "step_ms": round(step_ms, 4),
+        "mvoxels_per_s": round(world * w.n / (step_ms * 1e-3) / 1e6, 2),
+        "conv_ms": round(conv_ms, 4), "conv_ms_alone_l2_flushed": round(conv_cold, 4),
+        "conv_ms_alone_l2_warm": round(conv_warm, 4),
+        "conv_roofline": {"bound": "tensor", "achieved": round(tfl, 2), "peak": peaks["bf16_tflops"],
+                          "unit": "TFLOP/s", "frac": round(tfl / peaks["bf16_tflops"], 4),
+                          "frac_l2_warm": round(flops / (conv_warm * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)},
+        "map_ms": {"clears_and_lookups": round(look, 4), "tile_schedule": round(sched, 4),
+                   "pair_lists_side_stream": round(pairs_ms, 4)},
+        "map_roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "algorithmic_bytes": map_bytes},
+    }
+    if clk is not None:
+        rec["clocks"] = clk
+    del feats_d, out_d, coords_d
+    torch.cuda.empty_cache()
+    return rec
 
 
 def run_gpu(args):
@@ -375,63 +538,25 @@ def run_gpu(args):
     peaks = load_peaks()
 
     w = get_workload(args.workload)
-    f, wt, b = S.layer_tensors(w, "bf16")
+    dtype = "f16" if "f16" in w.dtypes and "bf16" not in w.dtypes else "bf16"
+    tdt = torch.float16 if dtype == "f16" else torch.bfloat16
+    f, wt, b = S.layer_tensors(w, dtype)
     coords_d = torch.from_numpy(w.coords).to(dev)
-    feats_d = torch.from_numpy(f).to(torch.bfloat16).to(dev)
-    w_d = torch.from_numpy(wt).to(torch.bfloat16).to(dev)
-    b_d = torch.from_numpy(b).to(torch.bfloat16).to(dev)
-    out_d = torch.empty((w.n, w.cout), dtype=torch.bfloat16, device=dev)
+    feats_d = torch.from_numpy(f).to(tdt).to(dev)
+    w_d = torch.from_numpy(wt).to(tdt).to(dev)
+    b_d = torch.from_numpy(b).to(tdt).to(dev)
+    out_d = torch.empty((w.n, w.cout), dtype=tdt, device=dev)
     batch = int(w.coords[:, 0].max()) + 1
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    runner = lambda profile=False: StepRunner(smc, torch, stream, flush, coords_d, w.grid, batch, feats_d, w_d,
+                                              b_d, out_d, profile=profile)
 
     smc.set_profiling(False)  # the timed steps carry no instrumentation
 
-    class Steps:
-        """Steps enqueued up to DEPTH ahead of the host, as a job would run
-        them: each step is the asynchronous map build and the conv behind it
-        on one stream, bracketed by its own CUDA events (the L2 flush sits
-        between steps, outside them).  A step is retired DEPTH steps later:
-        its map's outcome is checked, its event times are read and the map is
-        freed (stream-ordered)."""
-        DEPTH = 4
-
-        def __init__(self, profile=False):
-            self.profile = profile  # read the library's per-phase timing of each build
-            self.pending = []
-            self.times, self.conv_times, self.map_times = [], [], []
-
-        def submit(self):
-            e0, e1, ec, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
-            e0.record(stream)
-            m = smc.build_map(coords_d, w.grid, batch=batch, stream=stream, sync=False)
-            e1.record(stream)
-            smc.conv(m, feats_d, w_d, b_d, ksize=3, orientation=1, out=out_d, stream=stream)
-            ec.record(stream)
-            m.stream_wait(stream)  # the step ends when the whole build (pair lists too) is done
-            e2.record(stream)
-            self.pending.append((e0, e1, ec, e2, m))
-            if len(self.pending) > self.DEPTH:
-                self.retire()
-
-        def retire(self):
-            e0, e1, ec, e2, m = self.pending.pop(0)
-            e2.synchronize()
-            m.wait()  # raises if the build failed on the device
-            self.times.append(e0.elapsed_time(e2))
-            self.conv_times.append(e1.elapsed_time(ec))
-            if self.profile:
-                self.map_times.append(m.timing())
-            m.free()
-
-        def drain(self):
-            while self.pending:
-                self.retire()
-
     # warm-up
-    warm = Steps()
+    warm = runner()
     for _ in range(args.warmup):
-        flush.zero_()
         warm.submit()
     warm.drain()
     smc.status(stream)
@@ -448,28 +573,42 @@ def run_gpu(args):
     clocks.mark()
     t_wall0 = time.perf_counter()
     launches_before = smc.kernel_launches()
-    run = Steps()
+    run = runner()
     for _ in range(args.steps):
-        flush.zero_()
         run.submit()
     run.drain()
     torch.cuda.synchronize()
     times, conv_times = run.times, run.conv_times
     launches = smc.kernel_launches() - launches_before
     wall = time.perf_counter() - t_wall0
-    clk = clocks.stop()
+    clocks.mark_end()
+    # A timed region shorter than a few sampling intervals gets the same
+    # steps repeated right after it, untimed, so that the clock record has
+    # samples of this work under load.
+    window_note = None
+    if clocks.region_samples() < 5:
+        tw = time.perf_counter()
+        extra = runner()
+        while time.perf_counter() - tw < 0.4:
+            extra.submit()
+        extra.drain()
+        window_note = (f"the same steps repeated untimed for {1e3 * (time.perf_counter() - tw):.0f} ms right "
+                       f"after the timed region ({len(extra.times)} steps)")
+    clk = clocks.stop(window_note)
     barrier(world)
     smc.status(stream)
     # per-phase breakdown of the build from a separate, untimed pass with the
     # library's own CUDA events on
     smc.set_profiling(True)
-    prof = Steps(profile=True)
+    prof = runner(profile=True)
     for _ in range(min(args.steps, 50)):
-        flush.zero_()
         prof.submit()
     prof.drain()
     smc.set_profiling(False)
     map_times = prof.map_times
+    m1 = smc.build_map(coords_d, w.grid, batch=batch, stream=stream)
+    conv_cold, conv_warm = conv_alone_times(smc, torch, stream, flush, m1, feats_d, w_d, b_d, out_d)
+    m1.free()
     variants = conv_variant_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, w_d, b_d, out_d)
     subdiv = subdivide_times(smc, torch, stream, flush)
     epilogue = epilogue_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, w_d, b_d, out_d)
@@ -497,18 +636,25 @@ def run_gpu(args):
             traffic = tr.get("dram_bytes_per_launch")
 
     # end to end through the public API: pinned host inputs in, result out
-    e2e = run_e2e(w, f, wt, b, batch, dev, stream, args)
+    e2e = run_e2e(w, f, wt, b, batch, dev, stream, args, tdt)
     e2e_v = reduce_max(e2e["ms"], world, dev)
+
+    # the other configurations of the metric, measured the same way
+    configs = {}
+    if not args.skip_configs and args.workload == "shells6":
+        del f
+        for name, dtype in (("shells6_118k", "bf16"), ("full128", "bf16"), ("varlen4", "f16"), ("decoder3", "bf16")):
+            configs[name] = measure_config(smc, torch, stream, flush, dev, peaks, name, dtype, 10, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
-        cpu = run_cpu_baseline(w, f, wt, b, budget_s=args.cpu_seconds)
+        cpu = run_cpu_baseline(w, *S.layer_tensors(w, dtype), budget_s=args.cpu_seconds)
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype,
             "data": "synthetic (seeded union of 6 sphere shells; random-init KRSC weights)",
             "config": {
                 "workload": f"{w.name}: {w.note}", "n_voxels": w.n, "pairs": P, "grid": list(w.grid),
@@ -518,11 +664,12 @@ def run_gpu(args):
             },
             "pair_tflops": round(conv_tflops, 2),
             "map_build_gbs": round(map_gbs, 1),
-            "breakdown_ms": {"step": round(ms_per_step, 4), "map_lookups": round(look_ms, 4),
+            "breakdown_ms": {"step": round(ms_per_step, 4), "map_clears_and_lookups": round(look_ms, 4),
                              "tile_schedule": round(sched_ms, 4),
                              "pair_lists_side_stream": round(pairs_ms, 4), "conv": round(conv_ms, 4)},
             "step_ms_quantiles": {q: round(float(np.quantile(times, v)), 4)
                                   for q, v in (("p50", 0.5), ("p90", 0.9), ("p99", 0.99), ("max", 1.0))},
+            "conv_alone_ms": {"l2_flushed": round(conv_cold, 4), "l2_warm": round(conv_warm, 4)},
             "conv_mvoxels_per_s": round(w.n / (conv_ms * 1e-3) / 1e6, 2),
             "conv_tap_efficiency": round(eff, 4),
             "conv_variants_ms": variants,
@@ -532,13 +679,15 @@ def run_gpu(args):
             "roofline": {"kernel": "k_conv_tc", "bound": "tensor", "achieved": round(conv_tflops, 2),
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": round(conv_tflops / peaks["bf16_tflops"], 4), "traffic": traffic,
+                         "frac_l2_warm": round(flops / (conv_warm * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
                          "peak_source": f"{peaks['source']} bf16 burst (kernel timed alone)",
                          "algorithmic": "2 * pairs * Cin * Cout per launch"},
-            "map_roofline": {"kernels": "k_insert, k_neighbours, pair-list scan, k_pairs (time = lookups + pair lists)",
+            "map_roofline": {"kernels": "clears, k_insert, k_neighbours, pair-list scan, k_pairs (time = clears and lookups + pair lists)",
                              "bound": "hbm", "achieved": round(map_gbs, 1),
                              "peak": peaks["hbm_gbs"], "unit": "GB/s",
                              "frac": round(map_gbs / peaks["hbm_gbs"], 4),
                              "algorithmic": "16N coords + 108N map + 8P pairs"},
+            "configs": configs,
             "e2e": {"value": round(world * w.n / (e2e_v * 1e-3) / 1e6, 3), "unit": UNIT,
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                     "ms_per_step": round(e2e_v, 4)},
@@ -556,7 +705,7 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
-def run_e2e(w, f, wt, b, batch, dev, stream, args):
+def run_e2e(w, f, wt, b, batch, dev, stream, args, tdt=None):
     """Same step through the public API, with each step's inputs copied from
     pinned host memory and its result copied back inside the timed region.
     Steps are pipelined the way a serving loop runs them: inputs go up on a
@@ -567,17 +716,18 @@ def run_e2e(w, f, wt, b, batch, dev, stream, args):
     import torch
 
     import submanifold_sparse_convolution_packed_b200 as smc
+    tdt = tdt or torch.bfloat16
     coords_h = torch.from_numpy(w.coords).pin_memory()
-    feats_h = torch.from_numpy(f).to(torch.bfloat16).pin_memory()
-    w_h = torch.from_numpy(wt).to(torch.bfloat16).pin_memory()
-    b_h = torch.from_numpy(b).to(torch.bfloat16).pin_memory()
+    feats_h = torch.from_numpy(f).to(tdt).pin_memory()
+    w_h = torch.from_numpy(wt).to(tdt).pin_memory()
+    b_h = torch.from_numpy(b).to(tdt).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (coords_h, feats_h, w_h, b_h))
     depth = 2
-    outs_h = [torch.empty((w.n, w.cout), dtype=torch.bfloat16).pin_memory() for _ in range(depth)]
+    outs_h = [torch.empty((w.n, w.cout), dtype=tdt).pin_memory() for _ in range(depth)]
     d2h = outs_h[0].numel() * outs_h[0].element_size()
     slots = [dict(c=torch.empty_like(coords_h, device=dev), x=torch.empty_like(feats_h, device=dev),
                   w=torch.empty_like(w_h, device=dev), b=torch.empty_like(b_h, device=dev),
-                  y=torch.empty((w.n, w.cout), dtype=torch.bfloat16, device=dev)) for _ in range(depth)]
+                  y=torch.empty((w.n, w.cout), dtype=tdt, device=dev)) for _ in range(depth)]
     up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     ev = lambda: torch.cuda.Event()
     inputs_free = [None] * depth   # compute consumed the slot's inputs
@@ -635,16 +785,26 @@ def run_e2e(w, f, wt, b, batch, dev, stream, args):
 
 
 # ------------------------------------------------------------- CPU oracle
-def run_cpu_baseline(w, f, wt, b, budget_s: float = 20.0):
-    """The CPU oracle, as it stands, on a bounded sample of the same workload:
-    the full neighbour map plus the conv on a seeded sample of output rows;
-    throughput = voxels per second of (map cost per voxel + conv cost per row)."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
+def _oracle_rate(w, f, wt, b, budget_s: float, threads: int):
+    """Voxels/s of the oracle on a bounded sample: the full neighbour map plus
+    the conv on seeded batches of output rows until about budget_s / 2 of
+    conv time; returns (rate, description)."""
     from oracle import oracle
-    threads = os.cpu_count() or 1
     t0 = time.perf_counter()
     oracle.neighbour_map(w.coords, w.grid)
     t_map = time.perf_counter() - t0
-    rows_n = min(w.n, 2048)
+    rows_n = min(w.n, 2048 if threads > 1 else 256)
     rng = np.random.default_rng(0)
     t_conv, done = 0.0, 0
     while t_conv < budget_s * 0.5 and done < w.n:
@@ -654,9 +814,24 @@ def run_cpu_baseline(w, f, wt, b, budget_s: float = 20.0):
         t_conv += time.perf_counter() - t1
         done += rows_n
     per_voxel = t_map / w.n + t_conv / done
-    return {"value": round(1.0 / per_voxel / 1e6, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"map over all {w.n} voxels ({t_map:.2f} s) + fp64 conv on {done} seeded rows "
-                      f"({t_conv:.2f} s, {threads} threads), per-voxel cost scaled to the metric"}
+    return 1.0 / per_voxel, (f"map over all {w.n} voxels ({t_map:.2f} s) + fp64 conv on {done} seeded rows "
+                             f"({t_conv:.2f} s, {threads} thread{'s' if threads > 1 else ''}), per-voxel cost "
+                             f"scaled to the metric")
+
+
+def run_cpu_baseline(w, f, wt, b, budget_s: float = 20.0, single: bool = True):
+    """The CPU oracle, as it stands, on a bounded sample of the same workload,
+    on all host cores (the reported figure) and, when `single`, on one thread
+    too; the host's CPU model and core count are recorded beside them."""
+    threads = os.cpu_count() or 1
+    budget_all = budget_s * (0.6 if single else 1.0)
+    rate, desc = _oracle_rate(w, f, wt, b, budget_all, threads)
+    out = {"value": round(rate / 1e6, 6), "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
+           "cpu_model": cpu_model(), "nproc": threads}
+    if single:
+        r1, d1 = _oracle_rate(w, f, wt, b, budget_s - budget_all, 1)
+        out["single_thread"] = {"value": round(r1 / 1e6, 6), "unit": UNIT, "cores": 1, "sample": d1}
+    return out
 
 
 def run_reference(args):
@@ -672,11 +847,11 @@ def run_reference(args):
     f, wt, b = S.layer_tensors(w, "bf16")
     per_step = max(1.0, min(args.cpu_seconds, 150.0 / (args.steps + args.warmup)))
     for _ in range(args.warmup):
-        run_cpu_baseline(w, f, wt, b, budget_s=min(per_step, 2.0))
+        run_cpu_baseline(w, f, wt, b, budget_s=min(per_step, 2.0), single=False)
     vals = []
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        vals.append(run_cpu_baseline(w, f, wt, b, budget_s=per_step))
+        vals.append(run_cpu_baseline(w, f, wt, b, budget_s=per_step, single=False))
         if time.perf_counter() - t0 > 180.0:
             break
     elapsed = time.perf_counter() - t0
@@ -704,6 +879,8 @@ def main(argv=None):
                     help="shells6 (default), full128, varlen4, shell2, decoder0..decoder3")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-configs", action="store_true",
+                    help="measure the default workload only, not the other configurations")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

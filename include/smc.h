@@ -352,7 +352,8 @@ SMC_API const char* smc_strerror(int code);
  *   more).  Used to exercise SMC_E_CAPACITY.
  * smc_set_profiling: when on, smc_build_map records CUDA events on its stream
  *   around its kernels; smc_map_timing then returns, in milliseconds,
- *   ms[0] = hash insert + neighbour lookups, ms[1] = tile schedule, and
+ *   ms[0] = the clears of the lookup structure and scratch, the insert and the
+ *   neighbour lookups, ms[1] = tile schedule, and
  *   ms[2] = pair lists (built on a library-owned side stream, concurrently
  *   with the tile schedule; measured from the end of the lookups).
  * smc_kernel_launches: number of CUDA kernels this library has launched in

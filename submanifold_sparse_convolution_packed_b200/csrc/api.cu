@@ -448,9 +448,9 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   // schedule is done too -- the status copy, the completion event and the
   // release of the scratch.  A conv enqueued on s behind the build waits for
   // the schedule only, and overlaps the pair lists.
-  cudaError_t ce = cudaMemsetAsync(T + o_table, 0xFF, table_bytes, s);
+  cudaError_t ce = m->prof[0] ? cudaEventRecord(m->prof[0], s) : cudaSuccess;  // the clears count as lookups
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(T + o_table, 0xFF, table_bytes, s);
   if (ce == cudaSuccess) ce = cudaMemsetAsync(T + o_err, 0, zero_bytes, s);
-  if (ce == cudaSuccess && m->prof[0]) ce = cudaEventRecord(m->prof[0], s);
   if (ce == cudaSuccess && sub) {
     ce = cudaMemsetAsync(m->tile_mask, 0, a.nzero * sizeof(uint32_t), s);  // k_insert clears them otherwise
     if (ce == cudaSuccess) ce = smc::launch_subdiv_lookups(a, sub->parent_nbr, sub->child_src, sub->remap, s);

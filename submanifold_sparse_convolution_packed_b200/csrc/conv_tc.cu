@@ -21,6 +21,7 @@
 //              tile::gather4 row loads (missing neighbours are row -1, which
 //              TMA reads as zeros); then the epilogue for the same rows:
 //              tcgen05.ld, bias in fp32, rounding, 16-byte stores.
+//              (Or warps 2-9, 16 rows each, 4 issuing lanes: see kGW.)
 // Pipeline stages are (tap, channel block) pairs of KB = 32 or 64 channels in
 // swizzled shared memory (64-byte or 128-byte swizzle).  Every wait is
 // bounded; on timeout the error word gets a bit and the CTA winds down.
@@ -36,7 +37,7 @@
 
 namespace smc {
 
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 192;  // weight loader, MMA issuer and 4 gather / epilogue warps
 constexpr int kMaxStages = 8;
 
 struct TcSmemLayout {
@@ -82,8 +83,12 @@ struct TcParams {
 // this epilogue lengthens the tile's hold on its SM slot and the residual rows
 // are read in schedule order.  Separate instances keep the plain conv free of
 // the extra epilogue code, which measured 5-19% slower even when unused.
-template <bool kPair, int kEpi>
-__global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant__ CUtensorMap fmap,
+// kGW: gather warps (4 or 8).  With 8, warps w and w + 4 share a TMEM lane
+// quarter: each gathers 16 of its 32 rows (4 issuing lanes) and, in the
+// epilogue, writes half of its columns.  Selected by measurement for the
+// plain conv at three CTAs per SM.
+template <bool kPair, int kEpi, int kGW>
+__global__ void __launch_bounds__(64 + 32 * kGW, kGW == 8 ? 3 : 4) k_conv_tc(const __grid_constant__ CUtensorMap fmap,
                                                         const __grid_constant__ CUtensorMap wmap,
                                                         const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -120,11 +125,15 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
     if (p.orientation < 0) mask = mirror27(mask);
   }
 
-  // The gather / epilogue warps (2-5) own tile row r: its output row v and,
-  // for k = 3, its 27 neighbour rows, loaded here so that the loads overlap
-  // the barrier set-up and the TMEM allocation below.
-  const int q = warp & 3;       // TMEM lane quarter of warps 2..5
-  const int r = q * 32 + lane;  // tile row
+  // The gather / epilogue warps (2 ..) own epilogue tile row r (TMEM lane)
+  // and its output row v, and gather tile row rg: for k = 3 its 27 neighbour
+  // rows, loaded here so that the loads overlap the barrier set-up and the
+  // TMEM allocation below.  With 4 gather warps r == rg.
+  constexpr int kRPW = kTileRows / kGW;  // tile rows gathered per warp
+  const int q = warp & 3;                // TMEM lane quarter
+  const int h = kGW == 8 ? ((warp - 2) >> 2) : 0;  // half of the quarter (rows gathered, columns written)
+  const int r = q * 32 + lane;
+  const int rg = q * 32 + h * kRPW + (lane % kRPW);
   int32_t v = -1;
   int32_t nb[kTaps];
   // The unit's bias values go to shared memory once, so that the epilogue
@@ -137,17 +146,23 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
     if (p.bias_vec) {
       if (8 * t < nb_cols) reinterpret_cast<uint4*>(s_bias)[t] = __ldg(reinterpret_cast<const uint4*>(p.bias + n0) + t);
     } else {
-      for (int c = t; c < nb_cols; c += 128) s_bias[c] = __ldg(p.bias + n0 + c);
+      for (int c = t; c < nb_cols; c += 32 * kGW) s_bias[c] = __ldg(p.bias + n0 + c);
     }
   }
   if (warp >= 2) {
     const int64_t g = tile * kTileRows + r;
     v = g < p.n ? (k3 ? __ldg(p.perm + g) : static_cast<int32_t>(g)) : -1;
     if (v >= p.n) v = -1;  // a schedule left incomplete by a failed build is skipped, never followed
+    int32_t vg = v;
+    if (kGW != 4) {
+      const int64_t gg = tile * kTileRows + rg;
+      vg = gg < p.n ? (k3 ? __ldg(p.perm + gg) : static_cast<int32_t>(gg)) : -1;
+      if (vg >= p.n) vg = -1;
+    }
     if (k3) {
-      const int32_t* row = p.nbr + static_cast<int64_t>(v < 0 ? 0 : v) * kTaps;
+      const int32_t* row = p.nbr + static_cast<int64_t>(vg < 0 ? 0 : vg) * kTaps;
 #pragma unroll
-      for (int d = 0; d < kTaps; ++d) nb[d] = v >= 0 ? __ldg(row + (p.orientation > 0 ? d : kTaps - 1 - d)) : -1;
+      for (int d = 0; d < kTaps; ++d) nb[d] = vg >= 0 ? __ldg(row + (p.orientation > 0 ? d : kTaps - 1 - d)) : -1;
     }
   }
 
@@ -155,8 +170,8 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
     prefetch_tmap(&fmap);
     prefetch_tmap(&wmap);
     for (int s = 0; s < p.stages; ++s) {
-      // weight loader (+ 4 gather warps), of both CTAs for a pair
-      mbar_init(bar_full + 8 * s, (k3 ? 5 : 1) * (kPair ? 2 : 1));
+      // weight loader (+ the gather warps), of both CTAs for a pair
+      mbar_init(bar_full + 8 * s, (k3 ? 1 + kGW : 1) * (kPair ? 2 : 1));
       mbar_init(bar_empty + 8 * s, 1);
     }
     mbar_init(bar_acc, 1);
@@ -273,8 +288,8 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
 #pragma unroll
       for (int d = 0; d < kTaps; ++d) {
         if (!((mask >> d) & 1u) || !ok) continue;
-        // lane j < 8 gathers tile rows 32q + 4j .. 32q + 4j + 3
-        const int src = (lane & 7) * 4;
+        // lane j < kRPW / 4 gathers rows 4j .. 4j + 3 of the warp's kRPW rows
+        const int src = (lane % (kRPW / 4)) * 4;
         const int32_t r0 = __shfl_sync(0xffffffffu, nb[d], src + 0);
         const int32_t r1 = __shfl_sync(0xffffffffu, nb[d], src + 1);
         const int32_t r2 = __shfl_sync(0xffffffffu, nb[d], src + 2);
@@ -291,12 +306,12 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
           }
           const uint32_t full = full_tgt + 8 * stage;
           if (lane == 0) {
-            if (kPair) mbar_arrive_expect_tx_cluster(full, 32u * row_bytes);
-            else mbar_arrive_expect_tx(full, 32u * row_bytes);
+            if (kPair) mbar_arrive_expect_tx_cluster(full, kRPW * row_bytes);
+            else mbar_arrive_expect_tx(full, kRPW * row_bytes);
           }
           __syncwarp();
-          if (lane < 8) {
-            const uint32_t dst = sbase + L.a_off + stage * a_bytes + (q * 32 + 4 * lane) * row_bytes;
+          if (lane < kRPW / 4) {
+            const uint32_t dst = sbase + L.a_off + stage * a_bytes + (q * 32 + h * kRPW + 4 * lane) * row_bytes;
             if (kPair) tma_gather4_pair(dst, &fmap, full, kb * p.kb_elems, r0, r1, r2, r3);
             else tma_gather4(dst, &fmap, full, kb * p.kb_elems, r0, r1, r2, r3);
           }
@@ -334,10 +349,12 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
       // 16-byte stores (a row's bytes are contiguous in `out`), instead of 32
       // scattered rows per store instruction.
       const bool bf = p.is_bf16 != 0;
-      const uint32_t pitch = static_cast<uint32_t>(p.bn) * 2u + 16u;
-      uint8_t* blk = smem + L.a_off + static_cast<uint32_t>(q) * 32u * pitch;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-      int ncols_all = p.cout - n0 < p.bn ? p.cout - n0 : p.bn;
+      const int bw = p.bn / (kGW / 4);  // columns this warp writes
+      const int c_lo = h * bw;
+      const uint32_t pitch = static_cast<uint32_t>(bw) * 2u + 16u;
+      uint8_t* blk = smem + L.a_off + static_cast<uint32_t>(warp - 2) * 32u * pitch;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(c_lo);
+      int ncols_all = p.cout - n0 - c_lo < bw ? p.cout - n0 - c_lo : bw;
       for (int c0 = 0; c0 < ncols_all; c0 += 32) {
         float acc[32];
         tmem_ld_32cols(t_row + c0, acc);
@@ -346,12 +363,12 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
           if (c0 + j >= ncols_all) break;
           float bv[8];
           if (p.bias) {
-            const uint4 bq = *reinterpret_cast<const uint4*>(s_bias + c0 + j);
-            const uint32_t bw[4] = {bq.x, bq.y, bq.z, bq.w};
+            const uint4 bq = *reinterpret_cast<const uint4*>(s_bias + c_lo + c0 + j);
+            const uint32_t bwd[4] = {bq.x, bq.y, bq.z, bq.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              bv[2 * e] = half_bits_to_float(static_cast<uint16_t>(bw[e] & 0xFFFFu), bf);
-              bv[2 * e + 1] = half_bits_to_float(static_cast<uint16_t>(bw[e] >> 16), bf);
+              bv[2 * e] = half_bits_to_float(static_cast<uint16_t>(bwd[e] & 0xFFFFu), bf);
+              bv[2 * e + 1] = half_bits_to_float(static_cast<uint16_t>(bwd[e] >> 16), bf);
             }
           } else {
 #pragma unroll
@@ -377,7 +394,7 @@ __global__ void __launch_bounds__(kTcThreads, 4) k_conv_tc(const __grid_constant
         const int32_t vr = __shfl_sync(0xffffffffu, v, rr < 32 ? rr : 31);
         if (lane < rpp * cpr && rr < 32 && vr >= 0) {
           const uint4 x = *reinterpret_cast<const uint4*>(blk + rr * pitch + ch * 16);
-          *reinterpret_cast<uint4*>(p.out + static_cast<int64_t>(vr) * p.cout + n0 + ch * 8) = x;
+          *reinterpret_cast<uint4*>(p.out + static_cast<int64_t>(vr) * p.cout + n0 + c_lo + ch * 8) = x;
         }
       }
     } else if (ready) {
@@ -491,6 +508,7 @@ struct TcShape {
 };
 
 static std::atomic<int> g_conv_variant{0};
+static std::atomic<int> g_gather_warps{0};  // 0 = by shape; 4 = always four gather warps
 
 static TcShape choose_shape(int cin, int cout, int64_t ntiles) {
   TcShape t;
@@ -579,14 +597,20 @@ cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s) {
   p.tile_mask = a.tile_mask;
   p.bias = static_cast<const uint16_t*>(a.bias);
   p.bias_vec = a.bias && aligned16(a.bias) ? 1 : 0;
-  {
-    // the staged epilogue needs 4 warps x 32 rows x (row bytes + 16) of the
-    // stage buffers (A and B regions, contiguous); rows hold at most 32 chunks
-    const uint32_t need = 4u * 32u * (static_cast<uint32_t>(t.bn) * 2u + 16u);
+  const int epi = a.ep.act != kActNone || a.ep.residual ? 1 : 0;
+  // The staged epilogue needs gather warps x 32 rows x (the warp's row bytes
+  // + 16) of the stage buffers (A and B regions, contiguous).  Eight gather
+  // warps serve the plain k = 3 conv at three CTAs per SM when it fits.
+  auto staged_fits = [&](int gw) {
+    const uint32_t bw = static_cast<uint32_t>(t.bn) / (gw / 4);
+    const uint32_t need = static_cast<uint32_t>(gw) * 32u * (bw * 2u + 16u);
     const uint32_t have =
         static_cast<uint32_t>(t.stages) * (static_cast<uint32_t>(kTileRows + t.bn) * t.kb_elems * 2u);
-    p.stage_out = !t.pair && need <= have ? 1 : 0;
-  }
+    return need <= have;
+  };
+  const bool gw8 = !t.pair && epi == 0 && a.taps == kTaps && t.ctas_per_sm == 3 && t.bn % 64 == 0 &&
+                   staged_fits(8) && g_gather_warps.load() != 4;
+  p.stage_out = !t.pair && staged_fits(gw8 ? 8 : 4) ? 1 : 0;
   p.out = static_cast<uint16_t*>(a.out);
   p.err = a.err;
   p.n = a.n;
@@ -603,9 +627,8 @@ cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s) {
   p.tmem_cols = t.tmem_cols;
   p.ep = a.ep;
   cudaError_t e;
-  const int epi = a.ep.act != kActNone || a.ep.residual ? 1 : 0;
   if (t.pair) {
-    auto kern = epi == 1 ? k_conv_tc<true, 1> : k_conv_tc<true, 0>;
+    auto kern = epi == 1 ? k_conv_tc<true, 1, 4> : k_conv_tc<true, 0, 4>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(t.smem));
     if (e != cudaSuccess) return e;
     const int64_t ctas = 2 * ((ntiles + 1) / 2) * t.nsplit;
@@ -623,11 +646,12 @@ cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s) {
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kern, fmap, wmap, p);
   } else {
-    auto kern = epi == 1 ? k_conv_tc<false, 1> : k_conv_tc<false, 0>;
+    auto kern = gw8 ? k_conv_tc<false, 0, 8> : (epi == 1 ? k_conv_tc<false, 1, 4> : k_conv_tc<false, 0, 4>);
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(t.smem));
     if (e != cudaSuccess) return e;
     const int64_t units = ntiles * t.nsplit;
-    kern<<<static_cast<unsigned>(units), kTcThreads, t.smem, s>>>(fmap, wmap, p);
+    const int threads = gw8 ? 64 + 32 * 8 : kTcThreads;
+    kern<<<static_cast<unsigned>(units), threads, t.smem, s>>>(fmap, wmap, p);
     e = cudaGetLastError();
   }
   count_launches(1);

@@ -142,11 +142,13 @@ def test_per_offset_conv_and_stats_allocation_failure():
 
 
 def test_scan_wait_runs_out(oracle_mod):
-    w, coords = _shell2()
+    # a map large enough for several scan segments in each of its scans
+    w = S.workload("decoder2")
+    coords = torch.from_numpy(w.coords).cuda()
     ref_nbr = oracle_mod.neighbour_map(w.coords, w.grid)
     smc.set_wait_limit_ns(2_000_000)  # 2 ms
-    smc.set_scan_hold(1)  # the radix scans of this map have several segments
-    m = smc.build_map(coords, w.grid, batch=2, sync=False)
+    smc.set_scan_hold(1)
+    m = smc.build_map(coords, w.grid, batch=1, sync=False)
     with pytest.raises(smc.SmcError) as e:
         m.wait()
     assert e.value.code == SMC_E_TIMEOUT
@@ -160,14 +162,15 @@ def test_scan_wait_runs_out(oracle_mod):
     assert e.value.code == SMC_E_TIMEOUT
     m.free()
     # the downsample's scan of its flags runs out the same way
-    feats = torch.randn(w.n, 64, device="cuda").bfloat16()
+    ws, cs = _shell2()
+    feats = torch.randn(ws.n, 64, device="cuda").bfloat16()
     with pytest.raises(smc.SmcError) as e:
-        smc.downsample(coords, w.grid, feats, mode="mean", batch=2)
+        smc.downsample(cs, ws.grid, feats, mode="mean", batch=2)
     assert e.value.code == SMC_E_TIMEOUT
     # hooks off: the device is usable and the next build is exact
     smc.set_scan_hold(-1)
     smc.set_wait_limit_ns(0)
-    m = smc.build_map(coords, w.grid, batch=2)
+    m = smc.build_map(coords, w.grid, batch=1)
     np.testing.assert_array_equal(m.nbr().cpu().numpy(), ref_nbr)
     _, _, in_idx, out_idx = oracle_mod.pair_lists(ref_nbr)
     got_in, got_out, _ = m.pairs()

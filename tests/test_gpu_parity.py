@@ -90,14 +90,18 @@ def map_lookup(request):
 
 # The tile order of the tensor-core conv: rows stably sorted by a 20-bit key
 # whose bits, most significant first, say whether the 8 corner offsets and
-# then the 12 edge offsets have a neighbour.
+# then the 12 edge offsets have a neighbour; maps of at most ONE_PASS_ROWS
+# rows are sorted on the key's high 10 bits alone (one radix pass).
 _KEY_TAPS = [0, 2, 6, 8, 18, 20, 24, 26, 1, 3, 5, 7, 9, 11, 15, 17, 19, 21, 23, 25]
+ONE_PASS_ROWS = 131072
 
 
 def expected_schedule(nbr):
     key = np.zeros(nbr.shape[0], dtype=np.int64)
     for i, d in enumerate(_KEY_TAPS):
         key |= (nbr[:, d] >= 0).astype(np.int64) << (19 - i)
+    if nbr.shape[0] <= ONE_PASS_ROWS:
+        key >>= 10
     return np.argsort(key, kind="stable").astype(np.int32)
 
 
