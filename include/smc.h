@@ -73,7 +73,10 @@ enum {
 };
 
 /*
- * smc_build_map -- build the neighbour map of one coordinate set.
+ * smc_build_map -- build the neighbour map of one coordinate set: the pages'
+ * indice map, 27 lookups per voxel, built once per coordinate set and cached
+ * the way spconv's indice_key caches it (LATO.2 MLX port README, summary;
+ * the map table of its "The scope, once measured").
  *
  * coords : device, int32 [n, 4], rows (b, z, y, x), contiguous, 16-byte aligned.
  *          Row order is arbitrary; row v of the map corresponds to row v here.
@@ -85,10 +88,13 @@ enum {
  *          to read the per-offset counts and the error word.
  * out    : receives the handle; left NULL on failure.
  *
- * Builds, on the device: 64-bit site keys, an open-addressing hash table of
- * the sites, the int32 [n, 27] neighbour map (-1 = absent), the per-offset
- * pair lists (stable compaction of each map column, ascending output row),
- * and the tile schedule used by the tensor-core conv.  coords may be freed
+ * Builds, on the device: 64-bit site keys, a lookup structure of the sites
+ * (a dense int32 index grid over the batch x Z x Y x X box when the box has
+ * at most 2^28 sites and at most 256 sites per voxel, else an
+ * open-addressing hash table; smc_set_map_lookup forces either), the int32
+ * [n, 27] neighbour map (-1 = absent), the per-offset pair lists (stable
+ * compaction of each map column, ascending output row), and the tile
+ * schedule used by the tensor-core conv.  coords may be freed
  * once the call returns.  Device memory comes from a per-device
  * stream-ordered pool owned by the library that keeps freed memory for
  * later builds.  Errors: SMC_E_ARG, SMC_E_ALIGN, SMC_E_RANGE,
@@ -219,7 +225,10 @@ SMC_API int smc_upsample(const int32_t* coords, int64_t n, const uint8_t* mask, 
 SMC_API int smc_map_stream_wait(const smc_map* map, void* stream);
 
 /*
- * smc_conv -- one submanifold convolution over a built map.
+ * smc_conv -- one submanifold convolution over a built map:
+ * out[v] = bias + sum_d feats[nbr(v, d)] @ W[:, d, :]^T with KRSC weights
+ * (LATO.2 MLX port README, summary and "The scope, once measured"; the
+ * orientation choice per its "Correctness" section).
  *
  * feats  : device, [n, cin] row-major, dtype `dtype`.
  * weight : device, KRSC [cout, k, k, k, cin] row-major, dtype `dtype`.
@@ -309,14 +318,19 @@ SMC_API int smc_group_norm(const void* x, int64_t n, int64_t c, const int32_t* c
                    int32_t groups, const double* stats, const void* gamma, const void* beta, float eps,
                    int32_t act, void* out, int32_t dtype, void* stream);
 
-/* n and the per-offset pair counts counts[27] (host) of a map. */
+/* n and the per-offset pair counts counts[27] (host) of a map: the hit
+ * counts of the indice map's 27 offsets (LATO.2 MLX port README, "Correctness":
+ * indice-map hit rates). */
 SMC_API int smc_map_info(const smc_map* map, int64_t* n, int64_t counts[27]);
 
-/* Device pointer to the int32 [n, 27] neighbour map (-1 = absent). */
+/* Device pointer to the int32 [n, 27] neighbour map (-1 = absent): the
+ * indice map of the LATO.2 MLX port README summary. */
 SMC_API int smc_map_nbr(const smc_map* map, const int32_t** nbr);
 
 /*
- * Per-offset pair lists: device pointers in_idx[P], out_idx[P] (int32) and
+ * Per-offset pair lists, the operands of the per-offset gather-GEMM-scatter
+ * the pages compare their fused kernel with (shared sparse-core commit log,
+ * the 13.8 ms / 5.9x test commit): device pointers in_idx[P], out_idx[P] (int32) and
  * host offsets[28] (int64, offsets[0] = 0, offsets[27] = P).  Pairs of offset
  * d occupy [offsets[d], offsets[d+1]) in ascending out_idx:
  * (in_idx, out_idx) = (nbr[v][d], v) for every v with nbr[v][d] >= 0.
@@ -325,10 +339,12 @@ SMC_API int smc_map_pairs(const smc_map* map, const int32_t** in_idx, const int3
                   int64_t offsets[28]);
 
 /*
- * Tile schedule of the tensor-core conv: device pointer to perm[n] (int32),
- * the order in which output rows are grouped into tiles of 128 (a
- * permutation of 0..n-1: rows with similar neighbour sets are adjacent, so
- * each tile skips the offsets none of its rows has).
+ * Tile schedule of the tensor-core conv (this library's own; the pages give
+ * none): device pointer to perm[n] (int32), the order in which output rows
+ * are grouped into tiles of 128 (a permutation of 0..n-1: rows are stably
+ * sorted by which of the 8 corner and 12 edge offsets they hit, or, for maps
+ * of at most 131072 rows, by the 8 corners and the first 2 edges alone, so
+ * that each tile skips the offsets none of its rows has).
  */
 SMC_API int smc_map_schedule(const smc_map* map, const int32_t** perm);
 
