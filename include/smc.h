@@ -90,8 +90,9 @@ enum {
  *
  * Builds, on the device: 64-bit site keys, a lookup structure of the sites
  * (a dense int32 index grid over the batch x Z x Y x X box when the box has
- * at most 2^28 sites and at most 256 sites per voxel, else an
- * open-addressing hash table; smc_set_map_lookup forces either), the int32
+ * at most 2^28 sites and at most 256 sites per voxel, with an occupancy
+ * bitmap instead of a clear above 2^23 sites, else an open-addressing hash
+ * table; smc_set_map_lookup forces any of them), the int32
  * [n, 27] neighbour map (-1 = absent), the per-offset pair lists (stable
  * compaction of each map column, ascending output row), and the tile
  * schedule used by the tensor-core conv.  coords may be freed
@@ -348,6 +349,18 @@ SMC_API int smc_map_pairs(const smc_map* map, const int32_t** in_idx, const int3
  */
 SMC_API int smc_map_schedule(const smc_map* map, const int32_t** perm);
 
+/*
+ * Schedule segment (this library's own): the sort of smc_map_schedule runs
+ * within each segment of `rows` consecutive input rows, segments kept in
+ * input order, so that the tiles in flight at once gather from a window of
+ * nearby rows.  rows = 0 (the default): the whole map is one segment;
+ * rows > 0: a multiple of 2048; -1 restores the default.  Segments cut the
+ * conv's DRAM reads on maps whose features exceed L2 when the input rows are
+ * in a spatially coherent order, at some cost in skipped offsets.  Applies
+ * to maps built after the call.  SMC_E_ARG otherwise.
+ */
+SMC_API int smc_set_schedule_segment(int64_t rows);
+
 /* Release a map (its memory returns to the library's pool, ordered on the
  * build stream).  Work on other streams that reads the map must have
  * completed. */
@@ -376,9 +389,11 @@ SMC_API const char* smc_strerror(int code);
  *   the process so far (memsets and copies excluded).
  * smc_set_map_lookup: lookup structure of later builds: 0 = by size
  *   (default: a dense int32 index grid over the batch x Z x Y x X box when it
- *   has at most 2^28 sites and at most 256 sites per voxel, else a hash
- *   table), 1 = hash table, 2 = dense grid whenever the box has at most 2^28
- *   sites.  Maps are identical either way.  A forced hash capacity
+ *   has at most 2^28 sites and at most 256 sites per voxel -- cleared at
+ *   every build up to 2^23 sites, above that left uncleared behind a cleared
+ *   occupancy bitmap of one bit per site -- else a hash table), 1 = hash
+ *   table, 2 = cleared dense grid and 3 = dense grid with occupancy bitmap,
+ *   each whenever the box has at most 2^28 sites.  Maps are identical either way.  A forced hash capacity
  *   (smc_set_hash_capacity) always selects the hash table.  SMC_E_ARG for
  *   any other value.
  * smc_set_conv_variant: tensor-core conv kernel for later convs (bf16/fp16

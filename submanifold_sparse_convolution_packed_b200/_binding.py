@@ -32,7 +32,7 @@ EXPORTS = [
     "smc_build_map_async", "smc_map_wait", "smc_neighbour_map_noalloc", "smc_set_conv_variant",
     "smc_set_map_lookup", "smc_map_stream_wait", "smc_subdivide", "smc_conv_ex", "smc_group_stats",
     "smc_group_norm", "smc_downsample", "smc_upsample", "smc_set_conv_epilogue",
-    "smc_set_alloc_fail_after", "smc_set_wait_limit_ns", "smc_set_scan_hold",
+    "smc_set_alloc_fail_after", "smc_set_wait_limit_ns", "smc_set_scan_hold", "smc_set_schedule_segment",
 ]
 
 
@@ -87,6 +87,7 @@ def lib() -> ctypes.CDLL:
         L.smc_set_alloc_fail_after.argtypes = [i64]
         L.smc_set_wait_limit_ns.argtypes = [i64]
         L.smc_set_scan_hold.argtypes = [i64]
+        L.smc_set_schedule_segment.argtypes = [i64]
         for name in EXPORTS:
             if name != "smc_strerror":
                 getattr(L, name).restype = ctypes.c_int
@@ -517,6 +518,13 @@ def set_alloc_fail_after(k: int) -> None:
 def set_wait_limit_ns(ns: int) -> None:
     """Bound of the scans' device-side waits, in ns (0 = the default 2 s)."""
     _check(lib().smc_set_wait_limit_ns(int(ns)), "smc_set_wait_limit_ns")
+
+
+def set_schedule_segment(rows: int) -> None:
+    """Sort the tile schedule within segments of `rows` consecutive input rows
+    (0 = the whole map, the default; -1 = the default; else a multiple of 2048;
+    smc_set_schedule_segment).  Applies to maps built afterwards."""
+    _check(lib().smc_set_schedule_segment(int(rows)), "smc_set_schedule_segment")
 
 
 def set_scan_hold(ticket: int) -> None:

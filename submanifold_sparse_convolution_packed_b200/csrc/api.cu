@@ -64,6 +64,8 @@ std::atomic<int32_t> g_map_lookup{0};
 // Largest box (batch * Z * Y * X sites) that gets a dense index grid: 1 GB of
 // int32, cleared at every build.
 constexpr double kDenseMaxSites = 268435456.0;
+// Boxes above this many sites (a 32 MB grid) take the occupancy-bitmap grid.
+constexpr double kOccMinSites = 8388608.0;
 
 constexpr int kMaxDevices = 64;
 
@@ -331,7 +333,10 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   const int64_t forced = g_capacity_override.load();
   const int lookup = g_map_lookup.load();
   const bool dense = !sub && forced == 0 && sites <= kDenseMaxSites &&
-                     (lookup == 2 || (lookup == 0 && sites <= 256.0 * static_cast<double>(n)));
+                     (lookup == 2 || lookup == 3 || (lookup == 0 && sites <= 256.0 * static_cast<double>(n)));
+  // A grid larger than L2 is not cleared: an occupancy bitmap, 1/32 of its
+  // size, is cleared instead and guards every read of it.
+  const bool occ = dense && (lookup == 3 || (lookup == 0 && sites > kOccMinSites));
   const bool wide = !dense && sites > 4294967294.0;  // packed slots need keys < 2^32 - 1
   int lg = 4;
   // Packed slots: load <= 1/4, so lookups (which read 2-slot groups) resolve
@@ -342,8 +347,8 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   const int64_t cap = 1ll << lg;
   const int nb = smc::map_nblocks(n);
   const int64_t Lmap = 27ll * nb;
-  const int nblk = smc::radix_nblocks(n);
-  const int64_t Lrad = static_cast<int64_t>(smc::radix_bins()) * nblk;
+  const int radix_cps = smc::radix_seg_chunks(n);
+  const int64_t Lrad = smc::radix_hist_len(n, radix_cps);
   const int64_t pair_cap = 27ll * n;
 
   Carve keep;
@@ -373,6 +378,7 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   const size_t o_st2 = tmp.take<unsigned long long>(smc::scan_status_len(Lrad));
   const size_t o_h1 = tmp.take<int32_t>(Lrad);
   const size_t o_h2 = tmp.take<int32_t>(Lrad);
+  const size_t o_occ = tmp.take<uint32_t>(occ ? (static_cast<size_t>(sites) + 31) / 32 : 0);
   const size_t zero_bytes = tmp.off - o_err;
 
   void* tp = nullptr;
@@ -412,7 +418,8 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   a.Z = grid[0];
   a.Y = grid[1];
   a.X = grid[2];
-  a.kind = dense ? smc::kMapDense : (wide ? smc::kMapWide : smc::kMapPacked);
+  a.kind = occ ? smc::kMapDenseOcc : dense ? smc::kMapDense : (wide ? smc::kMapWide : smc::kMapPacked);
+  a.occ = occ ? reinterpret_cast<uint32_t*>(T + o_occ) : nullptr;
   a.table = reinterpret_cast<unsigned long long*>(T + o_table);
   a.lg = lg;
   a.err = err;
@@ -425,6 +432,7 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   a.scan_status = reinterpret_cast<unsigned long long*>(T + o_st0);
   a.scan_ticket = tickets;
   a.hist1 = reinterpret_cast<int32_t*>(T + o_h1);
+  a.radix_cps = radix_cps;
   a.info = reinterpret_cast<int64_t*>(T + o_err + offsetof(HostSlot, info));
   a.in_idx = m->in_idx;
   a.out_idx = m->out_idx;
@@ -432,6 +440,7 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   b.gkey = a.gkey;
   b.n = n;
   b.hist1 = a.hist1;
+  b.radix_cps = radix_cps;
   b.hist2 = reinterpret_cast<int32_t*>(T + o_h2);
   b.hoff = reinterpret_cast<int64_t*>(T + o_hoff);
   b.status1 = reinterpret_cast<unsigned long long*>(T + o_st1);
@@ -449,7 +458,7 @@ int build_async(const int32_t* coords, int64_t n, int32_t batch, const int32_t g
   // release of the scratch.  A conv enqueued on s behind the build waits for
   // the schedule only, and overlaps the pair lists.
   cudaError_t ce = m->prof[0] ? cudaEventRecord(m->prof[0], s) : cudaSuccess;  // the clears count as lookups
-  if (ce == cudaSuccess) ce = cudaMemsetAsync(T + o_table, 0xFF, table_bytes, s);
+  if (ce == cudaSuccess && !occ) ce = cudaMemsetAsync(T + o_table, 0xFF, table_bytes, s);
   if (ce == cudaSuccess) ce = cudaMemsetAsync(T + o_err, 0, zero_bytes, s);
   if (ce == cudaSuccess && sub) {
     ce = cudaMemsetAsync(m->tile_mask, 0, a.nzero * sizeof(uint32_t), s);  // k_insert clears them otherwise
@@ -574,8 +583,15 @@ int smc_set_scan_hold(int64_t ticket) {
   return SMC_OK;
 }
 
+int smc_set_schedule_segment(int64_t rows) {
+  if (rows == -1) rows = smc::kScheduleSegmentDefault;
+  if (rows < 0 || rows % 2048 != 0) return SMC_E_ARG;
+  smc::set_schedule_segment_rows(rows);
+  return SMC_OK;
+}
+
 int smc_set_map_lookup(int32_t mode) {
-  if (mode < 0 || mode > 2) return SMC_E_ARG;
+  if (mode < 0 || mode > 3) return SMC_E_ARG;
   g_map_lookup.store(mode);
   return SMC_OK;
 }

@@ -10,7 +10,9 @@
 namespace smc {
 
 // Lookup structure of a map build (see map_build.cu).
-enum MapKind : int { kMapPacked = 0, kMapWide = 1, kMapDense = 2 };
+// kMapDenseOcc: the dense grid is not cleared; an occupancy bitmap (one bit
+// per site, cleared) says which of its entries this build wrote.
+enum MapKind : int { kMapPacked = 0, kMapWide = 1, kMapDense = 2, kMapDenseOcc = 3 };
 
 struct MapBuildArgs {
   const int32_t* coords;  // [n, 4] (b, z, y, x)
@@ -18,6 +20,8 @@ struct MapBuildArgs {
   int32_t batch, Z, Y, X;
   int kind;                    // MapKind
   unsigned long long* table;   // hash: 2^lg slots pre-filled with ~0; dense: int32 grid pre-filled with -1
+                               // (kMapDenseOcc: int32 grid, not cleared)
+  uint32_t* occ;               // kMapDenseOcc: occupancy bitmap, one bit per site, zeroed
   int lg;
   uint32_t* err;               // error bits (zeroed)
   uint32_t* zero;              // [nzero] words k_insert clears (the tile tap masks)
@@ -28,7 +32,8 @@ struct MapBuildArgs {
   int64_t* block_offsets;      // [27, nblocks]
   unsigned long long* scan_status;  // [scan_status_len(27 * nblocks)], zeroed
   uint32_t* scan_ticket;       // zeroed
-  int32_t* hist1;              // [bins, radix nblk], zeroed: first schedule digit per chunk
+  int32_t* hist1;              // [radix_hist_len], zeroed: first schedule digit per chunk
+  int radix_cps;               // radix chunks per schedule segment (radix_seg_chunks)
   int64_t* info;               // [28]: offsets of the per-offset pair lists
   int32_t* in_idx;             // [27 n] capacity
   int32_t* out_idx;            // [27 n] capacity
@@ -37,10 +42,11 @@ struct MapBuildArgs {
 struct ScheduleArgs {
   const uint32_t* gkey;   // [n]
   int64_t n;
-  int32_t* hist1;         // [bins, nblk] filled by the neighbour kernel
-  int32_t* hist2;         // [bins, nblk] zeroed
-  int64_t* hoff;          // [bins, nblk]
-  unsigned long long* status1;  // [scan_status_len(bins * nblk)] each, zeroed
+  int radix_cps;          // radix chunks per schedule segment (radix_seg_chunks)
+  int32_t* hist1;         // [radix_hist_len] filled by the neighbour kernel
+  int32_t* hist2;         // [radix_hist_len] zeroed
+  int64_t* hoff;          // [radix_hist_len]
+  unsigned long long* status1;  // [scan_status_len(radix_hist_len)] each, zeroed
   unsigned long long* status2;
   uint32_t* tickets;      // [2], zeroed
   uint32_t* key_tmp;      // [n]
@@ -58,6 +64,15 @@ void count_launches(int k);
 int map_nblocks(int64_t n);
 int radix_nblocks(int64_t n);
 int radix_bins();
+// The tile schedule sorts rows within segments of consecutive input rows
+// (0 = the whole map is one segment).  radix_seg_chunks: 2048-row radix
+// chunks per segment for a map of n rows (the segment length in force now);
+// radix_hist_len: histogram length for that many chunks per segment.
+constexpr int64_t kScheduleSegmentDefault = 0;
+void set_schedule_segment_rows(int64_t rows);
+int64_t schedule_segment_rows();
+int radix_seg_chunks(int64_t n);
+int64_t radix_hist_len(int64_t n, int cps);
 int64_t scan_status_len(int64_t L);
 // Bound of the look-back scans' waits on their predecessors (2 s unless a
 // test sets it) and the test hook that holds one scan segment back (-1 = none).

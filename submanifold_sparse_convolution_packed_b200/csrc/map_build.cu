@@ -19,6 +19,7 @@
 //                 Each pass is one look-back scan of its histogram plus one
 //                 scatter; the first scatter also counts the second digit,
 //                 the second one ORs the tile tap masks.
+#include <atomic>
 #include <cstdint>
 #include <type_traits>
 
@@ -35,6 +36,14 @@ constexpr int kRadixThreads = 256;
 constexpr int kRadixRounds = 8;
 constexpr int kRadixChunk = kRadixThreads * kRadixRounds;  // rows per radix block
 static_assert(kRadixChunk % kMapBlock == 0, "a radix chunk is a whole number of map blocks");
+
+// Radix histograms are laid out segment by segment: [segment][digit][chunk of
+// the segment], cps chunks per segment.  Scanning that layout in order sorts
+// every segment of cps * kRadixChunk consecutive rows on its own and keeps the
+// segments in input order (cps = all chunks: one stable sort of the map).
+__host__ __device__ __forceinline__ int64_t hist_index(uint32_t digit, int64_t chunk, int cps) {
+  return ((chunk / cps) * kRadixBins + digit) * cps + chunk % cps;
+}
 constexpr uint64_t kFib = 0x9E3779B97F4A7C15ull;
 
 __device__ __forceinline__ uint64_t slot_of(uint64_t key, int lg) { return (key * kFib) >> (64 - lg); }
@@ -50,13 +59,15 @@ __device__ __forceinline__ uint64_t site_key(int4 c, int32_t Z, int32_t Y, int32
 
 // Lookup structures (MapKind): packed hash slots, one word (key << 32) | row,
 // for keys < 2^32 - 1; wide hash slots, two words, key then row; or a dense
-// index grid, one int32 row (-1 = empty) per site of the batch x Z x Y x X
-// box, for boxes small enough to clear at every build.
+// index grid, one int32 row per site of the batch x Z x Y x X box, either
+// cleared to -1 at every build (kMapDense) or left as it is and read only
+// where a cleared occupancy bitmap, one bit per site, has the site's bit set
+// (kMapDenseOcc: a 32x smaller clear for boxes much larger than L2).
 template <int kKind>
 __global__ void __launch_bounds__(256) k_insert(const int4* __restrict__ coords, int64_t n, int32_t batch,
                                                 int32_t Z, int32_t Y, int32_t X,
-                                                unsigned long long* table, int lg, uint32_t* err,
-                                                uint32_t* __restrict__ zero, int64_t nzero) {
+                                                unsigned long long* table, int lg, uint32_t* occ,
+                                                uint32_t* err, uint32_t* __restrict__ zero, int64_t nzero) {
   const uint64_t mask = (1ull << lg) - 1;
   // words later kernels accumulate into (the tile tap masks)
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nzero;
@@ -73,6 +84,14 @@ __global__ void __launch_bounds__(256) k_insert(const int4* __restrict__ coords,
     if (kKind == kMapDense) {
       const int prev = atomicCAS(reinterpret_cast<int*>(table) + key, -1, static_cast<int>(v));
       if (prev != -1) atomicOr(err, kErrDuplicate);
+      continue;
+    }
+    if (kKind == kMapDenseOcc) {
+      // the first row to set the site's bit owns the grid entry; the entry is
+      // read only after this kernel, so no later reader sees it unwritten
+      const uint32_t bit = 1u << (key & 31u);
+      if (atomicOr(occ + (key >> 5), bit) & bit) atomicOr(err, kErrDuplicate);
+      else reinterpret_cast<int32_t*>(table)[key] = static_cast<int32_t>(v);
       continue;
     }
     uint64_t s = slot_of(key, lg);
@@ -149,7 +168,11 @@ __device__ __forceinline__ uint32_t key_hits(uint32_t k) {
 // from the finer grouping (tap efficiency 0.855 vs 0.882 on the 6-shell
 // 128^3 workload, a 2% longer conv).
 constexpr int64_t kOnePassRows = 131072;
+
 __host__ __device__ __forceinline__ bool schedule_one_pass(int64_t n) { return n <= kOnePassRows; }
+
+// Schedule segments are whole radix chunks (see set_schedule_segment_rows).
+static_assert(kScheduleSegmentDefault % kRadixChunk == 0, "segments are whole radix chunks");
 
 // The end of a 256-row block of a map-building kernel, once each thread's row
 // is in s_nbr and its hit mask and schedule key are known: the first radix
@@ -158,7 +181,7 @@ __host__ __device__ __forceinline__ bool schedule_one_pass(int64_t n) { return n
 __device__ __forceinline__ void emit_map_block(const int32_t* s_nbr, int32_t (*s_cnt)[kTaps], uint32_t hits,
                                                uint32_t gk, int64_t base, int64_t n, int32_t* __restrict__ nbr,
                                                int32_t* __restrict__ block_counts, int nblocks,
-                                               int32_t* __restrict__ hist1, int radix_nblk) {
+                                               int32_t* __restrict__ hist1, int radix_cps) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t v = base + tid;
   if (hist1) {
@@ -168,7 +191,7 @@ __device__ __forceinline__ void emit_map_block(const int32_t* s_nbr, int32_t (*s
     const uint32_t digit = v < n ? ((gk >> shift) & (kRadixBins - 1)) : 0xFFFFFFFFu;
     const uint32_t peers = __match_any_sync(0xffffffffu, digit);
     if (v < n && (__ffs(peers) - 1) == lane)
-      atomicAdd(&hist1[static_cast<int64_t>(digit) * radix_nblk + (base / kRadixChunk)], __popc(peers));
+      atomicAdd(&hist1[hist_index(digit, base / kRadixChunk, radix_cps)], __popc(peers));
   }
 #pragma unroll
   for (int d = 0; d < kTaps; ++d) {
@@ -215,12 +238,50 @@ __device__ __forceinline__ uint32_t dense_row_lookups(const int32_t* __restrict_
   return hits;
 }
 
+// The same 27 lookups over a grid that was not cleared: each line's three
+// sites are first looked up in the occupancy bitmap (one or two words), and
+// only sites whose bit is set read the grid.
+__device__ __forceinline__ uint32_t dense_occ_row_lookups(const int32_t* __restrict__ g,
+                                                          const uint32_t* __restrict__ occ, int4 c, uint64_t key,
+                                                          int32_t Z, int32_t Y, int32_t X, int32_t* out) {
+  const int64_t sz = static_cast<int64_t>(Y) * X;
+  uint32_t hits = 0;
+#pragma unroll
+  for (int l = 0; l < 9; ++l) {
+    const int dz = l / 3 - 1, dy = l % 3 - 1;
+    const bool line = c.y + dz >= 0 && c.y + dz < Z && c.z + dy >= 0 && c.z + dy < Y;
+    const int64_t at = static_cast<int64_t>(key) + dz * sz + static_cast<int64_t>(dy) * X;
+    uint32_t b3 = 0;  // bit j: site at - 1 + j is occupied
+    if (line) {
+      const int64_t lo = c.w > 0 ? at - 1 : at;       // first site of the run inside the box
+      const int64_t hi = c.w + 1 < X ? at + 1 : at;   // last one
+      const uint32_t wl = __ldg(occ + (lo >> 5));
+      const uint32_t wh = (hi >> 5) != (lo >> 5) ? __ldg(occ + (hi >> 5)) : wl;
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        const int64_t k = at - 1 + j;
+        if (k < lo || k > hi) continue;
+        const uint32_t w = (k >> 5) == (lo >> 5) ? wl : wh;
+        b3 |= ((w >> (k & 31)) & 1u) << j;
+      }
+    }
+    const int32_t r0 = (b3 & 1u) ? __ldg(g + at - 1) : -1;
+    const int32_t r1 = (b3 & 2u) ? __ldg(g + at) : -1;
+    const int32_t r2 = (b3 & 4u) ? __ldg(g + at + 1) : -1;
+    out[3 * l + 0] = r0;
+    out[3 * l + 1] = r1;
+    out[3 * l + 2] = r2;
+    hits |= b3 << (3 * l);
+  }
+  return hits;
+}
+
 template <int kKind>
 __global__ void __launch_bounds__(kMapBlock) k_neighbours(
     const int4* __restrict__ coords, int64_t n, int32_t batch, int32_t Z, int32_t Y, int32_t X,
-    const unsigned long long* __restrict__ table, int lg, int32_t* __restrict__ nbr,
-    uint32_t* __restrict__ gkey, int32_t* __restrict__ block_counts, int nblocks,
-    int32_t* __restrict__ hist1, int radix_nblk) {
+    const unsigned long long* __restrict__ table, int lg, const uint32_t* __restrict__ occ,
+    int32_t* __restrict__ nbr, uint32_t* __restrict__ gkey, int32_t* __restrict__ block_counts, int nblocks,
+    int32_t* __restrict__ hist1, int radix_cps) {
   __shared__ int32_t s_nbr[kMapBlock * kTaps];
   __shared__ int32_t s_cnt[kMapBlock / 32][kTaps];
   const uint64_t mask = (1ull << lg) - 1;
@@ -241,6 +302,9 @@ __global__ void __launch_bounds__(kMapBlock) k_neighbours(
     const int64_t sz = static_cast<int64_t>(Y) * X;
     if (kKind == kMapDense) {
       hits = dense_row_lookups(reinterpret_cast<const int32_t*>(table), c, key, Z, Y, X, s_nbr + tid * kTaps);
+    } else if (kKind == kMapDenseOcc) {
+      hits = dense_occ_row_lookups(reinterpret_cast<const int32_t*>(table), occ, c, key, Z, Y, X,
+                                   s_nbr + tid * kTaps);
     } else if (kKind == kMapWide) {
       // two-word slots: plain linear probing per lookup
 #pragma unroll 1
@@ -319,7 +383,7 @@ __global__ void __launch_bounds__(kMapBlock) k_neighbours(
     gk = group_key(hits);
     gkey[v] = gk;
   }
-  emit_map_block(s_nbr, s_cnt, hits, gk, base, n, nbr, block_counts, nblocks, hist1, radix_nblk);
+  emit_map_block(s_nbr, s_cnt, hits, gk, base, n, nbr, block_counts, nblocks, hist1, radix_cps);
 }
 
 // ------------------------------------------------------------ subdivision
@@ -406,7 +470,7 @@ __global__ void __launch_bounds__(kEmitBlock) k_subdiv_emit(const int4* __restri
 __global__ void __launch_bounds__(kMapBlock) k_subdiv_neighbours(
     const int32_t* __restrict__ parent_nbr, const int32_t* __restrict__ child_src,
     const int32_t* __restrict__ remap, int64_t m, int32_t* __restrict__ nbr, uint32_t* __restrict__ gkey,
-    int32_t* __restrict__ block_counts, int nblocks, int32_t* __restrict__ hist1, int radix_nblk) {
+    int32_t* __restrict__ block_counts, int nblocks, int32_t* __restrict__ hist1, int radix_cps) {
   __shared__ int32_t s_nbr[kMapBlock * kTaps];
   __shared__ int32_t s_cnt[kMapBlock / 32][kTaps];
   const int tid = threadIdx.x;
@@ -430,7 +494,7 @@ __global__ void __launch_bounds__(kMapBlock) k_subdiv_neighbours(
     gk = group_key(hits);
     gkey[v] = gk;
   }
-  emit_map_block(s_nbr, s_cnt, hits, gk, base, m, nbr, block_counts, nblocks, hist1, radix_nblk);
+  emit_map_block(s_nbr, s_cnt, hits, gk, base, m, nbr, block_counts, nblocks, hist1, radix_cps);
 }
 
 // The block's share of every pair list, from its rows of the map staged in
@@ -659,7 +723,7 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_lookback(const int32_t* _
 
 // ------------------------------------------------------------ radix sort
 // Stable scatter of one radix pass over a histogram already scanned into
-// `offsets` ([bins, nblk], digit-major).  Warp w of a block ranks elements
+// `offsets` (laid out by hist_index, cps chunks per segment).  Warp w of a block ranks elements
 // 256w .. 256w + 255 of the block's chunk in 8 rounds of 32, keeping a
 // warp-private count per digit in shared memory (no block barrier between
 // rounds); the 8 warps' counts are then scanned per digit on top of the
@@ -672,7 +736,7 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_lookback(const int32_t* _
 template <bool kLast>
 __global__ void __launch_bounds__(kRadixThreads) k_radix_scatter(
     const uint32_t* __restrict__ keys_in, const int32_t* __restrict__ vals_in, int64_t n, int shift,
-    const int64_t* __restrict__ offsets, int nblk, uint32_t* __restrict__ keys_out,
+    const int64_t* __restrict__ offsets, int cps, uint32_t* __restrict__ keys_out,
     int32_t* __restrict__ vals_out, int32_t* __restrict__ hist_next, uint32_t* __restrict__ tile_mask,
     uint32_t* err) {
   constexpr int kWarps = kRadixThreads / 32;
@@ -704,7 +768,7 @@ __global__ void __launch_bounds__(kRadixThreads) k_radix_scatter(
   }
   __syncthreads();
   for (int d = tid; d < kRadixBins; d += kRadixThreads) {
-    int64_t run = offsets[static_cast<int64_t>(d) * nblk + blockIdx.x];
+    int64_t run = offsets[hist_index(static_cast<uint32_t>(d), blockIdx.x, cps)];
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
       const int32_t c = s_cnt[w][d];
@@ -737,7 +801,7 @@ __global__ void __launch_bounds__(kRadixThreads) k_radix_scatter(
                                     : 0xFFFFFFFFu;
       const uint32_t grp = __match_any_sync(0xffffffffu, tag);
       if (tag != 0xFFFFFFFFu && (__ffs(grp) - 1) == lane)
-        atomicAdd(&hist_next[static_cast<int64_t>(tag >> 21) * nblk + (tag & ((1u << 21) - 1))], __popc(grp));
+        atomicAdd(&hist_next[hist_index(tag >> 21, tag & ((1u << 21) - 1), cps)], __popc(grp));
     } else {
       // tile tap masks: a warp whose rows all land in one tile (dense data)
       // ORs them first; otherwise every row ORs its own mask in
@@ -771,20 +835,46 @@ int map_nblocks(int64_t n) { return static_cast<int>((n + kMapBlock - 1) / kMapB
 int radix_nblocks(int64_t n) { return static_cast<int>((n + kRadixChunk - 1) / kRadixChunk); }
 int radix_bins() { return kRadixBins; }
 
+// Schedule segment length in rows (0 = one segment, the default).  Segments
+// keep the rows of each wave of conv tiles within a window of consecutive
+// input rows, so a map whose input order is spatially coherent (C order,
+// subdivision order) gathers from a feature working set that stays in L2.
+// Measured on B200 with 131072-row segments: the conv's DRAM reads on the
+// 512^3 decoder stage (64 channels, 1.26M voxels) fell from 897 to 304 MB
+// with its time unchanged (0.49 ms: the gathers' L2 -> SM rate, not DRAM,
+// bounds it), while the split key groups cost tap efficiency (0.950 -> 0.891
+// on the four-item 256^3 set, a 3% longer conv).  So it is off by default.
+static std::atomic<int64_t> g_segment_rows{kScheduleSegmentDefault};
+void set_schedule_segment_rows(int64_t rows) { g_segment_rows.store(rows); }
+int64_t schedule_segment_rows() { return g_segment_rows.load(); }
+int radix_seg_chunks(int64_t n) {
+  const int nblk = radix_nblocks(n);
+  const int64_t rows = g_segment_rows.load();
+  if (rows <= 0 || nblk == 0) return nblk > 0 ? nblk : 1;
+  const int64_t cps = rows / kRadixChunk;
+  return cps >= nblk ? nblk : static_cast<int>(cps);
+}
+int64_t radix_hist_len(int64_t n, int cps) {
+  const int64_t nblk = radix_nblocks(n);
+  const int64_t nseg = (nblk + cps - 1) / cps;
+  return nseg * cps * kRadixBins;
+}
+
 cudaError_t launch_map_lookups(const MapBuildArgs& a, cudaStream_t s) {
   const int64_t n = a.n;
   if (n == 0) return cudaSuccess;
   const int nb = map_nblocks(n);
-  const int rnb = radix_nblocks(n);
   const int grid_ins = static_cast<int>((n + 255) / 256);
   auto run = [&](auto kind) {
     constexpr int K = decltype(kind)::value;
     k_insert<K><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.batch, a.Z, a.Y, a.X,
-                                         a.table, a.lg, a.err, a.zero, a.nzero);
+                                         a.table, a.lg, a.occ, a.err, a.zero, a.nzero);
     k_neighbours<K><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(a.coords), n, a.batch, a.Z, a.Y, a.X,
-                                             a.table, a.lg, a.nbr, a.gkey, a.block_counts, nb, a.hist1, rnb);
+                                             a.table, a.lg, a.occ, a.nbr, a.gkey, a.block_counts, nb, a.hist1,
+                                             a.radix_cps);
   };
   if (a.kind == kMapDense) run(std::integral_constant<int, kMapDense>());
+  else if (a.kind == kMapDenseOcc) run(std::integral_constant<int, kMapDenseOcc>());
   else if (a.kind == kMapWide) run(std::integral_constant<int, kMapWide>());
   else run(std::integral_constant<int, kMapPacked>());
   count_launches(2);
@@ -845,7 +935,7 @@ cudaError_t launch_subdiv_lookups(const MapBuildArgs& a, const int32_t* parent_n
   if (n == 0) return cudaSuccess;
   const int nb = map_nblocks(n);
   k_subdiv_neighbours<<<nb, kMapBlock, 0, s>>>(parent_nbr, child_src, remap, n, a.nbr, a.gkey, a.block_counts, nb,
-                                               a.hist1, radix_nblocks(n));
+                                               a.hist1, a.radix_cps);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -859,9 +949,9 @@ cudaError_t launch_neighbour_map_only(const int32_t* coords, int64_t n, int32_t 
   const int nb = map_nblocks(n);
   const int grid_ins = static_cast<int>((n + 255) / 256);
   k_insert<kMapPacked><<<grid_ins, 256, 0, s>>>(reinterpret_cast<const int4*>(coords), n, batch, Z, Y, X, table,
-                                                lg, err, nullptr, 0);
-  k_neighbours<kMapPacked><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(coords), n, batch, Z, Y, X, table, lg, nbr,
-                                               gkey, block_counts, nb, nullptr, 0);
+                                                lg, nullptr, err, nullptr, 0);
+  k_neighbours<kMapPacked><<<nb, kMapBlock, 0, s>>>(reinterpret_cast<const int4*>(coords), n, batch, Z, Y, X, table, lg,
+                                               nullptr, nbr, gkey, block_counts, nb, nullptr, 0);
   count_launches(2);
   return cudaGetLastError();
 }
@@ -870,13 +960,14 @@ cudaError_t launch_schedule(const ScheduleArgs& a, cudaStream_t s) {
   const int64_t n = a.n;
   if (n == 0) return cudaSuccess;
   const int nblk = radix_nblocks(n);
-  const int64_t L = static_cast<int64_t>(kRadixBins) * nblk;
+  const int cps = a.radix_cps;
+  const int64_t L = radix_hist_len(n, cps);
   if (schedule_one_pass(n)) {
     // small maps: one stable pass on the high 10 bits (the 8 corner and 2 edge
     // offsets); the histogram of that digit comes from the neighbour kernel
     cudaError_t e = scan_i32(a.hist1, L, a.hoff, a.status1, a.tickets, a.err, nullptr, 1, s);
     if (e != cudaSuccess) return e;
-    k_radix_scatter<true><<<nblk, kRadixThreads, 0, s>>>(a.gkey, nullptr, n, kRadixBits, a.hoff, nblk, nullptr,
+    k_radix_scatter<true><<<nblk, kRadixThreads, 0, s>>>(a.gkey, nullptr, n, kRadixBits, a.hoff, cps, nullptr,
                                                          a.perm, nullptr, a.tile_mask, a.err);
     count_launches(1);
     return cudaGetLastError();
@@ -884,13 +975,13 @@ cudaError_t launch_schedule(const ScheduleArgs& a, cudaStream_t s) {
   // pass 1: low 10 bits, rows in input order (histogram from the neighbour kernel)
   cudaError_t e = scan_i32(a.hist1, L, a.hoff, a.status1, a.tickets, a.err, nullptr, 1, s);
   if (e != cudaSuccess) return e;
-  k_radix_scatter<false><<<nblk, kRadixThreads, 0, s>>>(a.gkey, nullptr, n, 0, a.hoff, nblk, a.key_tmp,
+  k_radix_scatter<false><<<nblk, kRadixThreads, 0, s>>>(a.gkey, nullptr, n, 0, a.hoff, cps, a.key_tmp,
                                                         a.val_tmp, a.hist2, nullptr, a.err);
   count_launches(1);
   // pass 2: high 10 bits
   e = scan_i32(a.hist2, L, a.hoff, a.status2, a.tickets + 1, a.err, nullptr, 1, s);
   if (e != cudaSuccess) return e;
-  k_radix_scatter<true><<<nblk, kRadixThreads, 0, s>>>(a.key_tmp, a.val_tmp, n, kRadixBits, a.hoff, nblk,
+  k_radix_scatter<true><<<nblk, kRadixThreads, 0, s>>>(a.key_tmp, a.val_tmp, n, kRadixBits, a.hoff, cps,
                                                        nullptr, a.perm, nullptr, a.tile_mask, a.err);
   count_launches(1);
   return cudaGetLastError();

@@ -80,7 +80,7 @@ def sample_rows(n, k, seed):
 
 
 # ------------------------------------------------------------------ map
-@pytest.fixture(params=[1, 2], ids=["hash", "dense_grid"])
+@pytest.fixture(params=[1, 2, 3], ids=["hash", "dense_grid", "dense_occupancy"])
 def map_lookup(request):
     """Runs a test with each lookup structure of the map build."""
     smc.set_map_lookup(request.param)
@@ -91,17 +91,23 @@ def map_lookup(request):
 # The tile order of the tensor-core conv: rows stably sorted by a 20-bit key
 # whose bits, most significant first, say whether the 8 corner offsets and
 # then the 12 edge offsets have a neighbour; maps of at most ONE_PASS_ROWS
-# rows are sorted on the key's high 10 bits alone (one radix pass).
+# rows are sorted on the key's high 10 bits alone (one radix pass).  The sort
+# runs within segments of SEGMENT_ROWS consecutive input rows, the segments
+# kept in input order (0: the whole map is one segment).
 _KEY_TAPS = [0, 2, 6, 8, 18, 20, 24, 26, 1, 3, 5, 7, 9, 11, 15, 17, 19, 21, 23, 25]
 ONE_PASS_ROWS = 131072
+SEGMENT_ROWS = 0
 
 
-def expected_schedule(nbr):
-    key = np.zeros(nbr.shape[0], dtype=np.int64)
+def expected_schedule(nbr, segment=SEGMENT_ROWS):
+    n = nbr.shape[0]
+    key = np.zeros(n, dtype=np.int64)
     for i, d in enumerate(_KEY_TAPS):
         key |= (nbr[:, d] >= 0).astype(np.int64) << (19 - i)
-    if nbr.shape[0] <= ONE_PASS_ROWS:
+    if n <= ONE_PASS_ROWS:
         key >>= 10
+    if segment:
+        key |= (np.arange(n, dtype=np.int64) // segment) << 20
     return np.argsort(key, kind="stable").astype(np.int32)
 
 
@@ -123,6 +129,58 @@ def test_map_bit_exact(oracle_mod, name, map_lookup):
     np.testing.assert_array_equal(go.cpu().numpy(), out_idx)
     perm = m.schedule().cpu().numpy()
     np.testing.assert_array_equal(perm, expected_schedule(ref))
+
+
+@pytest.mark.parametrize("name,segment", [("shell2", 4096), ("shell2", 2048), ("varlen4", 2048),
+                                          ("varlen4", 131072), ("varlen4", 262144)])
+def test_schedule_segments(oracle_mod, name, segment):
+    """The schedule's sort runs segment by segment: one segment, a segment per
+    radix chunk, and lengths between, on the one-pass and two-pass paths."""
+    w = workload(name)
+    ref = oracle_mod.neighbour_map(w.coords, w.grid)
+    smc.set_schedule_segment(segment)
+    try:
+        m = build(w)
+    finally:
+        smc.set_schedule_segment(-1)
+    perm = m.schedule().cpu().numpy()
+    np.testing.assert_array_equal(perm, expected_schedule(ref, segment))
+    # the tile tap masks follow the order: a conv on the map stays exact
+    f, wt, b = _layer(w, "f16")
+    rows = np.sort(np.random.default_rng(5).choice(w.n, size=min(w.n, 2048), replace=False))
+    got, ref_out = _conv_pair(oracle_mod, w, m, "f16", f, wt, b, 3, 1, rows=rows)
+    check_close(got, ref_out, "f16", f"{name} conv, schedule segment {segment}")
+
+
+def test_schedule_segment_arguments():
+    lib = smc.lib()
+    assert lib.smc_set_schedule_segment(-2) == -1
+    assert lib.smc_set_schedule_segment(1000) == -1
+    assert lib.smc_set_schedule_segment(-1) == 0
+
+
+def test_map_uncleared_grid_reuse(oracle_mod):
+    """The occupancy-bitmap grid is never cleared: a build that reuses the
+    memory of an earlier build over the same box (from the library's pool)
+    finds that build's rows in it and must ignore every one of them."""
+    w = workload("shell2")
+    rng = np.random.default_rng(11)
+    smc.set_map_lookup(3)
+    try:
+        for trial in range(4):
+            keep = rng.random(w.n) < (0.3 if trial % 2 else 0.9)
+            coords = w.coords[keep]
+            coords = coords[rng.permutation(len(coords))]
+            m = smc.build_map(torch.from_numpy(coords).cuda(), w.grid, batch=2)
+            ref = oracle_mod.neighbour_map(coords, w.grid)
+            np.testing.assert_array_equal(m.nbr().cpu().numpy(), ref)
+            counts, offsets, in_idx, out_idx = oracle_mod.pair_lists(ref)
+            gi, go, _ = m.pairs()
+            np.testing.assert_array_equal(gi.cpu().numpy(), in_idx)
+            np.testing.assert_array_equal(go.cpu().numpy(), out_idx)
+            m.free()
+    finally:
+        smc.set_map_lookup(0)
 
 
 def test_map_shuffled_rows(oracle_mod, map_lookup):
