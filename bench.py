@@ -535,6 +535,8 @@ def run_gpu(args):
     dev = torch.device("cuda", local)
     init_dist(world, "nccl")
     smc.lib()
+    if args.schedule_segment is not None:
+        smc.set_schedule_segment(args.schedule_segment)
     peaks = load_peaks()
 
     w = get_workload(args.workload)
@@ -661,6 +663,7 @@ def run_gpu(args):
                 "cin": w.cin, "cout": w.cout, "step": "build_map (asynchronous entry point) + conv k=3 s=+1 on one stream, up to 4 steps enqueued ahead; every map checked and freed when its step retires",
                 "l2": "flushed before every step (256 MB write, outside the timed events)",
                 "parallelism": f"replicas x{world} (no collective on the data path)",
+                **({"schedule_segment_rows": args.schedule_segment} if args.schedule_segment is not None else {}),
             },
             "pair_tflops": round(conv_tflops, 2),
             "map_build_gbs": round(map_gbs, 1),
@@ -879,6 +882,9 @@ def main(argv=None):
                     help="shells6 (default), full128, varlen4, shell2, decoder0..decoder3")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--schedule-segment", type=int, default=None,
+                    help="sort the tile schedule within segments of this many rows (0 = whole map; default: "
+                         "the library's default)")
     ap.add_argument("--skip-configs", action="store_true",
                     help="measure the default workload only, not the other configurations")
     args = ap.parse_args(argv)

@@ -398,14 +398,18 @@ SMC_API const char* smc_strerror(int code);
  *   any other value.
  * smc_set_conv_variant: tensor-core conv kernel for later convs (bf16/fp16
  *   shapes the tensor cores take; others always use the FMA kernel): 0 =
- *   default (currently the same as 1), 1 = fused 27-tap gather-GEMM, one CTA
+ *   default (4 for a k = 3 conv with 64 output channels and no fused
+ *   activation or residual, else 1), 1 = fused 27-tap gather-GEMM, one CTA
  *   per 128-row tile, 2 = the same with CTA pairs (a cluster of two CTAs
  *   sharing M = 256 tcgen05 MMAs, each loading half of the weight block;
  *   slower on B200, where such clusters run one per TPC), 3 = per-offset
  *   gather-GEMM-scatter over the pair lists with fp32 atomic accumulation
- *   (k = 3 only; waits for the whole build; results equal to rounding).
- *   1 and 2 give identical bits.  Used to test and measure the variants.
- *   SMC_E_ARG for any other value.
+ *   (k = 3 only; waits for the whole build; results equal to rounding),
+ *   4 = fused, one CTA per two consecutive tiles, each weight stage feeding
+ *   both tiles' MMAs (k = 3 with 64 or 128 output channels and no fused
+ *   activation or residual; otherwise as 1).  1, 2 and 4 give identical
+ *   bits.  Used to test and measure the variants.  SMC_E_ARG for any other
+ *   value.
  */
 /*
  * smc_neighbour_map_noalloc -- the int32 [n, 27] neighbour map of smc_build_map

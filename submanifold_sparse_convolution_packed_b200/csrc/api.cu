@@ -603,7 +603,7 @@ int smc_set_conv_epilogue(int32_t where) {
 }
 
 int smc_set_conv_variant(int32_t variant) {
-  if (variant < 0 || variant > 3) return SMC_E_ARG;
+  if (variant < 0 || variant > 4) return SMC_E_ARG;
   smc::set_conv_variant(variant);
   return SMC_OK;
 }

@@ -21,7 +21,8 @@
 //              tile::gather4 row loads (missing neighbours are row -1, which
 //              TMA reads as zeros); then the epilogue for the same rows:
 //              tcgen05.ld, bias in fp32, rounding, 16-byte stores.
-//              (Or warps 2-9, 16 rows each, 4 issuing lanes: see kGW.)
+//              (Or warps 2-9, 16 rows each, 4 issuing lanes: see kGW; or
+//              two tiles per CTA, warps 2-9 with 32 rows each: see kMT.)
 // Pipeline stages are (tap, channel block) pairs of KB = 32 or 64 channels in
 // swizzled shared memory (64-byte or 128-byte swizzle).  Every wait is
 // bounded; on timeout the error word gets a bit and the CTA winds down.
@@ -44,9 +45,9 @@ struct TcSmemLayout {
   uint32_t a_off, b_off, bar_off, misc_off, bias_off, total;
 };
 
-__host__ __device__ inline TcSmemLayout tc_layout(int stages, int bn, int kb_elems) {
+__host__ __device__ inline TcSmemLayout tc_layout(int stages, int bn, int kb_elems, int mt = 1) {
   TcSmemLayout L;
-  const uint32_t a_bytes = static_cast<uint32_t>(kTileRows) * kb_elems * 2;
+  const uint32_t a_bytes = static_cast<uint32_t>(mt * kTileRows) * kb_elems * 2;
   const uint32_t b_bytes = static_cast<uint32_t>(bn) * kb_elems * 2;
   L.a_off = 0;
   L.b_off = L.a_off + stages * a_bytes;
@@ -87,8 +88,14 @@ struct TcParams {
 // quarter: each gathers 16 of its 32 rows (4 issuing lanes) and, in the
 // epilogue, writes half of its columns.  Selected by measurement for the
 // plain conv at three CTAs per SM.
-template <bool kPair, int kEpi, int kGW>
-__global__ void __launch_bounds__(64 + 32 * kGW, kGW == 8 ? 3 : 4) k_conv_tc(const __grid_constant__ CUtensorMap fmap,
+// kMT = 2 (with kGW = 8, plain epilogue, k = 3): the CTA owns two consecutive
+// schedule tiles and every weight stage feeds two M = 128 MMAs, one per tile,
+// into two TMEM accumulators (the union of the two tiles' tap masks is
+// issued); warps 2-5 gather and drain the first tile, warps 6-9 the second.
+// It halves the weight bytes per output row, at two CTAs per SM.
+template <bool kPair, int kEpi, int kGW, int kMT = 1>
+__global__ void __launch_bounds__(64 + 32 * kGW, kMT == 2 ? 2 : (kGW == 8 ? 3 : 4))
+    k_conv_tc(const __grid_constant__ CUtensorMap fmap,
                                                         const __grid_constant__ CUtensorMap wmap,
                                                         const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -96,7 +103,7 @@ __global__ void __launch_bounds__(64 + 32 * kGW, kGW == 8 ? 3 : 4) k_conv_tc(con
   const uint32_t sbase = (raw + 1023u) & ~1023u;  // swizzle atoms need aligned bases
   uint8_t* smem = smem_raw + (sbase - raw);
   const int bn_cta = kPair ? p.bn / 2 : p.bn;  // weight rows (output channels) this CTA loads
-  const TcSmemLayout L = tc_layout(p.stages, bn_cta, p.kb_elems);
+  const TcSmemLayout L = tc_layout(p.stages, bn_cta, p.kb_elems, kMT);
   const uint32_t bar_full = sbase + L.bar_off;
   const uint32_t bar_empty = bar_full + kMaxStages * 8;
   const uint32_t bar_acc = bar_empty + kMaxStages * 8;
@@ -106,7 +113,7 @@ __global__ void __launch_bounds__(64 + 32 * kGW, kGW == 8 ? 3 : 4) k_conv_tc(con
   const bool k3 = p.taps == kTaps;
   const uint32_t rank = kPair ? cluster_ctarank() : 0u;
   const uint32_t row_bytes = static_cast<uint32_t>(p.kb_elems) * 2;
-  const uint32_t a_bytes = kTileRows * row_bytes;
+  const uint32_t a_bytes = kMT * kTileRows * row_bytes;
   const uint32_t b_bytes = static_cast<uint32_t>(bn_cta) * row_bytes;
   const int kblocks = (p.cin + p.kb_elems - 1) / p.kb_elems;
   const int last_ksteps = (p.cin - (kblocks - 1) * p.kb_elems + 15) / 16;
@@ -115,13 +122,13 @@ __global__ void __launch_bounds__(64 + 32 * kGW, kGW == 8 ? 3 : 4) k_conv_tc(con
   // come last, and launching them first leaves the lighter tiles to fill the
   // final partial wave.
   const int64_t unit = kPair ? blockIdx.x / 2 : gridDim.x - 1 - blockIdx.x;
-  const int64_t tile0 = (unit / p.nsplit) * (kPair ? 2 : 1);  // first tile of the unit
+  const int64_t tile0 = (unit / p.nsplit) * (kPair ? 2 : kMT);  // first tile of the unit
   const int64_t tile = tile0 + rank;
   const int n0 = static_cast<int>(unit % p.nsplit) * p.bn;
   uint32_t mask = 1u;
   if (k3) {
     mask = __ldg(p.tile_mask + tile0);
-    if (kPair && tile0 + 1 < p.ntiles) mask |= __ldg(p.tile_mask + tile0 + 1);
+    if ((kPair || kMT == 2) && tile0 + 1 < p.ntiles) mask |= __ldg(p.tile_mask + tile0 + 1);
     if (p.orientation < 0) mask = mirror27(mask);
   }
 
@@ -129,11 +136,14 @@ __global__ void __launch_bounds__(64 + 32 * kGW, kGW == 8 ? 3 : 4) k_conv_tc(con
   // and its output row v, and gather tile row rg: for k = 3 its 27 neighbour
   // rows, loaded here so that the loads overlap the barrier set-up and the
   // TMEM allocation below.  With 4 gather warps r == rg.
-  constexpr int kRPW = kTileRows / kGW;  // tile rows gathered per warp
+  constexpr int kRPW = kMT * kTileRows / kGW;  // tile rows gathered per warp
   const int q = warp & 3;                // TMEM lane quarter
-  const int h = kGW == 8 ? ((warp - 2) >> 2) : 0;  // half of the quarter (rows gathered, columns written)
+  // kGW = 8: half of the quarter (rows gathered, columns written); with
+  // kMT = 2 the warp's tile instead (all of its 32 rows, all columns)
+  const int h = kGW == 8 ? ((warp - 2) >> 2) : 0;
   const int r = q * 32 + lane;
-  const int rg = q * 32 + h * kRPW + (lane % kRPW);
+  const int rg = kMT == 2 ? r : q * 32 + h * kRPW + (lane % kRPW);
+  const int64_t row0 = (kMT == 2 ? tile0 + h : tile) * kTileRows;  // first schedule entry of the warp's tile
   int32_t v = -1;
   int32_t nb[kTaps];
   // The unit's bias values go to shared memory once, so that the epilogue
@@ -150,12 +160,12 @@ __global__ void __launch_bounds__(64 + 32 * kGW, kGW == 8 ? 3 : 4) k_conv_tc(con
     }
   }
   if (warp >= 2) {
-    const int64_t g = tile * kTileRows + r;
+    const int64_t g = row0 + r;
     v = g < p.n ? (k3 ? __ldg(p.perm + g) : static_cast<int32_t>(g)) : -1;
     if (v >= p.n) v = -1;  // a schedule left incomplete by a failed build is skipped, never followed
     int32_t vg = v;
-    if (kGW != 4) {
-      const int64_t gg = tile * kTileRows + rg;
+    if (kGW != 4 && kMT == 1) {
+      const int64_t gg = row0 + rg;
       vg = gg < p.n ? (k3 ? __ldg(p.perm + gg) : static_cast<int32_t>(gg)) : -1;
       if (vg >= p.n) vg = -1;
     }
@@ -254,14 +264,20 @@ __global__ void __launch_bounds__(64 + 32 * kGW, kGW == 8 ? 3 : 4) k_conv_tc(con
             break;
           }
           tc_fence_after();
-          const uint64_t adesc = kmajor_desc(sbase + L.a_off + stage * a_bytes, row_bytes);
           const uint64_t bdesc = kmajor_desc(sbase + L.b_off + stage * b_bytes, row_bytes);
           const int ksteps = kb == kblocks - 1 ? last_ksteps : p.kb_elems / 16;
-          for (int k = 0; k < ksteps; ++k) {
-            if (kPair)
-              umma_f16_pair_elect(tmem_base, adesc + 2 * k, bdesc + 2 * k, idesc, (it > 0 || k > 0) ? 1u : 0u);
-            else
-              umma_f16_elect(tmem_base, adesc + 2 * k, bdesc + 2 * k, idesc, (it > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+          for (int t = 0; t < kMT; ++t) {
+            // tile t's rows and accumulator (columns t * BN ..)
+            const uint64_t adesc =
+                kmajor_desc(sbase + L.a_off + stage * a_bytes + t * kTileRows * row_bytes, row_bytes);
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(t * p.bn);
+            for (int k = 0; k < ksteps; ++k) {
+              if (kPair)
+                umma_f16_pair_elect(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (it > 0 || k > 0) ? 1u : 0u);
+              else
+                umma_f16_elect(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (it > 0 || k > 0) ? 1u : 0u);
+            }
           }
           if (kPair) umma_commit_pair_elect(bar_empty + 8 * stage, 3);
           else umma_commit_elect(bar_empty + 8 * stage);
@@ -311,7 +327,8 @@ __global__ void __launch_bounds__(64 + 32 * kGW, kGW == 8 ? 3 : 4) k_conv_tc(con
           }
           __syncwarp();
           if (lane < kRPW / 4) {
-            const uint32_t dst = sbase + L.a_off + stage * a_bytes + (q * 32 + h * kRPW + 4 * lane) * row_bytes;
+            const int arow = kMT == 2 ? h * kTileRows + q * 32 + 4 * lane : q * 32 + h * kRPW + 4 * lane;
+            const uint32_t dst = sbase + L.a_off + stage * a_bytes + arow * row_bytes;
             if (kPair) tma_gather4_pair(dst, &fmap, full, kb * p.kb_elems, r0, r1, r2, r3);
             else tma_gather4(dst, &fmap, full, kb * p.kb_elems, r0, r1, r2, r3);
           }
@@ -349,11 +366,12 @@ __global__ void __launch_bounds__(64 + 32 * kGW, kGW == 8 ? 3 : 4) k_conv_tc(con
       // 16-byte stores (a row's bytes are contiguous in `out`), instead of 32
       // scattered rows per store instruction.
       const bool bf = p.is_bf16 != 0;
-      const int bw = p.bn / (kGW / 4);  // columns this warp writes
-      const int c_lo = h * bw;
+      const int bw = kMT == 2 ? p.bn : p.bn / (kGW / 4);  // columns this warp writes
+      const int c_lo = kMT == 2 ? 0 : h * bw;
       const uint32_t pitch = static_cast<uint32_t>(bw) * 2u + 16u;
       uint8_t* blk = smem + L.a_off + static_cast<uint32_t>(warp - 2) * 32u * pitch;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(c_lo);
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(c_lo) +
+                             (kMT == 2 ? static_cast<uint32_t>(h * p.bn) : 0u);
       int ncols_all = p.cout - n0 - c_lo < bw ? p.cout - n0 - c_lo : bw;
       for (int c0 = 0; c0 < ncols_all; c0 += 32) {
         float acc[32];
@@ -399,7 +417,8 @@ __global__ void __launch_bounds__(64 + 32 * kGW, kGW == 8 ? 3 : 4) k_conv_tc(con
       }
     } else if (ready) {
       const bool bf = p.is_bf16 != 0;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             (kMT == 2 ? static_cast<uint32_t>(h * p.bn) : 0u);
       for (int c0 = 0; c0 < p.bn; c0 += 32) {
         if constexpr (extra) {
           if (c0 + 32 < p.bn) load_res(c0 + 32, rnext);
@@ -502,7 +521,7 @@ static uint32_t next_pow2(uint32_t x) {
 
 // Launch shape of one conv: channel split, channel block, CTA pairing and stage count.
 struct TcShape {
-  int nsplit, bn, kb_elems, stages, ctas_per_sm;
+  int nsplit, bn, kb_elems, stages, ctas_per_sm, mt;
   bool pair;
   uint32_t tmem_cols, smem;
 };
@@ -510,12 +529,13 @@ struct TcShape {
 static std::atomic<int> g_conv_variant{0};
 static std::atomic<int> g_gather_warps{0};  // 0 = by shape; 4 = always four gather warps
 
-static TcShape choose_shape(int cin, int cout, int64_t ntiles) {
+static TcShape choose_shape(int cin, int cout, int64_t ntiles, int mt) {
   TcShape t;
+  t.mt = mt;
   // At most 256 output channels (one MMA N) per CTA or CTA pair.
   t.nsplit = (cout + 255) / 256;
   t.bn = ((cout + t.nsplit - 1) / t.nsplit + 15) / 16 * 16;
-  t.tmem_cols = next_pow2(t.bn < 32 ? 32u : static_cast<uint32_t>(t.bn));
+  t.tmem_cols = next_pow2(t.bn < 32 ? 32u : static_cast<uint32_t>(mt * t.bn));
   // CTA pairs halve the weight bytes each CTA pulls through its TMA path, but
   // a cluster launch of a kernel that uses tcgen05 is limited to one cluster
   // per TPC (74 on B200, from the occupancy API and ncu), i.e. one CTA per
@@ -536,17 +556,18 @@ static TcShape choose_shape(int cin, int cout, int64_t ntiles) {
   // same per-CTA budget: sized for one CTA per SM, with eight stages, they
   // measured slower still.)
   t.ctas_per_sm = t.tmem_cols <= 64 ? 4 : (t.tmem_cols <= 128 ? 3 : 2);
+  if (mt == 2) t.ctas_per_sm = 2;  // TMEM: two accumulators of up to 128 columns
   t.kb_elems = 64;
   (void)cin;
   const uint32_t per_sm = 228u * 1024u;
   const uint32_t budget = per_sm / t.ctas_per_sm - 1024u;  // 1 KB per CTA is reserved by the system
-  const uint32_t stage_bytes = static_cast<uint32_t>(kTileRows + bn_cta) * t.kb_elems * 2;
-  const uint32_t fixed = tc_layout(0, bn_cta, t.kb_elems).total + 1024u;
+  const uint32_t stage_bytes = static_cast<uint32_t>(mt * kTileRows + bn_cta) * t.kb_elems * 2;
+  const uint32_t fixed = tc_layout(0, bn_cta, t.kb_elems, mt).total + 1024u;
   int stages = budget > fixed ? static_cast<int>((budget - fixed) / stage_bytes) : 0;
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) stages = 2;
   t.stages = stages;
-  t.smem = tc_layout(stages, bn_cta, t.kb_elems).total + 1024u;
+  t.smem = tc_layout(stages, bn_cta, t.kb_elems, mt).total + 1024u;
   return t;
 }
 
@@ -563,7 +584,19 @@ cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s) {
   if (!enc) return cudaErrorNotSupported;
   const CUtensorMapDataType dt = a.dtype == kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   const int64_t ntiles = (a.n + kTileRows - 1) / kTileRows;
-  const TcShape t = choose_shape(a.cin, a.cout, ntiles);
+  const int epi = a.ep.act != kActNone || a.ep.residual ? 1 : 0;
+  const int variant = g_conv_variant.load();
+  // Two tiles per CTA (the plain k = 3 conv, 64 or 128 output channels):
+  // the default for 64 output channels.  Measured on B200 (conv alone, L2
+  // flushed, one tile per CTA -> two): 512^3 decoder stage, 64 ch, 0.500 ->
+  // 0.447 ms; four-item 256^3 set, 64 ch fp16, 0.683 -> 0.628 ms.  At 128
+  // channels the weight bytes halve too, but the tiles fill fewer waves of
+  // the two CTA slots per SM: 6-shell 128^3, 0.098 -> 0.123 ms; full 128^3
+  // grid, about even (1.92 ms).  Four stages at one CTA per SM were slower
+  // everywhere (6-shell 0.125 ms, decoder stage 0.879 ms).
+  const bool two = (variant == 4 || (variant == 0 && a.cout == 64)) && epi == 0 && a.taps == kTaps &&
+                   a.cout <= 128 && a.cout % 64 == 0;
+  const TcShape t = choose_shape(a.cin, a.cout, ntiles, two ? 2 : 1);
   const CUtensorMapSwizzle sw = t.kb_elems == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
 
   CUtensorMap fmap, wmap;
@@ -597,20 +630,20 @@ cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s) {
   p.tile_mask = a.tile_mask;
   p.bias = static_cast<const uint16_t*>(a.bias);
   p.bias_vec = a.bias && aligned16(a.bias) ? 1 : 0;
-  const int epi = a.ep.act != kActNone || a.ep.residual ? 1 : 0;
   // The staged epilogue needs gather warps x 32 rows x (the warp's row bytes
   // + 16) of the stage buffers (A and B regions, contiguous).  Eight gather
   // warps serve the plain k = 3 conv at three CTAs per SM when it fits.
   auto staged_fits = [&](int gw) {
-    const uint32_t bw = static_cast<uint32_t>(t.bn) / (gw / 4);
+    const uint32_t bw = t.mt == 2 ? static_cast<uint32_t>(t.bn) : static_cast<uint32_t>(t.bn) / (gw / 4);
     const uint32_t need = static_cast<uint32_t>(gw) * 32u * (bw * 2u + 16u);
     const uint32_t have =
-        static_cast<uint32_t>(t.stages) * (static_cast<uint32_t>(kTileRows + t.bn) * t.kb_elems * 2u);
+        static_cast<uint32_t>(t.stages) * (static_cast<uint32_t>(t.mt * kTileRows + t.bn) * t.kb_elems * 2u);
     return need <= have;
   };
   const bool gw8 = !t.pair && epi == 0 && a.taps == kTaps && t.ctas_per_sm == 3 && t.bn % 64 == 0 &&
                    staged_fits(8) && g_gather_warps.load() != 4;
-  p.stage_out = !t.pair && staged_fits(gw8 ? 8 : 4) ? 1 : 0;
+  if (two && !staged_fits(8)) return cudaErrorInvalidConfiguration;  // does not happen for BN <= 128
+  p.stage_out = !t.pair && staged_fits(gw8 || two ? 8 : 4) ? 1 : 0;
   p.out = static_cast<uint16_t*>(a.out);
   p.err = a.err;
   p.n = a.n;
@@ -646,11 +679,13 @@ cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s) {
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kern, fmap, wmap, p);
   } else {
-    auto kern = gw8 ? k_conv_tc<false, 0, 8> : (epi == 1 ? k_conv_tc<false, 1, 4> : k_conv_tc<false, 0, 4>);
+    auto kern = two   ? k_conv_tc<false, 0, 8, 2>
+                : gw8 ? k_conv_tc<false, 0, 8>
+                      : (epi == 1 ? k_conv_tc<false, 1, 4> : k_conv_tc<false, 0, 4>);
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(t.smem));
     if (e != cudaSuccess) return e;
-    const int64_t units = ntiles * t.nsplit;
-    const int threads = gw8 ? 64 + 32 * 8 : kTcThreads;
+    const int64_t units = (two ? (ntiles + 1) / 2 : ntiles) * t.nsplit;
+    const int threads = gw8 || two ? 64 + 32 * 8 : kTcThreads;
     kern<<<static_cast<unsigned>(units), threads, t.smem, s>>>(fmap, wmap, p);
     e = cudaGetLastError();
   }

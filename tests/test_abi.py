@@ -35,7 +35,8 @@ def test_strerror_without_gpu():
     assert lib.smc_strerror(-3) == b"duplicate coordinate"
     assert lib.smc_set_hash_capacity(-1) == -1
     assert lib.smc_set_hash_capacity(0) == 0
-    assert lib.smc_set_conv_variant(4) == -1
+    assert lib.smc_set_conv_variant(5) == -1
+    assert lib.smc_set_conv_variant(4) == 0
     assert lib.smc_set_conv_variant(-1) == -1
     assert lib.smc_set_conv_variant(0) == 0
     assert lib.smc_set_conv_epilogue(2) == -1

@@ -63,11 +63,12 @@ def check_close(got, ref, dtype, what=""):
     assert err <= TOL[dtype] * scale, f"{what}: max err {err:.3e} vs bound {TOL[dtype] * scale:.3e}"
 
 
-@pytest.fixture(params=[1, 2, 3], ids=["one_cta", "cta_pair", "per_offset"])
+@pytest.fixture(params=[1, 2, 3, 4], ids=["one_cta", "cta_pair", "per_offset", "two_tiles"])
 def conv_variant(request):
     """Runs a test on each tensor-core conv: the fused 27-tap kernel with one
-    CTA per 128-row tile, the same with CTA pairs sharing M = 256 MMAs, and the
-    per-offset gather-GEMM-scatter over the pair lists."""
+    CTA per 128-row tile, the same with CTA pairs sharing M = 256 MMAs, the
+    per-offset gather-GEMM-scatter over the pair lists, and the fused kernel
+    with two tiles per CTA sharing each weight stage."""
     smc.set_conv_variant(request.param)
     yield request.param
     smc.set_conv_variant(0)
@@ -466,19 +467,21 @@ def test_conv_ragged_tail_and_no_bias(oracle_mod, rows, conv_variant):
 
 @pytest.mark.parametrize("name,dtype", [("shells6", "bf16"), ("decoder3", "bf16"), ("varlen4", "f16")])
 def test_conv_variants_agree(name, dtype):
-    """Both tensor-core kernels give the same output bits: a pair issues the
-    union of its two tiles' taps, and a tap a row lacks adds exact zeros."""
+    """The fused tensor-core kernels give the same output bits: one CTA per
+    tile, CTA pairs and two tiles per CTA issue the union of their tiles'
+    taps, and a tap a row lacks adds exact zeros."""
     w = workload(name)
     m = build(w)
     f, wt, b = _layer(w, dtype)
     outs = []
-    for v in (1, 2):
+    for v in (1, 2, 4, 0):
         smc.set_conv_variant(v)
         try:
             outs.append(smc.conv(m, dev(f, dtype), dev(wt, dtype), dev(b, dtype)).cpu())
         finally:
             smc.set_conv_variant(0)
-    assert torch.equal(outs[0], outs[1])
+    for o in outs[1:]:
+        assert torch.equal(outs[0], o)
     smc.status()
 
 
