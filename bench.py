@@ -230,6 +230,9 @@ def pair_flops(p: int, cin: int, cout: int) -> float:
 
 
 # ------------------------------------------------------------- GPU arm
+STEP_VARIANT = 0  # tensor-core conv variant of the timed steps (0: the library's choice)
+
+
 def conv_variant_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, w_d, b_d, out_d, reps=5):
     """Median device time (ms) of one conv with each tensor-core variant on
     the bench's map, L2 flushed before each: the fused 27-tap kernel (the
@@ -238,7 +241,7 @@ def conv_variant_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, w
     m = smc.build_map(coords_d, w.grid, batch=batch, stream=stream)
     res = {}
     try:
-        for name, v in (("fused", 1), ("per_offset", 3)):
+        for name, v in (("fused", STEP_VARIANT), ("per_offset", 3)):
             smc.set_conv_variant(v)
             ts = []
             for _ in range(reps + 1):
@@ -251,7 +254,7 @@ def conv_variant_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, w
                 ts.append(e0.elapsed_time(e1))
             res[name] = round(float(np.median(ts[1:])), 4)
     finally:
-        smc.set_conv_variant(0)
+        smc.set_conv_variant(STEP_VARIANT)
         m.free()
     smc.status(stream)
     res["fused_speedup"] = round(res["per_offset"] / res["fused"], 2)
@@ -537,6 +540,10 @@ def run_gpu(args):
     smc.lib()
     if args.schedule_segment is not None:
         smc.set_schedule_segment(args.schedule_segment)
+    if args.conv_variant is not None:
+        global STEP_VARIANT
+        STEP_VARIANT = args.conv_variant
+        smc.set_conv_variant(args.conv_variant)
     peaks = load_peaks()
 
     w = get_workload(args.workload)
@@ -664,6 +671,7 @@ def run_gpu(args):
                 "l2": "flushed before every step (256 MB write, outside the timed events)",
                 "parallelism": f"replicas x{world} (no collective on the data path)",
                 **({"schedule_segment_rows": args.schedule_segment} if args.schedule_segment is not None else {}),
+                **({"conv_variant": args.conv_variant} if args.conv_variant is not None else {}),
             },
             "pair_tflops": round(conv_tflops, 2),
             "map_build_gbs": round(map_gbs, 1),
@@ -882,6 +890,9 @@ def main(argv=None):
                     help="shells6 (default), full128, varlen4, shell2, decoder0..decoder3")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--conv-variant", type=int, default=None,
+                    help="tensor-core conv variant for the step's conv (smc_set_conv_variant; default: the "
+                         "library's choice)")
     ap.add_argument("--schedule-segment", type=int, default=None,
                     help="sort the tile schedule within segments of this many rows (0 = whole map; default: "
                          "the library's default)")
