@@ -389,43 +389,72 @@ def resample_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, peaks
     return out
 
 
-class StepRunner:
-    """Steps enqueued up to DEPTH ahead of the host, as a job would run them:
-    each step is the asynchronous map build and the conv behind it on one
-    stream, bracketed by its own CUDA events (an L2 flush sits between steps,
-    outside them).  A step is retired DEPTH steps later: its map's outcome is
-    checked, its event times are read and the map is freed (stream-ordered)."""
-    DEPTH = 4
+L2_BYTES = 126 << 20  # B200 L2
+PIPE_STREAMS = 2       # streams the timed steps alternate over
 
-    def __init__(self, smc, torch, stream, flush, coords_d, grid, batch, feats_d, w_d, b_d, out_d, profile=False):
-        self.smc, self.torch, self.stream, self.flush = smc, torch, stream, flush
-        self.coords_d, self.grid, self.batch = coords_d, grid, batch
-        self.feats_d, self.w_d, self.b_d, self.out_d = feats_d, w_d, b_d, out_d
+
+def input_sets(torch, dev, w, f, tdt, min_sets=2, max_sets=8):
+    """Copies of one step's inputs (coordinates, features) and output buffer,
+    enough that the copies together hold at least 3x the L2 size, so that a
+    step finds none of its inputs in L2 from earlier steps without a flush."""
+    per = w.n * (16 + 2 * w.cin + 2 * w.cout)
+    k = max(min_sets, min(max_sets, -(-3 * L2_BYTES // per)))
+    coords = torch.from_numpy(w.coords)
+    feats = torch.from_numpy(f).to(tdt)
+    return [(coords.to(dev), feats.to(dev), torch.empty((w.n, w.cout), dtype=tdt, device=dev)) for _ in range(k)]
+
+
+class StepRunner:
+    """Steps enqueued up to DEPTH per stream ahead of the host, as a job would run them:
+    each step is the asynchronous map build and the conv behind it, on one of
+    `streams` in turn and on the next of the input `sets`, bracketed by its
+    own CUDA events on its stream.  With `flush`, an L2 flush precedes every
+    step on its stream (outside its events).  A step is retired DEPTH steps
+    later: its map's outcome is checked, its event times are read and the map
+    is freed (stream-ordered)."""
+    DEPTH = 3
+
+    def __init__(self, smc, torch, streams, flush, sets, grid, batch, w_d, b_d, profile=False, step_events=True):
+        self.smc, self.torch, self.streams, self.flush = smc, torch, list(streams), flush
+        self.step_events = step_events  # events around whole steps (else around the conv only)
+        self.depth = self.DEPTH * len(self.streams)
+        self.sets, self.grid, self.batch, self.w_d, self.b_d = sets, grid, batch, w_d, b_d
         self.profile = profile  # read the library's per-phase timing of each build
         self.pending = []
+        self.count = 0
         self.times, self.conv_times, self.map_times = [], [], []
 
-    def submit(self, flush=True):
-        torch, smc, stream = self.torch, self.smc, self.stream
-        if flush:
-            self.flush.zero_()
-        e0, e1, ec, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
-        e0.record(stream)
-        m = smc.build_map(self.coords_d, self.grid, batch=self.batch, stream=stream, sync=False)
+    def submit(self):
+        torch, smc = self.torch, self.smc
+        stream = self.streams[self.count % len(self.streams)]
+        coords_d, feats_d, out_d = self.sets[self.count % len(self.sets)]
+        self.count += 1
+        if self.flush is not None:
+            with torch.cuda.stream(stream):
+                self.flush.zero_()
+        e0, e2 = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) \
+            if self.step_events else (None, None)
+        e1, ec = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if e0 is not None:
+            e0.record(stream)
+        m = smc.build_map(coords_d, self.grid, batch=self.batch, stream=stream, sync=False)
         e1.record(stream)
-        smc.conv(m, self.feats_d, self.w_d, self.b_d, ksize=3, orientation=1, out=self.out_d, stream=stream)
+        smc.conv(m, feats_d, self.w_d, self.b_d, ksize=3, orientation=1, out=out_d, stream=stream)
         ec.record(stream)
         m.stream_wait(stream)  # the step ends when the whole build (pair lists too) is done
-        e2.record(stream)
+        if e2 is not None:
+            e2.record(stream)
         self.pending.append((e0, e1, ec, e2, m))
-        if len(self.pending) > self.DEPTH:
+        if len(self.pending) > self.depth:
             self.retire()
 
     def retire(self):
         e0, e1, ec, e2, m = self.pending.pop(0)
-        e2.synchronize()
-        m.wait()  # raises if the build failed on the device
-        self.times.append(e0.elapsed_time(e2))
+        m.wait()  # the whole build is done (raises if it failed on the device)
+        ec.synchronize()
+        if e2 is not None:
+            e2.synchronize()
+            self.times.append(e0.elapsed_time(e2))
         self.conv_times.append(e1.elapsed_time(ec))
         if self.profile:
             self.map_times.append(m.timing())
@@ -434,6 +463,39 @@ class StepRunner:
     def drain(self):
         while self.pending:
             self.retire()
+
+
+def prime_pool(smc, sets, grid, batch, streams, count):
+    """Builds `count` maps at once over the streams and frees them, so that
+    the library's memory pool already holds what the pipelined steps keep in
+    flight (set-up, not a step: no conv runs)."""
+    maps = [smc.build_map(sets[i % len(sets)][0], grid, batch=batch, stream=streams[i % len(streams)], sync=False)
+            for i in range(count)]
+    for m in maps:
+        m.wait()
+    for m in maps:
+        m.free()
+
+
+def timed_steps(torch, runner, steps):
+    """Device time (ms) of `steps` steps of `runner` from the first one's
+    start to the end of the last one, on every stream: an event on the first
+    stream that the others wait for, and a join of all streams at the end."""
+    s0 = runner.streams[0]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(s0)
+    for s in runner.streams[1:]:
+        s.wait_event(start)
+    for _ in range(steps):
+        runner.submit()
+    for s in runner.streams[1:]:
+        ev = torch.cuda.Event()
+        ev.record(s)
+        s0.wait_event(ev)
+    end.record(s0)
+    runner.drain()
+    end.synchronize()
+    return start.elapsed_time(end)
 
 
 def conv_alone_times(smc, torch, stream, flush, m, feats_d, w_d, b_d, out_d, reps=10):
@@ -459,47 +521,62 @@ def conv_alone_times(smc, torch, stream, flush, m, feats_d, w_d, b_d, out_d, rep
 
 
 def measure_config(smc, torch, stream, flush, dev, peaks, name, dtype, steps, world, wl=None):
-    """One workload measured the way the headline is: timed steps (build +
-    conv, L2 flushed between steps), the conv alone flushed and L2-warm, and
-    the map phases from the library's own events; with the SM clocks sampled
-    while it runs.  Returns a sub-record for the bench line."""
+    """One workload measured the way the headline is: pipelined steps (build +
+    conv, alternating over two streams, inputs rotated over copies larger
+    than L2) for throughput; the same steps one at a time with L2 flushed
+    before each for latency; the conv alone flushed and L2-warm; and the map
+    phases from the library's own events; with the SM clocks sampled while
+    the pipelined steps run.  Returns a sub-record for the bench line."""
     w = wl if wl is not None else get_workload(name)
     tdt = {"bf16": torch.bfloat16, "f16": torch.float16}[dtype]
     f, wt, b = S.layer_tensors(w, dtype)
-    coords_d = torch.from_numpy(w.coords).to(dev)
-    feats_d = torch.from_numpy(f).to(tdt).to(dev)
+    sets = input_sets(torch, dev, w, f, tdt)
     w_d = torch.from_numpy(wt).to(tdt).to(dev)
     b_d = torch.from_numpy(b).to(tdt).to(dev)
-    out_d = torch.empty((w.n, w.cout), dtype=tdt, device=dev)
     batch = int(w.coords[:, 0].max()) + 1
     del f
-    args = (smc, torch, stream, flush, coords_d, w.grid, batch, feats_d, w_d, b_d, out_d)
-    warm = StepRunner(*args)
+    streams = [stream] + [torch.cuda.Stream(dev) for _ in range(PIPE_STREAMS - 1)]
+    mk = lambda st, fl, profile=False: StepRunner(smc, torch, st, fl, sets, w.grid, batch, w_d, b_d, profile=profile,
+                                                  step_events=len(st) == 1)
+    # latency: one step at a time on one stream, L2 flushed before each
+    lat = mk([stream], flush)
     for _ in range(3):
+        lat.submit()
+    lat.drain()
+    lat.times.clear()
+    lat.conv_times.clear()
+    for _ in range(steps):
+        lat.submit()
+    lat.drain()
+    latency = float(np.median(lat.times))
+    # throughput: pipelined steps, at least 0.3 s of them
+    prime_pool(smc, sets, w.grid, batch, streams, StepRunner.DEPTH * len(streams) + 2)
+    warm = mk(streams, None)
+    for _ in range(2 * StepRunner.DEPTH):
         warm.submit()
     warm.drain()
+    n_steps = max(steps, int(0.3 / (latency * 1e-3)))
     clocks = ClockSampler(dev.index or 0)
     clocks.start()
     clocks.mark()
-    run = StepRunner(*args)
-    t0 = time.perf_counter()
-    while len(run.times) + len(run.pending) < steps or time.perf_counter() - t0 < 0.3:
-        run.submit()
-    run.drain()
+    run = mk(streams, None)
+    total = timed_steps(torch, run, n_steps)
     clocks.mark_end()
     clk = clocks.stop()
-    prof = StepRunner(*args, profile=True)
+    prof = mk([stream], flush, profile=True)
     smc.set_profiling(True)
     for _ in range(min(steps, 20)):
         prof.submit()
     prof.drain()
     smc.set_profiling(False)
+    coords_d, feats_d, out_d = sets[0]
     m = smc.build_map(coords_d, w.grid, batch=batch, stream=stream)
     P = m.pairs_total
     conv_cold, conv_warm = conv_alone_times(smc, torch, stream, flush, m, feats_d, w_d, b_d, out_d)
     m.free()
-    step_ms = reduce_max(float(np.median(run.times)), world, dev)
-    conv_ms = reduce_max(float(np.median(run.conv_times)), world, dev)
+    step_ms = reduce_max(total / n_steps, world, dev)
+    latency_ms = reduce_max(latency, world, dev)
+    conv_ms = reduce_max(float(np.mean(run.conv_times)), world, dev)
     look = reduce_max(float(np.median([t[0] for t in prof.map_times])), world, dev)
     sched = reduce_max(float(np.median([t[1] for t in prof.map_times])), world, dev)
     pairs_ms = reduce_max(float(np.median([t[2] for t in prof.map_times])), world, dev)
@@ -507,15 +584,19 @@ def measure_config(smc, torch, stream, flush, dev, peaks, name, dtype, steps, wo
     map_bytes = algorithmic_map_bytes(w.n, P)
     tfl = flops / (conv_ms * 1e-3) / 1e12
     gbs = map_bytes / ((look + pairs_ms) * 1e-3) / 1e9
+    pk = peaks["bf16_tflops"]
     rec = {
         "workload": f"{w.name}: {w.note}", "dtype": dtype, "n_voxels": w.n, "pairs": P,
-        "steps_timed": len(run.times), "step_ms": round(step_ms, 4),
+        "steps_timed": n_steps, "step_ms": round(step_ms, 4),
         "mvoxels_per_s": round(world * w.n / (step_ms * 1e-3) / 1e6, 2),
+        "step_latency_ms": round(latency_ms, 4),
+        "input_sets": len(sets),
         "conv_ms": round(conv_ms, 4), "conv_ms_alone_l2_flushed": round(conv_cold, 4),
         "conv_ms_alone_l2_warm": round(conv_warm, 4),
-        "conv_roofline": {"bound": "tensor", "achieved": round(tfl, 2), "peak": peaks["bf16_tflops"],
-                          "unit": "TFLOP/s", "frac": round(tfl / peaks["bf16_tflops"], 4),
-                          "frac_l2_warm": round(flops / (conv_warm * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)},
+        "conv_roofline": {"bound": "tensor", "achieved": round(tfl, 2), "peak": pk,
+                          "unit": "TFLOP/s", "frac": round(tfl / pk, 4),
+                          "frac_alone_l2_flushed": round(flops / (conv_cold * 1e-3) / 1e12 / pk, 4),
+                          "frac_l2_warm": round(flops / (conv_warm * 1e-3) / 1e12 / pk, 4)},
         "map_ms": {"clears_and_lookups": round(look, 4), "tile_schedule": round(sched, 4),
                    "pair_lists_side_stream": round(pairs_ms, 4)},
         "map_roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -523,7 +604,7 @@ def measure_config(smc, torch, stream, flush, dev, peaks, name, dtype, steps, wo
     }
     if clk is not None:
         rec["clocks"] = clk
-    del feats_d, out_d, coords_d
+    del sets, feats_d, out_d, coords_d
     torch.cuda.empty_cache()
     return rec
 
@@ -550,21 +631,22 @@ def run_gpu(args):
     dtype = "f16" if "f16" in w.dtypes and "bf16" not in w.dtypes else "bf16"
     tdt = torch.float16 if dtype == "f16" else torch.bfloat16
     f, wt, b = S.layer_tensors(w, dtype)
-    coords_d = torch.from_numpy(w.coords).to(dev)
-    feats_d = torch.from_numpy(f).to(tdt).to(dev)
+    sets = input_sets(torch, dev, w, f, tdt)
+    coords_d, feats_d, out_d = sets[0]
     w_d = torch.from_numpy(wt).to(tdt).to(dev)
     b_d = torch.from_numpy(b).to(tdt).to(dev)
-    out_d = torch.empty((w.n, w.cout), dtype=tdt, device=dev)
     batch = int(w.coords[:, 0].max()) + 1
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    runner = lambda profile=False: StepRunner(smc, torch, stream, flush, coords_d, w.grid, batch, feats_d, w_d,
-                                              b_d, out_d, profile=profile)
+    streams = [stream] + [torch.cuda.Stream(dev) for _ in range(PIPE_STREAMS - 1)]
+    runner = lambda st, fl, profile=False: StepRunner(smc, torch, st, fl, sets, w.grid, batch, w_d, b_d,
+                                                      profile=profile, step_events=len(st) == 1)
 
     smc.set_profiling(False)  # the timed steps carry no instrumentation
 
-    # warm-up
-    warm = runner()
+    prime_pool(smc, sets, w.grid, batch, streams, StepRunner.DEPTH * len(streams) + 2)
+    # warm-up: W pipelined steps
+    warm = runner(streams, None)
     for _ in range(args.warmup):
         warm.submit()
     warm.drain()
@@ -575,6 +657,8 @@ def run_gpu(args):
     eff = tap_efficiency(m0.schedule().cpu().numpy(), m0.nbr().cpu().numpy())
     m0.free()
 
+    # the timed region: K steps, alternating over the streams, each on the
+    # next copy of the inputs (together more than 3x L2, so no flush)
     clocks = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize()
@@ -582,10 +666,8 @@ def run_gpu(args):
     clocks.mark()
     t_wall0 = time.perf_counter()
     launches_before = smc.kernel_launches()
-    run = runner()
-    for _ in range(args.steps):
-        run.submit()
-    run.drain()
+    run = runner(streams, None)
+    total_ms = timed_steps(torch, run, args.steps)
     torch.cuda.synchronize()
     times, conv_times = run.times, run.conv_times
     launches = smc.kernel_launches() - launches_before
@@ -597,19 +679,25 @@ def run_gpu(args):
     window_note = None
     if clocks.region_samples() < 5:
         tw = time.perf_counter()
-        extra = runner()
+        extra = runner(streams, None)
         while time.perf_counter() - tw < 0.4:
             extra.submit()
         extra.drain()
         window_note = (f"the same steps repeated untimed for {1e3 * (time.perf_counter() - tw):.0f} ms right "
-                       f"after the timed region ({len(extra.times)} steps)")
+                       f"after the timed region ({len(extra.conv_times)} steps)")
     clk = clocks.stop(window_note)
     barrier(world)
     smc.status(stream)
+    # latency: the same steps one at a time on one stream, L2 flushed before each
+    lat = runner([stream], flush)
+    for _ in range(min(args.steps, 200)):
+        lat.submit()
+    lat.drain()
+    lat_times = lat.times
     # per-phase breakdown of the build from a separate, untimed pass with the
-    # library's own CUDA events on
+    # library's own CUDA events on (one stream, L2 flushed before each step)
     smc.set_profiling(True)
-    prof = runner(profile=True)
+    prof = runner([stream], flush, profile=True)
     for _ in range(min(args.steps, 50)):
         prof.submit()
     prof.drain()
@@ -623,7 +711,7 @@ def run_gpu(args):
     epilogue = epilogue_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, w_d, b_d, out_d)
     resample = resample_times(smc, torch, stream, flush, coords_d, w, batch, feats_d, peaks)
 
-    total_ms = reduce_max(sum(times), world, dev)
+    total_ms = reduce_max(total_ms, world, dev)
     conv_ms = reduce_max(sum(conv_times) / len(conv_times), world, dev)
     look_ms = reduce_max(sum(t[0] for t in map_times) / len(map_times), world, dev)
     sched_ms = reduce_max(sum(t[1] for t in map_times) / len(map_times), world, dev)
@@ -667,8 +755,14 @@ def run_gpu(args):
             "data": "synthetic (seeded union of 6 sphere shells; random-init KRSC weights)",
             "config": {
                 "workload": f"{w.name}: {w.note}", "n_voxels": w.n, "pairs": P, "grid": list(w.grid),
-                "cin": w.cin, "cout": w.cout, "step": "build_map (asynchronous entry point) + conv k=3 s=+1 on one stream, up to 4 steps enqueued ahead; every map checked and freed when its step retires",
-                "l2": "flushed before every step (256 MB write, outside the timed events)",
+                "cin": w.cin, "cout": w.cout,
+                "step": ("build_map (asynchronous entry point) + conv k=3 s=+1; steps alternate over "
+                         f"{PIPE_STREAMS} streams, up to {StepRunner.DEPTH} per stream enqueued ahead, so one step's map build "
+                         "overlaps the previous step's conv; every map checked and freed when its step retires; "
+                         "value and ms_per_step from the device time of all K steps (first start to last end)"),
+                "l2": (f"no flush: steps rotate over {len(sets)} copies of their inputs and outputs "
+                       f"({len(sets) * w.n * (16 + 2 * w.cin + 2 * w.cout) / 1e6:.0f} MB, > 3x the 126 MB L2); "
+                       "step_latency_ms: one step at a time on one stream, L2 flushed (256 MB write) before each"),
                 "parallelism": f"replicas x{world} (no collective on the data path)",
                 **({"schedule_segment_rows": args.schedule_segment} if args.schedule_segment is not None else {}),
                 **({"conv_variant": args.conv_variant} if args.conv_variant is not None else {}),
@@ -678,8 +772,8 @@ def run_gpu(args):
             "breakdown_ms": {"step": round(ms_per_step, 4), "map_clears_and_lookups": round(look_ms, 4),
                              "tile_schedule": round(sched_ms, 4),
                              "pair_lists_side_stream": round(pairs_ms, 4), "conv": round(conv_ms, 4)},
-            "step_ms_quantiles": {q: round(float(np.quantile(times, v)), 4)
-                                  for q, v in (("p50", 0.5), ("p90", 0.9), ("p99", 0.99), ("max", 1.0))},
+            "step_latency_ms": {q: round(float(np.quantile(lat_times, v)), 4)
+                                for q, v in (("p50", 0.5), ("p90", 0.9), ("p99", 0.99), ("max", 1.0))},
             "conv_alone_ms": {"l2_flushed": round(conv_cold, 4), "l2_warm": round(conv_warm, 4)},
             "conv_mvoxels_per_s": round(w.n / (conv_ms * 1e-3) / 1e6, 2),
             "conv_tap_efficiency": round(eff, 4),
@@ -690,9 +784,12 @@ def run_gpu(args):
             "roofline": {"kernel": "k_conv_tc", "bound": "tensor", "achieved": round(conv_tflops, 2),
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": round(conv_tflops / peaks["bf16_tflops"], 4), "traffic": traffic,
+                         "frac_alone_l2_flushed": round(flops / (conv_cold * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
                          "frac_l2_warm": round(flops / (conv_warm * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
                          "peak_source": f"{peaks['source']} bf16 burst (kernel timed alone)",
-                         "algorithmic": "2 * pairs * Cin * Cout per launch"},
+                         "algorithmic": "2 * pairs * Cin * Cout per launch",
+                         "duration": "mean launch time over the timed region (events on its stream, next to the "
+                                     "other stream's map build)"},
             "map_roofline": {"kernels": "clears, k_insert, k_neighbours, pair-list scan, k_pairs (time = clears and lookups + pair lists)",
                              "bound": "hbm", "achieved": round(map_gbs, 1),
                              "peak": peaks["hbm_gbs"], "unit": "GB/s",

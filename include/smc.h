@@ -91,7 +91,8 @@ enum {
  * Builds, on the device: 64-bit site keys, a lookup structure of the sites
  * (a dense int32 index grid over the batch x Z x Y x X box when the box has
  * at most 2^28 sites and at most 256 sites per voxel, with an occupancy
- * bitmap instead of a clear above 2^23 sites, else an open-addressing hash
+ * bitmap instead of a clear above 2^23 sites or 16 sites per voxel, else an
+ * open-addressing hash
  * table; smc_set_map_lookup forces any of them), the int32
  * [n, 27] neighbour map (-1 = absent), the per-offset pair lists (stable
  * compaction of each map column, ascending output row), and the tile
@@ -390,8 +391,9 @@ SMC_API const char* smc_strerror(int code);
  * smc_set_map_lookup: lookup structure of later builds: 0 = by size
  *   (default: a dense int32 index grid over the batch x Z x Y x X box when it
  *   has at most 2^28 sites and at most 256 sites per voxel -- cleared at
- *   every build up to 2^23 sites, above that left uncleared behind a cleared
- *   occupancy bitmap of one bit per site -- else a hash table), 1 = hash
+ *   every build when it has at most 2^23 sites and fewer than 16 per voxel,
+ *   else left uncleared behind a cleared occupancy bitmap of one bit per
+ *   site -- else a hash table), 1 = hash
  *   table, 2 = cleared dense grid and 3 = dense grid with occupancy bitmap,
  *   each whenever the box has at most 2^28 sites.  Maps are identical either way.  A forced hash capacity
  *   (smc_set_hash_capacity) always selects the hash table.  SMC_E_ARG for
