@@ -400,8 +400,9 @@ SMC_API const char* smc_strerror(int code);
  *   any other value.
  * smc_set_conv_variant: tensor-core conv kernel for later convs (bf16/fp16
  *   shapes the tensor cores take; others always use the FMA kernel): 0 =
- *   default (4 for a k = 3 conv with 64 output channels and no fused
- *   activation or residual, else 1), 1 = fused 27-tap gather-GEMM, one CTA
+ *   default (4 for a k = 3 conv with no fused activation or residual and 64
+ *   output channels, or 128 on a map of at least 2 x 2 x 8 x SMs tiles of
+ *   128 rows; else 1), 1 = fused 27-tap gather-GEMM, one CTA
  *   per 128-row tile, 2 = the same with CTA pairs (a cluster of two CTAs
  *   sharing M = 256 tcgen05 MMAs, each loading half of the weight block;
  *   slower on B200, where such clusters run one per TPC), 3 = per-offset

@@ -505,6 +505,23 @@ EncodeTiledFn encode_fn() {
 
 static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
+// SMs of the current device (queried once per device).
+static int sm_count() {
+  static std::atomic<int> cache[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  int v = cache[dev].load();
+  if (v == 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+      cudaGetLastError();
+      v = 148;
+    }
+    cache[dev].store(v);
+  }
+  return v;
+}
+
 bool conv_tc_supported(const ConvArgs& a) {
   return (a.dtype == kBF16 || a.dtype == kF16) && a.cin >= 64 && a.cin % 16 == 0 && a.cout >= 16 &&
          a.cout % 16 == 0 && aligned16(a.feats) && aligned16(a.weight) && aligned16(a.out) &&
@@ -587,15 +604,19 @@ cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s) {
   const int epi = a.ep.act != kActNone || a.ep.residual ? 1 : 0;
   const int variant = g_conv_variant.load();
   // Two tiles per CTA (the plain k = 3 conv, 64 or 128 output channels):
-  // the default for 64 output channels.  Measured on B200 (conv alone, L2
-  // flushed, one tile per CTA -> two): 512^3 decoder stage, 64 ch, 0.500 ->
-  // 0.447 ms; four-item 256^3 set, 64 ch fp16, 0.683 -> 0.628 ms.  At 128
-  // channels the weight bytes halve too, but the tiles fill fewer waves of
-  // the two CTA slots per SM: 6-shell 128^3, 0.098 -> 0.123 ms; full 128^3
-  // grid, about even (1.92 ms).  Four stages at one CTA per SM were slower
-  // everywhere (6-shell 0.125 ms, decoder stage 0.879 ms).
-  const bool two = (variant == 4 || (variant == 0 && a.cout == 64)) && epi == 0 && a.taps == kTaps &&
-                   a.cout <= 128 && a.cout % 64 == 0;
+  // the default for 64 output channels, and for 128 when the map has at
+  // least eight waves of two-tile units at two CTAs per SM.  Measured on
+  // B200 (conv alone, L2 flushed, one tile per CTA -> two): 512^3 decoder
+  // stage, 64 ch, 0.500 -> 0.447 ms; four-item 256^3 set, 64 ch fp16, 0.683
+  // -> 0.628 ms.  At 128 channels the weight bytes halve too, but a small
+  // map's tiles fill fewer waves of the two CTA slots per SM: 6-shell 128^3,
+  // 0.098 -> 0.123 ms; on the full 128^3 grid (16384 tiles) even at full
+  // clock (1.92 ms) and 10% faster inside pipelined steps under the power
+  // cap (2.16 -> 1.94 ms at 1.6 GHz).  Four stages at one CTA per SM were
+  // slower everywhere (6-shell 0.125 ms, decoder stage 0.879 ms).
+  const bool big = ntiles >= 8ll * 2 * 2 * sm_count();
+  const bool two = (variant == 4 || (variant == 0 && (a.cout == 64 || (a.cout == 128 && big)))) && epi == 0 &&
+                   a.taps == kTaps && a.cout <= 128 && a.cout % 64 == 0;
   const TcShape t = choose_shape(a.cin, a.cout, ntiles, two ? 2 : 1);
   const CUtensorMapSwizzle sw = t.kb_elems == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
 
