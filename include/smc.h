@@ -469,10 +469,11 @@ SMC_API int smc_set_map_lookup(int32_t mode);
  *   the entry point that asked returns SMC_E_OOM, leaves its handle output
  *   NULL and releases whatever it had allocated.  0 disarms the hook.
  *   SMC_E_ARG for k < 0.
- * smc_set_wait_limit_ns: bound, in nanoseconds, of the single-pass scans'
- *   device-side waits on earlier segments (every build, subdivision,
- *   upsample and downsample runs such scans); 0 restores the default 2 s.
- *   SMC_E_ARG for ns < 0.
+ * smc_set_wait_limit_ns: bound, in nanoseconds, of every device-side wait:
+ *   the single-pass scans' waits on earlier segments (every build,
+ *   subdivision, upsample and downsample runs such scans) and the convs'
+ *   pipeline waits (never below 100 ms for those, so that no CTA gives up
+ *   with loads in flight); 0 restores the default 2 s.  SMC_E_ARG for ns < 0.
  * smc_set_scan_hold: in every later scan, the segment with this ticket
  *   (0-based, in start order) publishes nothing, so the waits of the
  *   segments after it run out and the call reports SMC_E_TIMEOUT; every

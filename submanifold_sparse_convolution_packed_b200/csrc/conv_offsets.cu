@@ -39,6 +39,7 @@ struct OffParams {
   uint32_t* err;
   int cin, cout, bn, nsplit, stages, kb_elems, orientation, is_bf16;
   uint32_t tmem_cols;
+  uint64_t wait_ns;  // bound of every mbarrier wait
 };
 
 __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
@@ -115,7 +116,7 @@ __global__ void __launch_bounds__(kOffThreads, 3) k_conv_offsets(const __grid_co
     if (lane == 0) {
       for (int kb = 0; kb < kblocks; ++kb) {
         const uint32_t stage = kb % p.stages, phase = (kb / p.stages) & 1u;
-        if (!mbar_wait_bounded(bar_empty + 8 * stage, phase ^ 1u, p.err) || s_misc[1]) {
+        if (!mbar_wait_bounded(bar_empty + 8 * stage, phase ^ 1u, p.err, p.wait_ns) || s_misc[1]) {
           s_misc[1] = 1;
           break;
         }
@@ -130,7 +131,7 @@ __global__ void __launch_bounds__(kOffThreads, 3) k_conv_offsets(const __grid_co
       const uint32_t idesc = idesc_f16(static_cast<uint32_t>(p.is_bf16), static_cast<uint32_t>(p.bn));
       for (int kb = 0; kb < kblocks; ++kb) {
         const uint32_t stage = kb % p.stages, phase = (kb / p.stages) & 1u;
-        if (!mbar_wait_bounded(bar_full + 8 * stage, phase, p.err) || s_misc[1]) {
+        if (!mbar_wait_bounded(bar_full + 8 * stage, phase, p.err, p.wait_ns) || s_misc[1]) {
           s_misc[1] = 1;
           break;
         }
@@ -158,7 +159,8 @@ __global__ void __launch_bounds__(kOffThreads, 3) k_conv_offsets(const __grid_co
     for (int kb = 0; kb < kblocks; ++kb) {
       const uint32_t stage = kb % p.stages, phase = (kb / p.stages) & 1u;
       int w_ok = 1;
-      if (lane == 0) w_ok = mbar_wait_bounded(bar_empty + 8 * stage, phase ^ 1u, p.err) && !s_misc[1];
+      if (lane == 0)
+        w_ok = mbar_wait_bounded(bar_empty + 8 * stage, phase ^ 1u, p.err, p.wait_ns) && !s_misc[1];
       w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
       if (!w_ok) {
         if (lane == 0) s_misc[1] = 1;
@@ -172,7 +174,7 @@ __global__ void __launch_bounds__(kOffThreads, 3) k_conv_offsets(const __grid_co
                     kb * p.kb_elems, r0, r1, r2, r3);
     }
     // ---------------------------------------------------------- scatter-add
-    const bool ready = mbar_wait_bounded(bar_acc, 0, p.err) && !s_misc[1];
+    const bool ready = mbar_wait_bounded(bar_acc, 0, p.err, p.wait_ns) && !s_misc[1];
     tc_fence_after();
     if (ready) {
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
@@ -275,6 +277,9 @@ cudaError_t launch_conv_offsets(const ConvArgs& a, float* acc, cudaStream_t s) {
   p.offsets = a.pair_offsets;
   p.acc = acc;
   p.err = a.err;
+  // A conv's waits are bounded too, but never below 100 ms: a CTA that
+  // gave up a wait early would leave with its TMA loads still in flight.
+  p.wait_ns = scan_wait_limit_ns() > 100000000ull ? scan_wait_limit_ns() : 100000000ull;
   p.cin = a.cin;
   p.cout = a.cout;
   p.orientation = a.orientation;

@@ -71,6 +71,7 @@ struct TcParams {
   int bias_vec;  // bias present and 16-byte aligned: read 8 values per load
   int stage_out;  // plain epilogue staged through the (then free) stage buffers
   uint32_t tmem_cols;
+  uint64_t wait_ns;  // bound of every mbarrier wait
   Epilogue ep;  // activation and residual
 };
 
@@ -218,7 +219,8 @@ __global__ void __launch_bounds__(64 + 32 * kGW, kMT == 2 ? 2 : (kGW == 8 ? 3 : 
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const uint32_t stage = it % p.stages, phase = (it / p.stages) & 1u;
           int w_ok = 1;
-          if (lane == 0) w_ok = mbar_wait_bounded(bar_empty + 8 * stage, phase ^ 1u, p.err) && !s_misc[1];
+          if (lane == 0)
+            w_ok = mbar_wait_bounded(bar_empty + 8 * stage, phase ^ 1u, p.err, p.wait_ns) && !s_misc[1];
           if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
             if (lane == 0) s_misc[1] = 1;
             ok = false;
@@ -257,7 +259,7 @@ __global__ void __launch_bounds__(64 + 32 * kGW, kMT == 2 ? 2 : (kGW == 8 ? 3 : 
       for (uint32_t m = mask; m && ok; m &= m - 1) {
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const uint32_t stage = it % p.stages, phase = (it / p.stages) & 1u;
-          const bool w_ok = mbar_wait_bounded(bar_full + 8 * stage, phase, p.err);
+          const bool w_ok = mbar_wait_bounded(bar_full + 8 * stage, phase, p.err, p.wait_ns);
           if (!__all_sync(0xffffffffu, w_ok && !s_misc[1])) {
             if (lane == 0) s_misc[1] = 1;
             ok = false;
@@ -313,7 +315,8 @@ __global__ void __launch_bounds__(64 + 32 * kGW, kMT == 2 ? 2 : (kGW == 8 ? 3 : 
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const uint32_t stage = it % p.stages, phase = (it / p.stages) & 1u;
           int w_ok = 1;
-          if (lane == 0) w_ok = mbar_wait_bounded(bar_empty + 8 * stage, phase ^ 1u, p.err) && !s_misc[1];
+          if (lane == 0)
+            w_ok = mbar_wait_bounded(bar_empty + 8 * stage, phase ^ 1u, p.err, p.wait_ns) && !s_misc[1];
           w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
           if (!w_ok) {
             if (lane == 0) s_misc[1] = 1;
@@ -356,7 +359,7 @@ __global__ void __launch_bounds__(64 + 32 * kGW, kMT == 2 ? 2 : (kGW == 8 ? 3 : 
     };
     uint4 rcur[4], rnext[4];
     if constexpr (extra) load_res(0, rcur);
-    const bool ready = mbar_wait_bounded(bar_acc, 0, p.err) && !s_misc[1];
+    const bool ready = mbar_wait_bounded(bar_acc, 0, p.err, p.wait_ns) && !s_misc[1];
     tc_fence_after();
     if (!extra && ready && p.stage_out) {
       // Plain epilogue through shared memory: the accumulator is complete, so
@@ -667,6 +670,9 @@ cudaError_t launch_conv_tc(const ConvArgs& a, cudaStream_t s) {
   p.stage_out = !t.pair && staged_fits(gw8 || two ? 8 : 4) ? 1 : 0;
   p.out = static_cast<uint16_t*>(a.out);
   p.err = a.err;
+  // A conv's waits are bounded too, but never below 100 ms: a CTA that
+  // gave up a wait early would leave with its TMA loads still in flight.
+  p.wait_ns = scan_wait_limit_ns() > 100000000ull ? scan_wait_limit_ns() : 100000000ull;
   p.n = a.n;
   p.ntiles = ntiles;
   p.cin = a.cin;

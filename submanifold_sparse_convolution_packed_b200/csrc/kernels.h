@@ -74,8 +74,9 @@ int64_t schedule_segment_rows();
 int radix_seg_chunks(int64_t n);
 int64_t radix_hist_len(int64_t n, int cps);
 int64_t scan_status_len(int64_t L);
-// Bound of the look-back scans' waits on their predecessors (2 s unless a
-// test sets it) and the test hook that holds one scan segment back (-1 = none).
+// Bound of every device-side wait -- the look-back scans' waits on their
+// predecessors and the convs' mbarrier waits -- (2 s unless a test sets it),
+// and the test hook that holds one scan segment back (-1 = none).
 uint64_t scan_wait_limit_ns();
 int64_t scan_hold_ticket();
 
