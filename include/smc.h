@@ -451,6 +451,17 @@ SMC_API int smc_set_profiling(int32_t on);
 SMC_API int smc_map_timing(const smc_map* map, float ms[3]);
 SMC_API int smc_kernel_launches(int64_t* count);
 SMC_API int smc_set_conv_variant(int32_t variant);
+
+/*
+ * Stream of the convs (this library's own): 1 (default) runs each conv's
+ * kernels on one of two library-owned streams of the greatest priority,
+ * forked from the caller's stream by an event and joined back to it by
+ * another, so the caller's stream orders the conv exactly as if it ran there;
+ * the conv's CTAs are then dispatched before those of other work queued beside
+ * it (e.g. a map build on another stream).  0 runs them on the caller's
+ * stream.  SMC_E_ARG for any other value.
+ */
+SMC_API int smc_set_conv_priority(int32_t on);
 /* smc_set_conv_epilogue: where smc_conv_ex applies the activation and the
  *   residual for the tensor-core conv: 0 = a row pass behind the conv, in
  *   row order, with the GroupNorm statistics in the same pass (default;

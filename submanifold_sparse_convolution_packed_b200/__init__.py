@@ -12,5 +12,5 @@ from ._binding import (  # noqa: F401
     EXPORTS, LIB_PATH, Map, SmcError, build_map, clear_cache, conv, kernel_launches, lib,
     NOALLOC_MAX_N, neighbour_map_noalloc, set_conv_variant, set_hash_capacity, set_map_lookup, set_profiling, status, subdivide, group_stats, group_norm,
     downsample, upsample, POOL_MODES, set_conv_epilogue, set_alloc_fail_after, set_wait_limit_ns, set_scan_hold,
-    set_schedule_segment,
+    set_schedule_segment, set_conv_priority,
 )

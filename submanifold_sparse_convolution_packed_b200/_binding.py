@@ -33,6 +33,7 @@ EXPORTS = [
     "smc_set_map_lookup", "smc_map_stream_wait", "smc_subdivide", "smc_conv_ex", "smc_group_stats",
     "smc_group_norm", "smc_downsample", "smc_upsample", "smc_set_conv_epilogue",
     "smc_set_alloc_fail_after", "smc_set_wait_limit_ns", "smc_set_scan_hold", "smc_set_schedule_segment",
+    "smc_set_conv_priority",
 ]
 
 
@@ -88,6 +89,7 @@ def lib() -> ctypes.CDLL:
         L.smc_set_wait_limit_ns.argtypes = [i64]
         L.smc_set_scan_hold.argtypes = [i64]
         L.smc_set_schedule_segment.argtypes = [i64]
+        L.smc_set_conv_priority.argtypes = [i32]
         for name in EXPORTS:
             if name != "smc_strerror":
                 getattr(L, name).restype = ctypes.c_int
@@ -518,6 +520,13 @@ def set_alloc_fail_after(k: int) -> None:
 def set_wait_limit_ns(ns: int) -> None:
     """Bound of the scans' device-side waits, in ns (0 = the default 2 s)."""
     _check(lib().smc_set_wait_limit_ns(int(ns)), "smc_set_wait_limit_ns")
+
+
+def set_conv_priority(on: bool) -> None:
+    """Run convs on the library's high-priority streams, forked from and
+    joined back to the caller's stream (default), or on the caller's stream
+    itself (smc_set_conv_priority)."""
+    _check(lib().smc_set_conv_priority(1 if on else 0), "smc_set_conv_priority")
 
 
 def set_schedule_segment(rows: int) -> None:

@@ -123,6 +123,31 @@ cudaStream_t side_stream(int dev) {
   return g_side[dev];
 }
 
+// Per-device streams of the greatest priority that the convs run on, forked
+// from and joined back to the caller's stream (smc_set_conv_priority): a
+// conv's CTAs are then dispatched before those of map builds and other work
+// queued beside it, e.g. the next step's build on another stream.  Two, used
+// in turn, so that consecutive convs of different callers can overlap.
+constexpr int kPrioStreams = 2;
+cudaStream_t g_prio[kMaxDevices][kPrioStreams] = {};
+std::atomic<uint32_t> g_prio_next[kMaxDevices] = {};
+std::atomic<int32_t> g_conv_priority{1};
+
+cudaStream_t prio_stream(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  const uint32_t k = g_prio_next[dev].fetch_add(1, std::memory_order_relaxed) % kPrioStreams;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_prio[dev][k]) {
+    int lo = 0, hi = 0;
+    if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&g_prio[dev][k], cudaStreamNonBlocking, hi) != cudaSuccess) {
+      cudaGetLastError();
+      g_prio[dev][k] = nullptr;
+    }
+  }
+  return g_prio[dev][k];
+}
+
 // Per-device pool of timing-free events (fork/join points and the maps'
 // completion events), reused instead of created per build.
 std::mutex g_ev_mu;
@@ -602,6 +627,12 @@ int smc_set_map_lookup(int32_t mode) {
   return SMC_OK;
 }
 
+int smc_set_conv_priority(int32_t on) {
+  if (on != 0 && on != 1) return SMC_E_ARG;
+  g_conv_priority.store(on);
+  return SMC_OK;
+}
+
 int smc_set_conv_epilogue(int32_t where) {
   if (where != 0 && where != 1) return SMC_E_ARG;
   smc::set_conv_epilogue(where);
@@ -1025,43 +1056,73 @@ int smc_conv_ex(const smc_map* map, const void* feats, int64_t cin, const void* 
     a.ep.residual = nullptr;
     a.ep.act = SMC_ACT_NONE;
   }
-  cudaError_t e;
-  if (per_offset) {
-    void* acc = nullptr;
-    cudaMemPool_t pool = device_pool(dev);
-    if (pool_alloc(&acc, static_cast<size_t>(n) * cout * sizeof(float), pool, s) != cudaSuccess) {
+  // The conv runs on one of the library's streams of the greatest priority,
+  // forked from the caller's stream and joined back to it (unless
+  // smc_set_conv_priority(0)), so that its CTAs are dispatched before those
+  // of work queued beside it.  Measured on B200 with steps pipelined over two
+  // streams (the next step's map build beside this conv): 6-shell 128^3,
+  // 0.117-0.123 -> 0.112-0.113 ms per step; the large maps even; one step
+  // alone about 2 us longer (the fork and the join).
+  cudaStream_t run = s;
+  if (g_conv_priority.load() != 0) {
+    cudaStream_t hp = prio_stream(dev);
+    cudaEvent_t fork = hp ? take_event(dev) : nullptr;
+    if (fork && cudaEventRecord(fork, s) == cudaSuccess && cudaStreamWaitEvent(hp, fork, 0) == cudaSuccess)
+      run = hp;
+    else
       cudaGetLastError();
-      return SMC_E_OOM;
+    give_event(dev, fork);  // its wait is enqueued
+  }
+  auto launch = [&](cudaStream_t ls) -> int {
+    cudaError_t e;
+    if (per_offset) {
+      void* acc = nullptr;
+      cudaMemPool_t pool = device_pool(dev);
+      if (pool_alloc(&acc, static_cast<size_t>(n) * cout * sizeof(float), pool, ls) != cudaSuccess) {
+        cudaGetLastError();
+        return SMC_E_OOM;
+      }
+      e = smc::launch_conv_offsets(a, static_cast<float*>(acc), ls);
+      cudaFreeAsync(acc, ls);
+    } else {
+      e = tc ? smc::launch_conv_tc(a, ls) : smc::launch_conv_simt(a, ls);
     }
-    e = smc::launch_conv_offsets(a, static_cast<float*>(acc), s);
-    cudaFreeAsync(acc, s);
-  } else {
-    e = tc ? smc::launch_conv_tc(a, s) : smc::launch_conv_simt(a, s);
-  }
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return SMC_E_CUDA;
-  }
-  // Group statistics of the stored output: in the row pass, or a statistics
-  // pass right behind the conv on the same stream (both measured faster than
-  // folding them into the conv's epilogue, see conv_tc.cu).
-  if (pass) {
-    smc::Epilogue ep;
-    ep.batch = map->batch;
-    ep.groups = stats ? groups : 1;
-    ep.stripes = kStatStripes;
-    if (stats) {
-      const int rc = stats_begin(dev, s, map->batch, groups, &ep.stats);
-      if (rc != SMC_OK) return rc;
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return SMC_E_CUDA;
     }
-    e = smc::launch_rows_pass(out, out, residual, act, n, static_cast<int>(cout), coords, ep, dtype, s);
-    if (e != cudaSuccess) cudaGetLastError();
-    const int rc2 = stats ? stats_end(ep.stats, map->batch, groups, stats, s, e == cudaSuccess) : SMC_OK;
-    if (e != cudaSuccess) return SMC_E_CUDA;
-    return rc2;
+    // Group statistics of the stored output: in the row pass, or a statistics
+    // pass right behind the conv on the same stream (both measured faster than
+    // folding them into the conv's epilogue, see conv_tc.cu).
+    if (pass) {
+      smc::Epilogue ep;
+      ep.batch = map->batch;
+      ep.groups = stats ? groups : 1;
+      ep.stripes = kStatStripes;
+      if (stats) {
+        const int rc = stats_begin(dev, ls, map->batch, groups, &ep.stats);
+        if (rc != SMC_OK) return rc;
+      }
+      e = smc::launch_rows_pass(out, out, residual, act, n, static_cast<int>(cout), coords, ep, dtype, ls);
+      if (e != cudaSuccess) cudaGetLastError();
+      const int rc2 = stats ? stats_end(ep.stats, map->batch, groups, stats, ls, e == cudaSuccess) : SMC_OK;
+      if (e != cudaSuccess) return SMC_E_CUDA;
+      return rc2;
+    }
+    if (stats) return smc_group_stats(out, n, cout, coords, map->batch, groups, stats, dtype, ls);
+    return SMC_OK;
+  };
+  int rc = launch(run);
+  if (run != s) {
+    cudaEvent_t join = take_event(dev);
+    if (!join || cudaEventRecord(join, run) != cudaSuccess || cudaStreamWaitEvent(s, join, 0) != cudaSuccess) {
+      cudaGetLastError();
+      cudaStreamSynchronize(run);  // no join event: the caller's stream must not run ahead of the conv
+      if (rc == SMC_OK) rc = SMC_E_CUDA;
+    }
+    give_event(dev, join);
   }
-  if (stats) return smc_group_stats(out, n, cout, coords, map->batch, groups, stats, dtype, stream);
-  return SMC_OK;
+  return rc;
 }
 
 int smc_map_info(const smc_map* map, int64_t* n, int64_t counts[27]) {

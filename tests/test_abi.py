@@ -41,6 +41,8 @@ def test_strerror_without_gpu():
     assert lib.smc_set_conv_variant(0) == 0
     assert lib.smc_set_conv_epilogue(2) == -1
     assert lib.smc_set_conv_epilogue(0) == 0
+    assert lib.smc_set_conv_priority(2) == -1
+    assert lib.smc_set_conv_priority(1) == 0
     assert lib.smc_set_map_lookup(4) == -1
     assert lib.smc_set_map_lookup(3) == 0
     assert lib.smc_set_map_lookup(0) == 0

@@ -485,6 +485,35 @@ def test_conv_variants_agree(name, dtype):
     smc.status()
 
 
+def test_conv_priority_streams_keep_order():
+    """Convs forked to the library's high-priority streams stay ordered on the
+    caller's stream: three stacked layers, each reading the previous output,
+    give the same bits as on the caller's stream itself, on the map's stream
+    and on another one."""
+    w = workload("shell2")
+    f, wt, b = _layer(w, "bf16")
+    results = []
+    for prio in (0, 1):
+        smc.set_conv_priority(bool(prio))
+        try:
+            for other in (False, True):
+                st = torch.cuda.Stream() if other else torch.cuda.current_stream()
+                m = smc.build_map(torch.from_numpy(w.coords).cuda(), w.grid, batch=2, sync=False)
+                x = dev(f, "bf16")
+                with torch.cuda.stream(st):
+                    st.wait_stream(torch.cuda.current_stream())
+                    for _ in range(3):
+                        x = smc.conv(m, x, dev(wt, "bf16"), dev(b, "bf16"), stream=st)
+                st.synchronize()
+                results.append(x.cpu())
+                smc.status(st)
+                m.free()
+        finally:
+            smc.set_conv_priority(True)
+    for r in results[1:]:
+        assert torch.equal(results[0], r)
+
+
 # ------------------------------------------------------------------ epilogue (row pass / in the conv) and GroupNorm
 @pytest.fixture(params=[0, 1], ids=["row_pass", "in_conv"])
 def conv_epilogue(request):
