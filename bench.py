@@ -401,7 +401,8 @@ def input_sets(torch, dev, w, f, tdt, min_sets=2, max_sets=8):
     k = max(min_sets, min(max_sets, -(-3 * L2_BYTES // per)))
     coords = torch.from_numpy(w.coords)
     feats = torch.from_numpy(f).to(tdt)
-    return [(coords.to(dev), feats.to(dev), torch.empty((w.n, w.cout), dtype=tdt, device=dev)) for _ in range(k)]
+    return [(coords.to(dev, copy=True), feats.to(dev, copy=True), torch.empty((w.n, w.cout), dtype=tdt, device=dev))
+            for _ in range(k)]
 
 
 class StepRunner:

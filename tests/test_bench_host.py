@@ -49,3 +49,18 @@ def test_cpu_baseline_record_fields():
 def test_workload_118k_draw():
     w = S.workload("shells6_118k")
     assert w.n == 117818 and w.grid == (128, 128, 128) and w.cin == w.cout == 128
+
+
+def test_input_sets_exceed_l2():
+    """The pipelined steps rotate over copies of their inputs whose total is
+    at least 3x L2 (so no flush is needed), with at least two copies."""
+    import torch
+    w = S.workload("shell2")
+    f, _, _ = S.layer_tensors(w, "bf16")
+    sets = bench.input_sets(torch, torch.device("cpu"), w, f, torch.bfloat16)
+    per = w.n * (16 + 2 * w.cin + 2 * w.cout)
+    assert 2 <= len(sets) <= 8
+    assert len(sets) == 8 or len(sets) * per >= 3 * bench.L2_BYTES
+    c, x, y = sets[0]
+    assert c.shape == (w.n, 4) and x.shape == (w.n, w.cin) and y.shape == (w.n, w.cout)
+    assert all(s[0].data_ptr() != sets[0][0].data_ptr() for s in sets[1:])
