@@ -345,7 +345,7 @@ SMC_API int smc_map_pairs(const smc_map* map, const int32_t** in_idx, const int3
  * none): device pointer to perm[n] (int32), the order in which output rows
  * are grouped into tiles of 128 (a permutation of 0..n-1: rows are stably
  * sorted by which of the 8 corner and 12 edge offsets they hit, or, for maps
- * of at most 131072 rows, by the 8 corners and the first 2 edges alone, so
+ * of at most 131072 rows, by the 8 corners alone, so
  * that each tile skips the offsets none of its rows has).
  */
 SMC_API int smc_map_schedule(const smc_map* map, const int32_t** perm);

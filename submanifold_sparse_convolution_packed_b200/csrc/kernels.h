@@ -63,7 +63,6 @@ void count_launches(int k);
 
 int map_nblocks(int64_t n);
 int radix_nblocks(int64_t n);
-int radix_bins();
 // The tile schedule sorts rows within segments of consecutive input rows
 // (0 = the whole map is one segment).  radix_seg_chunks: 2048-row radix
 // chunks per segment for a map of n rows (the segment length in force now);

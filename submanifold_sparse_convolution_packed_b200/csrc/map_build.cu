@@ -41,8 +41,8 @@ static_assert(kRadixChunk % kMapBlock == 0, "a radix chunk is a whole number of 
 // the segment], cps chunks per segment.  Scanning that layout in order sorts
 // every segment of cps * kRadixChunk consecutive rows on its own and keeps the
 // segments in input order (cps = all chunks: one stable sort of the map).
-__host__ __device__ __forceinline__ int64_t hist_index(uint32_t digit, int64_t chunk, int cps) {
-  return ((chunk / cps) * kRadixBins + digit) * cps + chunk % cps;
+__host__ __device__ __forceinline__ int64_t hist_index(uint32_t digit, int64_t chunk, int cps, int bins) {
+  return ((chunk / cps) * bins + digit) * cps + chunk % cps;
 }
 constexpr uint64_t kFib = 0x9E3779B97F4A7C15ull;
 
@@ -162,14 +162,21 @@ __device__ __forceinline__ uint32_t key_hits(uint32_t k) {
 }
 
 // Maps of at most kOnePassRows rows get a one-pass tile schedule: a stable
-// sort on the high 10 bits of the key (the 8 corner and 2 edge offsets).  For
-// them the schedule's launches are latency-bound and a second pass costs more
+// sort on the high 8 bits of the key (the 8 corner offsets), 256 bins.  For
+// them the schedule's launches are latency-bound: a second pass costs more
 // (a look-back scan and a scatter, about 20 us on B200) than the conv gains
-// from the finer grouping (tap efficiency 0.855 vs 0.882 on the 6-shell
-// 128^3 workload, a 2% longer conv).
+// from the finer grouping (tap efficiency 0.855 with 10 bits and 0.882 with
+// all 20 on the 6-shell 128^3 workload), and 256 bins instead of 1024 cut
+// the scatter's per-block work (its digit table and offsets) by four for a
+// tap efficiency of 0.846.
 constexpr int64_t kOnePassRows = 131072;
-
+constexpr int kOnePassBits = 8;
+constexpr int kOnePassBins = 1 << kOnePassBits;
 __host__ __device__ __forceinline__ bool schedule_one_pass(int64_t n) { return n <= kOnePassRows; }
+// Radix bins of a map's first (or only) schedule pass.
+__host__ __device__ __forceinline__ int schedule_bins(int64_t n) {
+  return schedule_one_pass(n) ? kOnePassBins : kRadixBins;
+}
 
 // Schedule segments are whole radix chunks (see set_schedule_segment_rows).
 static_assert(kScheduleSegmentDefault % kRadixChunk == 0, "segments are whole radix chunks");
@@ -187,11 +194,13 @@ __device__ __forceinline__ void emit_map_block(const int32_t* s_nbr, int32_t (*s
   if (hist1) {
     // the digit of the schedule's first pass: the low 10 bits, or the high
     // 10 for a map sorted in one pass
-    const int shift = schedule_one_pass(n) ? kRadixBits : 0;
-    const uint32_t digit = v < n ? ((gk >> shift) & (kRadixBins - 1)) : 0xFFFFFFFFu;
+    const bool one = schedule_one_pass(n);
+    const int shift = one ? 2 * kRadixBits - kOnePassBits : 0;
+    const int bins = one ? kOnePassBins : kRadixBins;
+    const uint32_t digit = v < n ? ((gk >> shift) & static_cast<uint32_t>(bins - 1)) : 0xFFFFFFFFu;
     const uint32_t peers = __match_any_sync(0xffffffffu, digit);
     if (v < n && (__ffs(peers) - 1) == lane)
-      atomicAdd(&hist1[hist_index(digit, base / kRadixChunk, radix_cps)], __popc(peers));
+      atomicAdd(&hist1[hist_index(digit, base / kRadixChunk, radix_cps, bins)], __popc(peers));
   }
 #pragma unroll
   for (int d = 0; d < kTaps; ++d) {
@@ -733,16 +742,16 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_lookback(const int32_t* _
 // First pass (kLast false): writes keys and row indices and counts the next
 // digit per destination chunk into hist_next.  Last pass: writes the row
 // order and ORs each row's hit mask into the mask of its 128-row tile.
-template <bool kLast>
+template <bool kLast, int kBins>
 __global__ void __launch_bounds__(kRadixThreads) k_radix_scatter(
     const uint32_t* __restrict__ keys_in, const int32_t* __restrict__ vals_in, int64_t n, int shift,
     const int64_t* __restrict__ offsets, int cps, uint32_t* __restrict__ keys_out,
     int32_t* __restrict__ vals_out, int32_t* __restrict__ hist_next, uint32_t* __restrict__ tile_mask,
     uint32_t* err) {
   constexpr int kWarps = kRadixThreads / 32;
-  __shared__ int32_t s_cnt[kWarps][kRadixBins];  // counts, then positions (< n < 2^31)
+  __shared__ int32_t s_cnt[kWarps][kBins];  // counts, then positions (< n < 2^31)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int i = tid; i < kWarps * kRadixBins; i += kRadixThreads) (&s_cnt[0][0])[i] = 0;
+  for (int i = tid; i < kWarps * kBins; i += kRadixThreads) (&s_cnt[0][0])[i] = 0;
   const int64_t w0 = static_cast<int64_t>(blockIdx.x) * kRadixChunk + warp * (kRadixRounds * 32);
   const uint32_t lt = (1u << lane) - 1u;
   uint32_t keys[kRadixRounds];
@@ -758,7 +767,7 @@ __global__ void __launch_bounds__(kRadixThreads) k_radix_scatter(
 #pragma unroll
   for (int round = 0; round < kRadixRounds; ++round) {
     const bool valid = w0 + round * 32 + lane < n;
-    const uint32_t digit = (keys[round] >> shift) & (kRadixBins - 1);
+    const uint32_t digit = (keys[round] >> shift) & (kBins - 1);
     const uint32_t peers = __match_any_sync(0xffffffffu, valid ? digit : 0xFFFFFFFFu);
     const int32_t before = valid ? my[digit] : 0;
     rank[round] = before + __popc(peers & lt);
@@ -767,8 +776,8 @@ __global__ void __launch_bounds__(kRadixThreads) k_radix_scatter(
     __syncwarp();
   }
   __syncthreads();
-  for (int d = tid; d < kRadixBins; d += kRadixThreads) {
-    int64_t run = offsets[hist_index(static_cast<uint32_t>(d), blockIdx.x, cps)];
+  for (int d = tid; d < kBins; d += kRadixThreads) {
+    int64_t run = offsets[hist_index(static_cast<uint32_t>(d), blockIdx.x, cps, kBins)];
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
       const int32_t c = s_cnt[w][d];
@@ -781,7 +790,7 @@ __global__ void __launch_bounds__(kRadixThreads) k_radix_scatter(
   for (int round = 0; round < kRadixRounds; ++round) {
     const bool valid = w0 + round * 32 + lane < n;
     const uint32_t key = keys[round];
-    const uint32_t digit = (key >> shift) & (kRadixBins - 1);
+    const uint32_t digit = (key >> shift) & (kBins - 1);
     long long pos = -1;
     if (valid) {
       pos = static_cast<long long>(my[digit]) + rank[round];
@@ -801,7 +810,7 @@ __global__ void __launch_bounds__(kRadixThreads) k_radix_scatter(
                                     : 0xFFFFFFFFu;
       const uint32_t grp = __match_any_sync(0xffffffffu, tag);
       if (tag != 0xFFFFFFFFu && (__ffs(grp) - 1) == lane)
-        atomicAdd(&hist_next[hist_index(tag >> 21, tag & ((1u << 21) - 1), cps)], __popc(grp));
+        atomicAdd(&hist_next[hist_index(tag >> 21, tag & ((1u << 21) - 1), cps, kRadixBins)], __popc(grp));
     } else {
       // tile tap masks: a warp whose rows all land in one tile (dense data)
       // ORs them first; otherwise every row ORs its own mask in
@@ -833,7 +842,6 @@ static cudaError_t scan_i32(const int32_t* in, int64_t L, int64_t* out, unsigned
 int64_t scan_status_len(int64_t L) { return (L + kScanSeg - 1) / kScanSeg; }
 int map_nblocks(int64_t n) { return static_cast<int>((n + kMapBlock - 1) / kMapBlock); }
 int radix_nblocks(int64_t n) { return static_cast<int>((n + kRadixChunk - 1) / kRadixChunk); }
-int radix_bins() { return kRadixBins; }
 
 // Schedule segment length in rows (0 = one segment, the default).  Segments
 // keep the rows of each wave of conv tiles within a window of consecutive
@@ -857,7 +865,7 @@ int radix_seg_chunks(int64_t n) {
 int64_t radix_hist_len(int64_t n, int cps) {
   const int64_t nblk = radix_nblocks(n);
   const int64_t nseg = (nblk + cps - 1) / cps;
-  return nseg * cps * kRadixBins;
+  return nseg * cps * schedule_bins(n);
 }
 
 cudaError_t launch_map_lookups(const MapBuildArgs& a, cudaStream_t s) {
@@ -963,25 +971,25 @@ cudaError_t launch_schedule(const ScheduleArgs& a, cudaStream_t s) {
   const int cps = a.radix_cps;
   const int64_t L = radix_hist_len(n, cps);
   if (schedule_one_pass(n)) {
-    // small maps: one stable pass on the high 10 bits (the 8 corner and 2 edge
-    // offsets); the histogram of that digit comes from the neighbour kernel
+    // small maps: one stable pass on the high 8 bits (the 8 corner offsets);
+    // the histogram of that digit comes from the neighbour kernel
     cudaError_t e = scan_i32(a.hist1, L, a.hoff, a.status1, a.tickets, a.err, nullptr, 1, s);
     if (e != cudaSuccess) return e;
-    k_radix_scatter<true><<<nblk, kRadixThreads, 0, s>>>(a.gkey, nullptr, n, kRadixBits, a.hoff, cps, nullptr,
-                                                         a.perm, nullptr, a.tile_mask, a.err);
+    k_radix_scatter<true, kOnePassBins><<<nblk, kRadixThreads, 0, s>>>(
+        a.gkey, nullptr, n, 2 * kRadixBits - kOnePassBits, a.hoff, cps, nullptr, a.perm, nullptr, a.tile_mask, a.err);
     count_launches(1);
     return cudaGetLastError();
   }
   // pass 1: low 10 bits, rows in input order (histogram from the neighbour kernel)
   cudaError_t e = scan_i32(a.hist1, L, a.hoff, a.status1, a.tickets, a.err, nullptr, 1, s);
   if (e != cudaSuccess) return e;
-  k_radix_scatter<false><<<nblk, kRadixThreads, 0, s>>>(a.gkey, nullptr, n, 0, a.hoff, cps, a.key_tmp,
+  k_radix_scatter<false, kRadixBins><<<nblk, kRadixThreads, 0, s>>>(a.gkey, nullptr, n, 0, a.hoff, cps, a.key_tmp,
                                                         a.val_tmp, a.hist2, nullptr, a.err);
   count_launches(1);
   // pass 2: high 10 bits
   e = scan_i32(a.hist2, L, a.hoff, a.status2, a.tickets + 1, a.err, nullptr, 1, s);
   if (e != cudaSuccess) return e;
-  k_radix_scatter<true><<<nblk, kRadixThreads, 0, s>>>(a.key_tmp, a.val_tmp, n, kRadixBits, a.hoff, cps,
+  k_radix_scatter<true, kRadixBins><<<nblk, kRadixThreads, 0, s>>>(a.key_tmp, a.val_tmp, n, kRadixBits, a.hoff, cps,
                                                        nullptr, a.perm, nullptr, a.tile_mask, a.err);
   count_launches(1);
   return cudaGetLastError();

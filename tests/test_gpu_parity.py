@@ -92,7 +92,7 @@ def map_lookup(request):
 # The tile order of the tensor-core conv: rows stably sorted by a 20-bit key
 # whose bits, most significant first, say whether the 8 corner offsets and
 # then the 12 edge offsets have a neighbour; maps of at most ONE_PASS_ROWS
-# rows are sorted on the key's high 10 bits alone (one radix pass).  The sort
+# rows are sorted on the key's high 8 bits alone, the corners (one radix pass).  The sort
 # runs within segments of SEGMENT_ROWS consecutive input rows, the segments
 # kept in input order (0: the whole map is one segment).
 _KEY_TAPS = [0, 2, 6, 8, 18, 20, 24, 26, 1, 3, 5, 7, 9, 11, 15, 17, 19, 21, 23, 25]
@@ -106,7 +106,7 @@ def expected_schedule(nbr, segment=SEGMENT_ROWS):
     for i, d in enumerate(_KEY_TAPS):
         key |= (nbr[:, d] >= 0).astype(np.int64) << (19 - i)
     if n <= ONE_PASS_ROWS:
-        key >>= 10
+        key >>= 12
     if segment:
         key |= (np.arange(n, dtype=np.int64) // segment) << 20
     return np.argsort(key, kind="stable").astype(np.int32)
