@@ -552,13 +552,13 @@ def measure_config(smc, torch, stream, flush, dev, peaks, name, dtype, steps, wo
     latency = float(np.median(lat.times))
     # throughput: pipelined steps, at least 0.3 s of them
     prime_pool(smc, sets, w.grid, batch, streams, StepRunner.DEPTH * len(streams) + 2)
+    clocks = ClockSampler(dev.index or 0)
+    clocks.start()
     warm = mk(streams, None)
     for _ in range(2 * StepRunner.DEPTH):
         warm.submit()
     warm.drain()
     n_steps = max(steps, int(0.3 / (latency * 1e-3)))
-    clocks = ClockSampler(dev.index or 0)
-    clocks.start()
     clocks.mark()
     run = mk(streams, None)
     total = timed_steps(torch, run, n_steps)
@@ -646,24 +646,26 @@ def run_gpu(args):
     smc.set_profiling(False)  # the timed steps carry no instrumentation
 
     prime_pool(smc, sets, w.grid, batch, streams, StepRunner.DEPTH * len(streams) + 2)
+    # reference of the schedule quality (host-side, untimed)
+    m0 = smc.build_map(coords_d, w.grid, batch=batch, stream=stream)
+    P = m0.pairs_total
+    eff = tap_efficiency(m0.schedule().cpu().numpy(), m0.nbr().cpu().numpy())
+    m0.free()
+    # the clock sampler starts before the warm-up, so that the timed region
+    # follows the warm-up steps directly (only its own samples are reported)
+    clocks = ClockSampler(local)
+    clocks.start()
     # warm-up: W pipelined steps
     warm = runner(streams, None)
     for _ in range(args.warmup):
         warm.submit()
     warm.drain()
     smc.status(stream)
-    # reference of the schedule quality (host-side, untimed)
-    m0 = smc.build_map(coords_d, w.grid, batch=batch, stream=stream)
-    P = m0.pairs_total
-    eff = tap_efficiency(m0.schedule().cpu().numpy(), m0.nbr().cpu().numpy())
-    m0.free()
 
     # the timed region: K steps, alternating over the streams, each on the
     # next copy of the inputs (together more than 3x L2, so no flush)
-    clocks = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize()
-    clocks.start()
     clocks.mark()
     t_wall0 = time.perf_counter()
     launches_before = smc.kernel_launches()
