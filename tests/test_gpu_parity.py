@@ -436,10 +436,13 @@ def test_conv_small_integers_bit_exact(oracle_mod, dtype, orientation, conv_vari
     np.testing.assert_array_equal(got, ref)
 
 
-@pytest.mark.parametrize("cin,cout", [(64, 16), (64, 512), (96, 48), (48, 64), (200, 24), (128, 272)])
+@pytest.mark.parametrize("cin,cout", [(64, 16), (64, 512), (96, 48), (48, 64), (200, 24), (128, 272), (96, 64),
+                                      (160, 128)])
 def test_conv_channel_shapes_bf16(oracle_mod, cin, cout, conv_variant):
     """Tensor-core path with ragged K blocks, narrow and split N tiles; shapes
-    outside its limits run on the FMA kernel; all must meet the same bar."""
+    outside its limits run on the FMA kernel; all must meet the same bar.
+    (96, 64) and (160, 128) take ragged K blocks through the two-tile kernel
+    (the default at 64 output channels, the forced variant at 128)."""
     w = workload("shell2")
     m = build(w)
     f, wt, b = _layer(w, "bf16", 7, 3, cin, cout)
