@@ -393,9 +393,9 @@ SMC_API const char* smc_strerror(int code);
  *   has at most 2^28 sites and at most 256 sites per voxel -- cleared at
  *   every build when it has at most 2^23 sites and fewer than 16 per voxel,
  *   else left uncleared behind a cleared occupancy bitmap of one bit per
- *   site -- else a hash table), 1 = hash
- *   table, 2 = cleared dense grid and 3 = dense grid with occupancy bitmap,
- *   each whenever the box has at most 2^28 sites.  Maps are identical either way.  A forced hash capacity
+ *   site -- else a hash table), 1 = hash table, 2 = cleared dense grid and
+ *   3 = dense grid with occupancy bitmap, each whenever the box has at most
+ *   2^28 sites.  Maps are identical either way.  A forced hash capacity
  *   (smc_set_hash_capacity) always selects the hash table.  SMC_E_ARG for
  *   any other value.
  * smc_set_conv_variant: tensor-core conv kernel for later convs (bf16/fp16
@@ -438,8 +438,8 @@ SMC_API const char* smc_strerror(int code);
  * device address (cudaGetSymbolAddress) with that device current and caches
  * it with the device's current context; make that first call before any
  * stream capture.  After cudaDeviceReset (a new context) the next call looks
- * the address up again, so it too should come before any capture.  Every call shares the
- * array and clears what it reads; calls whose work overlaps on the GPU
+ * the address up again, so it too should come before any capture.  Every
+ * call shares the array and clears what it reads; calls whose work overlaps on the GPU
  * (different streams or host threads) race on it and must be serialised by
  * the caller.  No pair lists or tile schedule are produced.
  */
@@ -468,8 +468,8 @@ SMC_API int smc_set_conv_priority(int32_t on);
  *   measured faster; a residual that is the output buffer itself always
  *   goes through the epilogue), 1 = in the conv's own epilogue.  Results
  *   agree to rounding: the row pass sees the conv's stored (rounded) output,
- *   as a separate activation layer would.  Used to test and measure the two.  SMC_E_ARG for any other
- *   value. */
+ *   as a separate activation layer would.  Used to test and measure the
+ *   two.  SMC_E_ARG for any other value. */
 SMC_API int smc_set_conv_epilogue(int32_t where);
 SMC_API int smc_set_map_lookup(int32_t mode);
 
